@@ -1,0 +1,136 @@
+"""CPU oracle for the compressed-tensor decoders -- TEST INFRASTRUCTURE ONLY.
+
+Plain, slow, element-by-element statement of what the on-device decoders
+compute (``lt_oracle.c``, plain C, built in-tree as ``liblt_oracle.so``).
+Only the test suite, the smoke check and the benchmark's CPU-baseline leg
+may use it; the product path never does, and it shares no code with the CUDA
+library. Every function here is a ctypes marshalling shim over one C
+function; the arithmetic lives in the C file, which cites its sources.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(_HERE, "lt_oracle.c")
+LIB = os.path.join(_HERE, "liblt_oracle.so")
+
+OK, INVALID, CORRUPT, SIZE_MISMATCH = 0, 1, 4, 5
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``lt_oracle.c`` (gcc, -O2, no fast-math)."""
+    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
+        return LIB
+    tmp = LIB + ".tmp"
+    subprocess.run(["gcc", "-O2", "-std=gnu11", "-fPIC", "-shared", "-fvisibility=hidden",
+                    "-fno-fast-math", SRC, "-o", tmp, "-lm"], check=True)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(LIB)
+        P, I64, U64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint64, ctypes.c_int
+        lib.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
+        lib.oracle_f16_to_f64.restype = ctypes.c_double
+        lib.oracle_f16_from_f64.argtypes = [ctypes.c_double]
+        lib.oracle_f16_from_f64.restype = ctypes.c_uint16
+        lib.oracle_f16_from_f64_array.argtypes = [P, I64, P]
+        lib.oracle_f16_to_f64_array.argtypes = [P, I64, P]
+        lib.oracle_dequant_int4.argtypes = [P, P, P, I64, I64, I64, P]
+        lib.oracle_dequant_int8.argtypes = [P, P, P, I32, I64, I64, P]
+        lib.oracle_zrle_decode.argtypes = [P, U64, P, I64, I64, P]
+        lib.oracle_lz4_block_decode.argtypes = [P, U64, P, U64]
+        lib.oracle_lz4_decode_blocks.argtypes = [P, U64, P, I64, P, U64]
+        lib.oracle_lz4_int4_decode.argtypes = [P, U64, P, I64, P, P, I64, I64, I64, P]
+        for f in ("oracle_dequant_int4", "oracle_dequant_int8", "oracle_zrle_decode",
+                  "oracle_lz4_block_decode", "oracle_lz4_decode_blocks", "oracle_lz4_int4_decode"):
+            getattr(lib, f).restype = I32
+        _lib = lib
+    return _lib
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data
+
+
+def f16_from_f64(x) -> np.ndarray:
+    """Round doubles to fp16 bit patterns (RNE), own implementation."""
+    x = _c(np.atleast_1d(x), np.float64)
+    out = np.zeros(x.size, dtype=np.uint16)
+    _load().oracle_f16_from_f64_array(_p(x), x.size, _p(out))
+    return out
+
+
+def f16_to_f64(h) -> np.ndarray:
+    h = _c(np.atleast_1d(h), np.uint16)
+    out = np.zeros(h.size, dtype=np.float64)
+    _load().oracle_f16_to_f64_array(_p(h), h.size, _p(out))
+    return out
+
+
+def dequant_int4(packed, scales, zeros, rows: int, cols: int, group_size: int):
+    """Returns (fp16 bits as uint16 [rows*cols], status)."""
+    packed = _c(packed, np.uint8)
+    scales = _c(scales, np.uint16)
+    zeros = None if zeros is None else _c(zeros, np.uint8)
+    out = np.zeros(rows * cols, dtype=np.uint16)
+    st = _load().oracle_dequant_int4(_p(packed), _p(scales), _p(zeros), rows, cols, group_size, _p(out))
+    return out, st
+
+
+def dequant_int8(q, scales, zeros, per_row: bool, rows: int, cols: int):
+    q = _c(q, np.int8)
+    scales = _c(scales, np.uint16)
+    zeros = None if zeros is None else _c(zeros, np.int8)
+    out = np.zeros(rows * cols, dtype=np.uint16)
+    st = _load().oracle_dequant_int8(_p(q), _p(scales), _p(zeros), int(per_row), rows, cols, _p(out))
+    return out, st
+
+
+def zrle_decode(enc, offsets, n: int, chunk_elems: int):
+    enc = _c(enc, np.uint8)
+    offsets = _c(offsets, np.uint64)
+    out = np.zeros(n, dtype=np.uint16)
+    st = _load().oracle_zrle_decode(_p(enc), enc.size, _p(offsets), n, chunk_elems, _p(out))
+    return out, st
+
+
+def lz4_block_decode(src, dst_len: int):
+    src = _c(np.frombuffer(bytes(src), np.uint8) if not isinstance(src, np.ndarray) else src, np.uint8)
+    out = np.zeros(max(dst_len, 1), dtype=np.uint8)
+    st = _load().oracle_lz4_block_decode(_p(src), src.size, _p(out), dst_len)
+    return out[:dst_len], st
+
+
+def lz4_decode_blocks(comp, offsets, block_bytes: int, dst_len: int):
+    comp = _c(comp, np.uint8)
+    offsets = _c(offsets, np.uint64)
+    out = np.zeros(max(dst_len, 1), dtype=np.uint8)
+    st = _load().oracle_lz4_decode_blocks(_p(comp), comp.size, _p(offsets), block_bytes, _p(out), dst_len)
+    return out[:dst_len], st
+
+
+def lz4_int4_decode(comp, offsets, block_bytes: int, scales, zeros, rows: int, cols: int, group_size: int):
+    comp = _c(comp, np.uint8)
+    offsets = _c(offsets, np.uint64)
+    scales = _c(scales, np.uint16)
+    zeros = None if zeros is None else _c(zeros, np.uint8)
+    out = np.zeros(rows * cols, dtype=np.uint16)
+    st = _load().oracle_lz4_int4_decode(_p(comp), comp.size, _p(offsets), block_bytes, _p(scales), _p(zeros),
+                                        rows, cols, group_size, _p(out))
+    return out, st

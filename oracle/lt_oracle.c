@@ -1,0 +1,308 @@
+/*
+ * lt_oracle.c -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, element-by-element CPU statement of what the on-device
+ * decoders compute. It exists so that the CUDA library can be checked
+ * against it; no product code path may call, link or load it. It shares no
+ * code, header, table or constant generator with the CUDA library or with
+ * the input generator; only the bytes those produce pass through it.
+ *
+ * Sources it follows (web pages, cited by title and section):
+ *   [R]  "GPU Compression Pipeline - TDD Roadmap" (abaddon docs):
+ *        Phase 1.1 INT4 Dequantization (test_int4_dequant_basic: packed
+ *        [0x10,0x32,0x54,0x76] are codes 0..7, low nibble first; scale f16,
+ *        zero point; "block-level dequantization (GPTQ/AWQ compatible)"),
+ *        Phase 1.2 INT8 Dequantization ("Expected: values * scale";
+ *        per-tensor and per-channel scales), Phase 2.1 LZ4 + INT4 Fused
+ *        Kernel (cpu_lz4_decompress_then_dequant: decompress, then
+ *        dequantize), Phase 3.1 (64 KB LZ4 blocks), Phase 6.1 (block_size
+ *        65536).
+ *   [L]  "LoreToken-powered GPU memory layer" (freemwiki ChatGPT export):
+ *        compression strategies, "Zero-run encoding - extremely effective on
+ *        ReLU activations that are mostly zero".
+ *   LZ4 block format: the public description of the LZ4 block layout
+ *        (token, literal run, 2-byte little-endian offset, match length
+ *        with minimum 4, 255-continuation length bytes, literal-only last
+ *        sequence). The pages name LZ4 but do not restate its format.
+ *   IEEE 754-2008 binary16 for the fp16 encoding and round-to-nearest-even.
+ *
+ * Readings where the pages are silent (each stated again in the design
+ * notes): the dequantized value is (q - z) * s with one rounding to fp16
+ * (round to nearest, ties to even, subnormals kept, overflow to infinity);
+ * groups run along the contiguous row of a row-major [rows, cols] tensor;
+ * per-channel means per row; the zero-run chunk format is the
+ * (u16 zero run, u16 literal count, fp16 literals)* record list with
+ * little-endian fields.
+ *
+ * Status values returned: 0 ok, 4 corrupt stream, 5 decoded size differs
+ * from the declared size, 1 invalid argument.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_EXPORT __attribute__((visibility("default")))
+
+enum { ORACLE_OK = 0, ORACLE_INVALID = 1, ORACLE_CORRUPT = 4, ORACLE_SIZE = 5 };
+
+/* ------------------------------------------------------------------ */
+/* IEEE 754 binary16                                                   */
+/* ------------------------------------------------------------------ */
+
+/* binary16 bits -> exact double value. Layout: 1 sign bit, 5 exponent bits
+ * (bias 15), 10 fraction bits; exponent 0 is zero/subnormal (f * 2^-24),
+ * exponent 31 is infinity (f == 0) or NaN. */
+ORACLE_EXPORT double oracle_f16_to_f64(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int e = (h >> 10) & 0x1F;
+  int f = h & 0x3FF;
+  double v;
+  if (e == 0) {
+    v = ldexp((double)f, -24);
+  } else if (e == 31) {
+    v = f ? NAN : INFINITY;
+  } else {
+    v = ldexp((double)(1024 + f), e - 25);
+  }
+  return sign ? -v : v;
+}
+
+/* double -> binary16 bits, round to nearest, ties to even.
+ * Method: the representable binary16 values near |x| are the integer
+ * multiples of the quantum 2^(max(E, -14) - 10), E = floor(log2 |x|); round
+ * |x| / quantum to the nearest integer (ties to the even integer), which is
+ * exact arithmetic in double, then encode that multiple. Results at or above
+ * 2^16 are infinity (the largest finite value is 65504). NaN becomes the
+ * quiet NaN 0x7E00 with the input's sign. */
+ORACLE_EXPORT uint16_t oracle_f16_from_f64(double x) {
+  uint16_t sign = signbit(x) ? 0x8000 : 0;
+  if (isnan(x)) return (uint16_t)(sign | 0x7E00);
+  double a = fabs(x);
+  if (isinf(a)) return (uint16_t)(sign | 0x7C00);
+  if (a == 0.0) return sign;
+  int e2;
+  frexp(a, &e2); /* a = m * 2^e2, m in [0.5, 1) -> floor(log2 a) = e2 - 1 */
+  int E = e2 - 1;
+  if (E < -14) E = -14; /* subnormal range: fixed quantum 2^-24 */
+  double quantum = ldexp(1.0, E - 10);
+  double k = a / quantum; /* exact: division by a power of two */
+  double kf = floor(k);
+  double rem = k - kf;
+  if (rem > 0.5 || (rem == 0.5 && fmod(kf, 2.0) != 0.0)) kf += 1.0;
+  double v = kf * quantum; /* the rounded magnitude */
+  if (v >= 65536.0) return (uint16_t)(sign | 0x7C00);
+  if (v < ldexp(1.0, -14)) {
+    /* subnormal (or +-0): fraction = v / 2^-24 */
+    return (uint16_t)(sign | (uint16_t)ldexp(v, 24));
+  }
+  int ev2;
+  double m = frexp(v, &ev2); /* v = m * 2^ev2, m in [0.5, 1) */
+  int exp_field = (ev2 - 1) + 15;
+  uint16_t frac = (uint16_t)(ldexp(m, 11) - 1024.0); /* (2m - 1) * 1024 */
+  return (uint16_t)(sign | (uint16_t)(exp_field << 10) | frac);
+}
+
+ORACLE_EXPORT void oracle_f16_from_f64_array(const double *x, int64_t n, uint16_t *out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_f16_from_f64(x[i]);
+}
+
+ORACLE_EXPORT void oracle_f16_to_f64_array(const uint16_t *h, int64_t n, double *out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_f16_to_f64(h[i]);
+}
+
+/* ------------------------------------------------------------------ */
+/* INT4 group dequantization   [R] Phase 1.1                          */
+/* ------------------------------------------------------------------ */
+
+/* Code k of the packed array: byte k/2, low nibble for even k, high nibble
+ * for odd k (the worked example lists [0x10,0x32,0x54,0x76] as 0..7). */
+static int int4_code(const uint8_t *packed, int64_t k) {
+  uint8_t b = packed[k / 2];
+  return (k % 2 == 0) ? (b & 0x0F) : (b >> 4);
+}
+
+/* out[r, c] = fp16_rn((q[r, c] - z[g]) * s[g]), g = r * (cols / G) + c / G:
+ * groups of G consecutive codes along each row of a row-major
+ * [rows, cols] tensor. zeros == NULL means zero point 0. */
+ORACLE_EXPORT int oracle_dequant_int4(const uint8_t *packed, const uint16_t *scales, const uint8_t *zeros,
+                                      int64_t rows, int64_t cols, int64_t group_size, uint16_t *out) {
+  if (rows < 0 || cols < 0 || group_size < 1 || (cols % group_size) != 0) return ORACLE_INVALID;
+  int64_t groups_per_row = cols / group_size;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t c = 0; c < cols; ++c) {
+      int64_t k = r * cols + c;
+      int64_t g = r * groups_per_row + c / group_size;
+      int q = int4_code(packed, k);
+      int z = zeros ? zeros[g] : 0;
+      double s = oracle_f16_to_f64(scales[g]);
+      out[k] = oracle_f16_from_f64((double)(q - z) * s);
+    }
+  }
+  return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* INT8 dequantization   [R] Phase 1.2                                 */
+/* ------------------------------------------------------------------ */
+
+/* per_row == 0: one scale (and zero point) for the tensor;
+ * per_row == 1: one per row (output channel).
+ * out[r, c] = fp16_rn((q[r, c] - z) * s). zeros == NULL means 0. */
+ORACLE_EXPORT int oracle_dequant_int8(const int8_t *q, const uint16_t *scales, const int8_t *zeros, int per_row,
+                                      int64_t rows, int64_t cols, uint16_t *out) {
+  if (rows < 0 || cols < 0 || (per_row != 0 && per_row != 1)) return ORACLE_INVALID;
+  for (int64_t r = 0; r < rows; ++r) {
+    int64_t i = per_row ? r : 0;
+    double s = oracle_f16_to_f64(scales[i]);
+    int z = zeros ? zeros[i] : 0;
+    for (int64_t c = 0; c < cols; ++c) {
+      int64_t k = r * cols + c;
+      out[k] = oracle_f16_from_f64((double)((int)q[k] - z) * s);
+    }
+  }
+  return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Zero-run decoding   [L] compression strategies                      */
+/* ------------------------------------------------------------------ */
+
+static unsigned rd_u16le(const uint8_t *p) { return (unsigned)p[0] | ((unsigned)p[1] << 8); }
+
+/* Chunk c covers elements [c * chunk_elems, min(n, (c + 1) * chunk_elems)).
+ * Its bytes are enc[offsets[c], offsets[c + 1]), a list of records
+ * (u16 zero_run, u16 literal_count, literal_count fp16 bit patterns).
+ * Each record emits zero_run elements equal to +0 (0x0000) and then the
+ * literals as they are. Decoding stops once the chunk is full; remaining
+ * bytes are padding. A record that would overrun the chunk, or a record
+ * that does not fit in the chunk's bytes, is a corrupt stream; running out
+ * of bytes before the chunk is full is a size mismatch. */
+ORACLE_EXPORT int oracle_zrle_decode(const uint8_t *enc, uint64_t enc_bytes, const uint64_t *offsets, int64_t n,
+                                     int64_t chunk_elems, uint16_t *out) {
+  if (n < 0 || chunk_elems < 1) return ORACLE_INVALID;
+  int status = ORACLE_OK;
+  int64_t n_chunks = (n + chunk_elems - 1) / chunk_elems;
+  for (int64_t c = 0; c < n_chunks; ++c) {
+    int64_t e0 = c * chunk_elems;
+    int64_t len = n - e0 < chunk_elems ? n - e0 : chunk_elems;
+    for (int64_t i = 0; i < len; ++i) out[e0 + i] = 0;
+    uint64_t b0 = offsets[c], b1 = offsets[c + 1];
+    if (b1 < b0 || b1 > enc_bytes) {
+      if (!status) status = ORACLE_CORRUPT;
+      continue;
+    }
+    uint64_t p = b0;
+    int64_t done = 0;
+    while (done < len) {
+      if (p + 4 > b1) {
+        if (!status) status = ORACLE_SIZE;
+        break;
+      }
+      int64_t zrun = rd_u16le(enc + p);
+      int64_t nlit = rd_u16le(enc + p + 2);
+      p += 4;
+      if (done + zrun + nlit > len || p + 2 * (uint64_t)nlit > b1) {
+        if (!status) status = ORACLE_CORRUPT;
+        break;
+      }
+      for (int64_t i = 0; i < zrun; ++i) out[e0 + done + i] = 0;
+      done += zrun;
+      for (int64_t i = 0; i < nlit; ++i) out[e0 + done + i] = (uint16_t)rd_u16le(enc + p + 2 * i);
+      done += nlit;
+      p += 2 * (uint64_t)nlit;
+    }
+  }
+  return status;
+}
+
+/* ------------------------------------------------------------------ */
+/* LZ4 block decoding   (public LZ4 block format; [R] Phases 2.1, 3.1) */
+/* ------------------------------------------------------------------ */
+
+/* Decode one raw LZ4 block src[0, src_len) into dst, which must come out
+ * exactly dst_len bytes long. Sequence: token; literal count = high nibble,
+ * extended by following bytes while they are 255 (the first byte below 255
+ * ends it) when the nibble is 15; the literals; unless the input ends right
+ * after the literals: 2-byte little-endian offset (1..65535, not beyond the
+ * bytes already produced), match length = low nibble + 4, extended the same
+ * way; the match copies byte by byte from dst[pos - offset], so an offset
+ * smaller than the length repeats the last `offset` bytes. */
+ORACLE_EXPORT int oracle_lz4_block_decode(const uint8_t *src, uint64_t src_len, uint8_t *dst, uint64_t dst_len) {
+  uint64_t ip = 0, op = 0;
+  if (src_len == 0) return dst_len == 0 ? ORACLE_OK : ORACLE_SIZE;
+  for (;;) {
+    if (ip >= src_len) return ORACLE_CORRUPT;
+    unsigned token = src[ip++];
+    uint64_t lit = token >> 4;
+    if (lit == 15) {
+      unsigned b;
+      do {
+        if (ip >= src_len) return ORACLE_CORRUPT;
+        b = src[ip++];
+        lit += b;
+      } while (b == 255);
+    }
+    if (ip + lit > src_len) return ORACLE_CORRUPT;
+    if (op + lit > dst_len) return ORACLE_CORRUPT;
+    for (uint64_t i = 0; i < lit; ++i) dst[op + i] = src[ip + i];
+    ip += lit;
+    op += lit;
+    if (ip == src_len) break; /* the last sequence holds literals only */
+    if (ip + 2 > src_len) return ORACLE_CORRUPT;
+    uint64_t off = (uint64_t)src[ip] | ((uint64_t)src[ip + 1] << 8);
+    ip += 2;
+    if (off == 0 || off > op) return ORACLE_CORRUPT;
+    uint64_t mlen = (token & 0x0F) + 4;
+    if ((token & 0x0F) == 15) {
+      unsigned b;
+      do {
+        if (ip >= src_len) return ORACLE_CORRUPT;
+        b = src[ip++];
+        mlen += b;
+      } while (b == 255);
+    }
+    if (op + mlen > dst_len) return ORACLE_CORRUPT;
+    for (uint64_t i = 0; i < mlen; ++i) dst[op + i] = dst[op - off + i];
+    op += mlen;
+  }
+  return op == dst_len ? ORACLE_OK : ORACLE_SIZE;
+}
+
+/* Independent blocks: block b decodes enc[offsets[b], offsets[b + 1]) into
+ * dst[b * block_bytes, ...) (the last block holds the remainder of
+ * dst_len). Decodes every block; returns the first failing status. */
+ORACLE_EXPORT int oracle_lz4_decode_blocks(const uint8_t *comp, uint64_t comp_bytes, const uint64_t *offsets,
+                                           int64_t block_bytes, uint8_t *dst, uint64_t dst_len) {
+  if (block_bytes < 1) return ORACLE_INVALID;
+  int status = ORACLE_OK;
+  uint64_t n_blocks = (dst_len + (uint64_t)block_bytes - 1) / (uint64_t)block_bytes;
+  for (uint64_t b = 0; b < n_blocks; ++b) {
+    uint64_t d0 = b * (uint64_t)block_bytes;
+    uint64_t dl = dst_len - d0 < (uint64_t)block_bytes ? dst_len - d0 : (uint64_t)block_bytes;
+    uint64_t s0 = offsets[b], s1 = offsets[b + 1];
+    int st;
+    if (s1 < s0 || s1 > comp_bytes)
+      st = ORACLE_CORRUPT;
+    else
+      st = oracle_lz4_block_decode(comp + s0, s1 - s0, dst + d0, dl);
+    if (st && !status) status = st;
+  }
+  return status;
+}
+
+/* [R] Phase 2.1 cpu_lz4_decompress_then_dequant: decompress all blocks into
+ * the packed INT4 bytes, then dequantize them as oracle_dequant_int4. */
+ORACLE_EXPORT int oracle_lz4_int4_decode(const uint8_t *comp, uint64_t comp_bytes, const uint64_t *offsets,
+                                         int64_t block_bytes, const uint16_t *scales, const uint8_t *zeros,
+                                         int64_t rows, int64_t cols, int64_t group_size, uint16_t *out) {
+  if (rows < 0 || cols < 0) return ORACLE_INVALID;
+  int64_t n = rows * cols;
+  uint64_t packed_len = (uint64_t)((n + 1) / 2);
+  uint8_t *packed = (uint8_t *)calloc(packed_len ? packed_len : 1, 1);
+  if (!packed) return ORACLE_INVALID;
+  int st = oracle_lz4_decode_blocks(comp, comp_bytes, offsets, block_bytes, packed, packed_len);
+  int st2 = oracle_dequant_int4(packed, scales, zeros, rows, cols, group_size, out);
+  free(packed);
+  return st ? st : st2;
+}

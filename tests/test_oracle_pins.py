@@ -1,0 +1,412 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Nothing here is checked against the oracle itself: expected values come from
+the pages' worked examples (tests/golden), from numpy's own binary16
+conversion, from an exact-rational brute-force search of the binary16 grid,
+from closed forms and invariants, and from the system LZ4 library.
+"""
+from __future__ import annotations
+
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+from tests._pins import hexbytes, liblz4, lz4_lib_compress, lz4_lib_decompress, nearest_f16_bits
+
+RNG = np.random.default_rng(20261202)
+
+
+# ---------------------------------------------------------------------------
+# binary16 conversion (IEEE 754-2008)
+# ---------------------------------------------------------------------------
+
+def _np_f16_bits(x: np.ndarray) -> np.ndarray:
+    with np.errstate(over="ignore", invalid="ignore"):
+        return np.asarray(x, dtype=np.float64).astype(np.float16).view(np.uint16)
+
+
+def test_f16_to_f64_exhaustive_matches_numpy():
+    h = np.arange(1 << 16, dtype=np.uint16)
+    got = oracle.f16_to_f64(h)
+    ref = h.view(np.float16).astype(np.float64)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    # signed zeros keep their sign
+    assert np.signbit(got[0x8000]) and not np.signbit(got[0])
+
+
+def test_f16_from_f64_on_every_grid_point_and_midpoint():
+    # every finite binary16 value, each midpoint to its successor (an exact
+    # tie), and the doubles just either side of each midpoint
+    h = np.arange(0x7C00, dtype=np.uint16)
+    v = h.view(np.float16).astype(np.float64)
+    nxt = np.append(v[1:], 65536.0)
+    mid = (v + nxt) / 2  # exact in double
+    cases = np.concatenate([v, mid, np.nextafter(mid, -np.inf), np.nextafter(mid, np.inf)])
+    cases = np.concatenate([cases, -cases])
+    got = oracle.f16_from_f64(cases)
+    ref = _np_f16_bits(cases)
+    assert np.array_equal(got, ref)
+
+
+def test_f16_from_f64_ties_go_to_even():
+    # 1 + 2^-11 lies halfway between 1 (0x3C00, even) and 1 + 2^-10 (0x3C01)
+    assert oracle.f16_from_f64(1 + 2.0 ** -11)[0] == 0x3C00
+    # 1 + 3 * 2^-11 lies halfway between 0x3C01 (odd) and 0x3C02 (even)
+    assert oracle.f16_from_f64(1 + 3 * 2.0 ** -11)[0] == 0x3C02
+    # smallest subnormal is 2^-24; half of it ties to 0 (even)
+    assert oracle.f16_from_f64(2.0 ** -25)[0] == 0x0000
+    assert oracle.f16_from_f64(3 * 2.0 ** -25)[0] == 0x0002
+    # 65520 is the midpoint between 65504 and 2^16 and rounds to infinity
+    assert oracle.f16_from_f64(65519.99)[0] == 0x7BFF
+    assert oracle.f16_from_f64(65520.0)[0] == 0x7C00
+    assert oracle.f16_from_f64(-65520.0)[0] == 0xFC00
+
+
+def test_f16_from_f64_special_values():
+    got = oracle.f16_from_f64(np.array([0.0, -0.0, np.inf, -np.inf, np.nan, 1e300, -1e-300]))
+    assert list(got[:4]) == [0x0000, 0x8000, 0x7C00, 0xFC00]
+    assert (got[4] & 0x7C00) == 0x7C00 and (got[4] & 0x03FF) != 0
+    assert got[5] == 0x7C00 and got[6] == 0x8000
+
+
+def test_f16_from_f64_random_doubles_match_numpy():
+    # log-uniform magnitudes over the whole binary16 range and beyond
+    e = RNG.uniform(-30, 17, size=400_000)
+    x = np.exp2(e) * RNG.choice([-1.0, 1.0], size=e.size)
+    assert np.array_equal(oracle.f16_from_f64(x), _np_f16_bits(x))
+
+
+def test_f16_from_f64_random_float32_match_numpy():
+    # random fp32 bit patterns in the finite range (fp32 -> fp16 is the
+    # conversion the dequantization needs)
+    b = RNG.integers(0, 0x7F800000, size=1_000_000, dtype=np.uint32)
+    x = b.view(np.float32).astype(np.float64) * RNG.choice([-1.0, 1.0], size=b.size)
+    assert np.array_equal(oracle.f16_from_f64(x), _np_f16_bits(x))
+
+
+def test_f16_from_f64_brute_force_grid_search():
+    # exact rationals, rounded by searching the binary16 grid
+    for _ in range(300):
+        t = Fraction(int(RNG.integers(-(1 << 40), 1 << 40)), 1 << int(RNG.integers(20, 60)))
+        assert oracle.f16_from_f64(float(t))[0] == nearest_f16_bits(t), t
+
+
+# ---------------------------------------------------------------------------
+# INT4 group dequantization (roadmap Phase 1.1)
+# ---------------------------------------------------------------------------
+
+def test_int4_worked_example(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "int4_worked_example.json")))
+    out, st = oracle.dequant_int4(np.array(g["packed"], np.uint8), np.array([g["scale_f16_bits"]], np.uint16),
+                                  np.array([g["zero_point"]], np.uint8), 1, 8, 8)
+    assert st == 0
+    assert list(out) == g["expected_f16_bits"]
+    assert list(out.view(np.float16).astype(np.float64)) == g["expected_values"]
+
+
+def test_int4_zero_point_none_equals_zero():
+    packed = RNG.integers(0, 256, 64, dtype=np.uint8)
+    s = np.full(4, 0x3800, np.uint16)
+    a, _ = oracle.dequant_int4(packed, s, None, 4, 32, 32)
+    b, _ = oracle.dequant_int4(packed, s, np.zeros(4, np.uint8), 4, 32, 32)
+    assert np.array_equal(a, b)
+
+
+def test_int4_all_codes_zero_points_and_scales_brute_force():
+    # every (q, z) pair with every binary16 scale; expected through numpy's
+    # binary16 rounding of the exact product (q - z) * s
+    n_s = 1 << 16
+    q = np.tile(np.arange(16, dtype=np.uint8), 16 * n_s)          # code varies fastest
+    z = np.tile(np.repeat(np.arange(16, dtype=np.uint8), 1), n_s)  # one zero point per group of 16
+    s = np.repeat(np.arange(n_s, dtype=np.uint32).astype(np.uint16), 16)  # 16 groups per scale
+    rows, cols, G = n_s, 256, 16
+    packed = (q[0::2] | (q[1::2] << 4)).astype(np.uint8)
+    out, st = oracle.dequant_int4(packed, s, z, rows, cols, G)
+    assert st == 0
+    sv = s.view(np.float16).astype(np.float64)
+    with np.errstate(invalid="ignore"):
+        expect = ((q.reshape(-1, 16).astype(np.float64) - z[:, None]) * sv[:, None]).ravel()
+    ref = _np_f16_bits(expect)
+    nan = np.isnan(expect)
+    assert np.array_equal(out[~nan], ref[~nan])
+    assert np.all((out[nan] & 0x7C00) == 0x7C00) and np.all((out[nan] & 0x3FF) != 0)
+
+
+def test_int4_group_layout_rows_and_nibbles():
+    # distinct scale per group, groups of G along each row of [rows, cols]
+    rows, cols, G = 6, 48, 8
+    codes = RNG.integers(0, 16, rows * cols).astype(np.uint8)
+    packed = (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)
+    n_g = rows * cols // G
+    scales = (np.arange(n_g) + 1).astype(np.float16).view(np.uint16)  # 1, 2, 3, ... exact
+    zeros = RNG.integers(0, 16, n_g).astype(np.uint8)
+    out, st = oracle.dequant_int4(packed, scales, zeros, rows, cols, G)
+    assert st == 0
+    c3 = codes.reshape(rows, cols // G, G).astype(np.int64)
+    z3 = zeros.reshape(rows, cols // G, 1).astype(np.int64)
+    s3 = (np.arange(n_g) + 1).reshape(rows, cols // G, 1)
+    expect = ((c3 - z3) * s3).ravel().astype(np.float64)  # small integers: exact in fp16
+    assert np.array_equal(out.view(np.float16).astype(np.float64), expect)
+
+
+def test_int4_equal_code_and_zero_point_gives_signed_zero():
+    packed = np.array([0x77], np.uint8)
+    pos, _ = oracle.dequant_int4(packed, np.array([0x3C00], np.uint16), np.array([7], np.uint8), 1, 2, 2)
+    neg, _ = oracle.dequant_int4(packed, np.array([0xBC00], np.uint16), np.array([7], np.uint8), 1, 2, 2)
+    assert list(pos) == [0x0000, 0x0000]
+    assert list(neg) == [0x8000, 0x8000]  # (+0) * negative scale = -0 under IEEE
+
+
+def test_int4_odd_element_count_ignores_last_high_nibble():
+    packed = np.array([0x21, 0xF3], np.uint8)  # codes 1, 2, 3 (+ ignored 0xF)
+    out, st = oracle.dequant_int4(packed, np.array([0x3C00], np.uint16), None, 1, 3, 3)
+    assert st == 0 and list(out.view(np.float16)) == [1.0, 2.0, 3.0]
+
+
+# ---------------------------------------------------------------------------
+# INT8 dequantization (roadmap Phase 1.2)
+# ---------------------------------------------------------------------------
+
+def test_int8_example_values_times_scale(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "int8_example.json")))
+    s_bits = int(np.float32(g["scale_f32"]).astype(np.float16).view(np.uint16))
+    assert s_bits == 0x211F
+    s_exact = Fraction(float(np.uint16(s_bits).view(np.float16)))
+    vals = np.array(g["values"], np.int8)
+    out, st = oracle.dequant_int8(vals, np.array([s_bits], np.uint16), None, False, 1, 8)
+    assert st == 0
+    expect = [nearest_f16_bits(int(v) * s_exact) for v in g["values"]]
+    assert list(out) == expect
+    # 96 * s lands exactly halfway between two binary16 values and must go to
+    # the even encoding (0.9599609375, not 0.96044921875)
+    assert float(out.view(np.float16)[5]) == 0.9599609375
+
+
+def test_int8_per_channel_uses_row_scale_and_zero_point():
+    rows, cols = 5, 7
+    q = RNG.integers(-128, 128, rows * cols).astype(np.int8)
+    s = np.array([1, 2, 4, 0.5, -1], np.float16)
+    z = np.array([0, 3, -5, 127, -128], np.int8)
+    out, st = oracle.dequant_int8(q, s.view(np.uint16), z, True, rows, cols)
+    assert st == 0
+    expect = (q.reshape(rows, cols).astype(np.float64) - z[:, None]) * s.astype(np.float64)[:, None]
+    assert np.array_equal(out, _np_f16_bits(expect.ravel()))
+
+
+def test_int8_per_tensor_equals_per_row_with_repeated_scale():
+    rows, cols = 9, 33
+    q = RNG.integers(-128, 128, rows * cols).astype(np.int8)
+    s = np.array([0x2A3B], np.uint16)
+    a, _ = oracle.dequant_int8(q, s, None, False, rows, cols)
+    b, _ = oracle.dequant_int8(q, np.repeat(s, rows), None, True, rows, cols)
+    assert np.array_equal(a, b)
+
+
+def test_int8_symmetric_quantizer_round_trip_within_half_step():
+    # the per-tensor symmetric quantizer of the KV-compression benchmark page
+    # (scale = max|x| / 127, q = clip(round(x / scale), -128, 127)); with the
+    # scale stored in binary16 the reconstruction stays within half a step
+    # plus the scale's own rounding and the output's binary16 rounding
+    x = RNG.standard_normal(4096) * 3.0
+    scale = np.max(np.abs(x)) / 127
+    q = np.clip(np.round(x / scale), -128, 127).astype(np.int8)
+    s16 = np.float16(scale)
+    out, st = oracle.dequant_int8(q, np.array([s16]).view(np.uint16), None, False, 1, x.size)
+    assert st == 0
+    xhat = out.view(np.float16).astype(np.float64)
+    bound = scale / 2 + np.abs(q) * abs(float(s16) - scale) + np.abs(xhat) * 2.0 ** -11
+    assert np.all(np.abs(xhat - x) <= bound * (1 + 1e-12))
+
+
+# ---------------------------------------------------------------------------
+# zero-run decoding (LoreToken page, compression strategies)
+# ---------------------------------------------------------------------------
+
+def _zrle_cases(golden_dir):
+    return json.load(open(os.path.join(golden_dir, "zrle_handmade.json")))["cases"]
+
+
+@pytest.mark.parametrize("idx", range(12))
+def test_zrle_handmade(golden_dir, idx):
+    cases = _zrle_cases(golden_dir)
+    assert len(cases) == 12
+    c = cases[idx]
+    enc = np.frombuffer(hexbytes(c["enc"]), np.uint8)
+    out, st = oracle.zrle_decode(enc, np.array(c["offsets"], np.uint64), c["n"], c["chunk"])
+    assert st == c["status"], c["name"]
+    if c["status"] == 0:
+        assert list(out) == c["out"], c["name"]
+
+
+def test_zrle_round_trip_generated_relu():
+    from weight_dequantization_b200.synth import relu_runs, zrle_encode
+    x = relu_runs(7, 100_003)
+    enc, off = zrle_encode(x, 4096)
+    out, st = oracle.zrle_decode(enc, off, x.size, 4096)
+    assert st == 0 and np.array_equal(out, x)
+    # the law: about 90 % zeros
+    assert 0.85 < np.mean(x == 0) < 0.95
+
+
+def test_zrle_decoder_independent_of_chunk_partition():
+    # the same tensor encoded with different chunk sizes decodes identically
+    x = RNG.integers(1, 0x7C00, 5000).astype(np.uint16)
+    x[RNG.random(5000) < 0.8] = 0
+    from weight_dequantization_b200.synth import zrle_encode
+    for chunk in (1, 7, 64, 4096, 5000, 65535):
+        enc, off = zrle_encode(x, chunk, pad=1)
+        out, st = oracle.zrle_decode(enc, off, x.size, chunk)
+        assert st == 0 and np.array_equal(out, x), chunk
+
+
+# ---------------------------------------------------------------------------
+# LZ4 block decoding
+# ---------------------------------------------------------------------------
+
+def _lz4_cases(golden_dir):
+    return json.load(open(os.path.join(golden_dir, "lz4_handmade.json")))["cases"]
+
+
+def _expected_out(c) -> bytes:
+    if "out" in c:
+        return hexbytes(c["out"])
+    r = c["out_repeat"]
+    return hexbytes(r["unit"]) * r["count"] + hexbytes(r["extra"]) + hexbytes(r["tail"])
+
+
+@pytest.mark.parametrize("idx", range(16))
+def test_lz4_handmade(golden_dir, idx):
+    cases = _lz4_cases(golden_dir)
+    assert len(cases) == 16
+    c = cases[idx]
+    comp = hexbytes(c["comp"])
+    if c["status"] == 0:
+        want = _expected_out(c)
+        out, st = oracle.lz4_block_decode(comp, len(want))
+        assert st == 0, c["name"]
+        assert out.tobytes() == want, c["name"]
+    else:
+        out, st = oracle.lz4_block_decode(comp, c["out_len"])
+        assert st == c["status"], c["name"]
+
+
+@pytest.mark.skipif(liblz4() is None, reason="system liblz4 not present")
+def test_lz4_handmade_strict_cases_agree_with_liblz4(golden_dir):
+    for c in _lz4_cases(golden_dir):
+        if c["status"] == 0 and c.get("strict"):
+            want = _expected_out(c)
+            assert lz4_lib_decompress(hexbytes(c["comp"]), len(want)) == want, c["name"]
+
+
+@pytest.mark.skipif(liblz4() is None, reason="system liblz4 not present")
+@pytest.mark.parametrize("kind", ["zeros", "random", "0xab", "int4_law", "text", "short"])
+def test_lz4_decodes_liblz4_output(kind):
+    n = 65536
+    if kind == "zeros":
+        data = bytes(n)
+    elif kind == "random":
+        data = RNG.integers(0, 256, n, dtype=np.uint8).tobytes()
+    elif kind == "0xab":
+        data = b"\xab" * n
+    elif kind == "int4_law":
+        from weight_dequantization_b200.synth import int4_gauss_groups_packed
+        data = int4_gauss_groups_packed(11, 2 * n).tobytes()
+    elif kind == "text":
+        words = [b"alpha", b"beta", b"gamma", b"delta", b"lz4", b"block"]
+        data = b" ".join(words[i] for i in RNG.integers(0, len(words), 20000))[:n]
+    else:
+        data = b"abcdefghijklm"
+    comp = lz4_lib_compress(data)
+    out, st = oracle.lz4_block_decode(comp, len(data))
+    assert st == 0 and out.tobytes() == data
+
+
+@pytest.mark.skipif(liblz4() is None, reason="system liblz4 not present")
+def test_generator_lz4_output_accepted_by_liblz4():
+    # the roadmap's 64 KB test block (0xAB x 65536), a literal-only random
+    # block, and the INT4 workload law: the input generator's compressor must
+    # emit blocks that an outside decoder reads back exactly
+    from weight_dequantization_b200.synth import int4_gauss_groups_packed, lz4_compress_block
+    cases = [b"\xab" * 65536, RNG.integers(0, 256, 65536, dtype=np.uint8).tobytes(),
+             int4_gauss_groups_packed(5, 131072).tobytes(), b"x", b"", bytes(13)]
+    for data in cases:
+        comp = lz4_compress_block(np.frombuffer(data, np.uint8) if data else np.zeros(0, np.uint8))
+        assert lz4_lib_decompress(comp.tobytes(), len(data)) == data
+        out, st = oracle.lz4_block_decode(comp, len(data))
+        assert st == 0 and out.tobytes() == data
+    # 0xAB x 65536 is not stored as 64 KB of literals: one literal + a long
+    # offset-1 match
+    comp = lz4_compress_block(np.full(65536, 0xAB, np.uint8))
+    assert comp.size < 300
+
+
+def test_lz4_literal_only_64k_block():
+    from weight_dequantization_b200.synth import lz4_compress_block
+    data = RNG.integers(0, 256, 65536, dtype=np.uint8)
+    comp = lz4_compress_block(data, force_literals=True)
+    # token + 256 extension bytes for 65536 - 15 + the literals
+    assert comp.size == 1 + (65536 - 15) // 255 + 1 + 65536
+    out, st = oracle.lz4_block_decode(comp, data.size)
+    assert st == 0 and np.array_equal(out, data)
+
+
+def test_lz4_match_at_maximum_offset():
+    # a match reaching back exactly 65535 bytes
+    head = RNG.integers(0, 256, 65535, dtype=np.uint8).tobytes()
+    tok_lit = bytes([0xF4]) + bytes([255] * ((65535 - 15) // 255)) + bytes([(65535 - 15) % 255])
+    comp = tok_lit + head + bytes([0xFF, 0xFF]) + bytes([0x50]) + b"tail!"
+    # token 0xF4: 65535 literals, match length 8 at offset 65535, then 5 literals
+    out, st = oracle.lz4_block_decode(comp, 65535 + 8 + 5)
+    assert st == 0
+    assert out.tobytes() == head + head[:8] + b"tail!"
+    if liblz4() is not None:
+        assert lz4_lib_decompress(comp, 65535 + 8 + 5) == out.tobytes()
+
+
+def test_lz4_blocks_and_fused_equal_decompress_then_dequant():
+    from weight_dequantization_b200.synth import fp16_uniform, int4_gauss_groups_packed, lz4_compress_blocks, u8_uniform
+    rows, cols, G = 48, 4096, 128
+    n = rows * cols
+    packed = int4_gauss_groups_packed(3, n)
+    comp, off = lz4_compress_blocks(packed, 16384)
+    s = fp16_uniform(3, n // G, 0.001, 0.1, stream=1)
+    z = u8_uniform(3, n // G, 0, 15, stream=2)
+    raw, st = oracle.lz4_decode_blocks(comp, off, 16384, packed.size)
+    assert st == 0 and np.array_equal(raw, packed)
+    fused, st = oracle.lz4_int4_decode(comp, off, 16384, s, z, rows, cols, G)
+    assert st == 0
+    # independent dequant of the raw packed bytes through numpy
+    codes = np.empty(n, np.int64)
+    codes[0::2] = packed & 0xF
+    codes[1::2] = packed >> 4
+    sv = s.view(np.float16).astype(np.float64)
+    expect = ((codes.reshape(-1, G) - z[:, None].astype(np.int64)) * sv[:, None]).ravel()
+    assert np.array_equal(fused, _np_f16_bits(expect))
+
+
+def test_lz4_corrupt_block_is_reported_not_crashing():
+    from weight_dequantization_b200.synth import int4_gauss_groups_packed, lz4_compress_block
+    data = int4_gauss_groups_packed(9, 131072)
+    comp = lz4_compress_block(data)
+    bad = 0
+    for i in range(200):
+        c = comp.copy()
+        pos = int(RNG.integers(0, c.size))
+        c[pos] ^= np.uint8(1 << int(RNG.integers(0, 8)))
+        out, st = oracle.lz4_block_decode(c, data.size)
+        if st != 0:
+            bad += 1
+        else:
+            # a flip inside a literal decodes fine but differs from the input
+            assert not np.array_equal(out, data) or c.tobytes() == comp.tobytes()
+    assert bad > 0
+    # truncation always fails
+    for cut in (1, 2, 10, comp.size // 2):
+        _, st = oracle.lz4_block_decode(comp[:-cut], data.size)
+        assert st != 0
