@@ -1,0 +1,581 @@
+#!/usr/bin/env python
+"""Decode benchmark on B200: decoded fp16 GB/s and fraction of the HBM roofline.
+
+One step = one pass of every decode workload over its synthetic input:
+  C1  INT4 group dequant, 1,048,576 codes, group 256
+  C2  INT8 per-row dequant, 8192 x 8192
+  C3  zero-run decode, 8 x 2048 x 11008 fp16 ReLU-like activations
+  C4  fused LZ4 -> INT4 -> fp16, 4096 x 14336, group 128, 64 KB blocks
+  C5  8 Llama-2-70B-shaped layers (q, o, k, v, gate, up, down), fused LZ4 ->
+      INT4 -> fp16, each layer decoded (one launch) into one reused buffer
+The headline value is the step's total decoded fp16 bytes / step time
+(GB/s, 1e9). Inputs are resident in HBM when the timed region starts; the
+step touches ~16 GB, far more than L2, so no L2 flush is needed between
+steps. Per-codec figures and the roofline fraction of the dominant kernel
+(the fused LZ4 decode of C5) are reported beside it.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lt|reference]
+Under torchrun each rank decodes its own copy of the workload (weak scaling,
+no data-path collective); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decoded FP16 GB/s per codec; % of B200 HBM roofline (bytes read+written)"
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of the fused LZ4
+# kernel on one C5 layer, from the ncu capture summarised under profiles/;
+# valid only while the kernel sources hash to `sources_sha256`.
+NCU_TRAFFIC = {"sources_sha256": None, "bytes_per_launch": None, "profile": None}
+
+
+def kernel_sources_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("lt_lz4.cu", "lt_common.cuh"):
+        with open(os.path.join(ROOT, "weight_dequantization_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["lt", "reference"], default="lt")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=8, help="C5 layers (8 is the workload)")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_init(world):
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, dist) -> float:
+    if dist is None:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, dist) -> float:
+    if dist is None:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.rows = []
+        self.proc = None
+        self.gpu_id = gpu_id
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 7:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, smax, reasons = [], [], set()
+        for r in self.rows:
+            try:
+                sm.append(float(r[0]))
+                smax.append(float(r[1]))
+            except ValueError:
+                continue
+            for i, nm in enumerate(names):
+                if r[3 + i].lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_id_for(dev_index: int) -> str:
+    import torch
+
+    try:
+        u = str(torch.cuda.get_device_properties(dev_index).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        return vis.split(",")[dev_index] if vis else str(dev_index)
+
+
+# ----------------------------------------------------------------------------
+# workloads
+# ----------------------------------------------------------------------------
+
+def build_host_workload(rank: int, layers: int):
+    """Seeded host inputs; each rank gets its own seeds (weak scaling)."""
+    from weight_dequantization_b200.synth import workloads as W
+
+    off = 1000 * rank
+    return {
+        "C1": W.c1_int4(seed=1 + off),
+        "C2": W.c2_int8(seed=2 + off),
+        "C3": W.c3_zrle(seed=3 + off),
+        "C4": W.c4_lz4_int4(seed=4 + off),
+        "C5": W.c5_layers(layers=layers, seed=5 + off),
+    }
+
+
+def nbytes(a) -> int:
+    return 0 if a is None else int(a.nbytes)
+
+
+def algorithmic_bytes(hw):
+    """Bytes the method must read + write per codec (actual buffers)."""
+    c1, c2, c3, c4 = hw["C1"], hw["C2"], hw["C3"], hw["C4"]
+    n1 = c1["rows"] * c1["cols"]
+    n2 = c2["rows"] * c2["cols"]
+    out = {
+        "C1": (nbytes(c1["packed"]) + nbytes(c1["scales"]) + nbytes(c1["zeros"]), 2 * n1),
+        "C2": (nbytes(c2["q"]) + nbytes(c2["scales"]) + nbytes(c2["zeros"]), 2 * n2),
+        "C3": (nbytes(c3["enc"]) + nbytes(c3["offsets"]), 2 * c3["n"]),
+        "C4": (nbytes(c4["comp"]) + nbytes(c4["offsets"]) + nbytes(c4["scales"]) + nbytes(c4["zeros"]),
+               2 * c4["rows"] * c4["cols"]),
+    }
+    layer = []
+    for mats in hw["C5"]:
+        rd = sum(nbytes(m["comp"]) + nbytes(m["offsets"]) + nbytes(m["scales"]) + nbytes(m["zeros"]) for m in mats)
+        wr = sum(2 * m["rows"] * m["cols"] for m in mats)
+        layer.append((rd, wr))
+    out["C5"] = (sum(r for r, _ in layer), sum(w for _, w in layer))
+    return out, layer
+
+
+class DeviceWorkload:
+    """Device copies of the inputs, output buffers, and pinned host staging
+    buffers for the end-to-end measurement."""
+
+    def __init__(self, hw, pinned: bool):
+        import numpy as np
+        import torch
+
+        self.torch = torch
+        self.hw = hw
+        self.h2d = []  # (pinned host tensor, device tensor)
+
+        def put(a):
+            if a is None:
+                return None
+            a = np.ascontiguousarray(a)
+            if a.dtype == np.uint16:
+                a = a.view(np.int16)
+            elif a.dtype == np.uint64:
+                a = a.view(np.int64)
+            host = torch.from_numpy(a)
+            d = host.to("cuda")
+            if pinned:
+                ph = torch.empty_like(host).pin_memory()
+                ph.copy_(host)
+                self.h2d.append((ph, d))
+            return d
+
+        c1, c2, c3, c4 = hw["C1"], hw["C2"], hw["C3"], hw["C4"]
+        self.c1 = dict(packed=put(c1["packed"]), scales=put(c1["scales"]), zeros=put(c1["zeros"]))
+        self.c1_out = torch.empty(c1["rows"] * c1["cols"], dtype=torch.float16, device="cuda")
+        self.c2 = dict(q=put(c2["q"]), scales=put(c2["scales"]))
+        self.c2_out = torch.empty(c2["rows"] * c2["cols"], dtype=torch.float16, device="cuda")
+        self.c3 = dict(enc=put(c3["enc"]), offsets=put(c3["offsets"]))
+        self.c3_out = torch.empty(c3["n"], dtype=torch.float16, device="cuda")
+        self.c4 = dict(comp=put(c4["comp"]), offsets=put(c4["offsets"]), scales=put(c4["scales"]),
+                       zeros=put(c4["zeros"]))
+        self.c4_out = torch.empty(c4["rows"] * c4["cols"], dtype=torch.float16, device="cuda")
+        layer_elems = max(sum(m["rows"] * m["cols"] for m in mats) for mats in hw["C5"])
+        self.c5_out = torch.empty(layer_elems, dtype=torch.float16, device="cuda")  # one reused layer buffer
+        self.c5 = []
+        for mats in hw["C5"]:
+            descs, base = [], 0
+            for m in mats:
+                n = m["rows"] * m["cols"]
+                descs.append(dict(comp=put(m["comp"]), comp_bytes=int(m["comp"].size), block_offsets=put(m["offsets"]),
+                                  scales=put(m["scales"]), zeros=put(m["zeros"]), out=self.c5_out[base:base + n],
+                                  rows=m["rows"], cols=m["cols"], group_size=m["group_size"],
+                                  block_bytes=m["block_bytes"]))
+                base += n
+            self.c5.append(descs)
+        self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.status_host = torch.zeros(1, dtype=torch.int32).pin_memory() if pinned else None
+        self.h2d_bytes = sum(int(p.numel() * p.element_size()) for p, _ in self.h2d)
+
+    # one pass of the whole hot path; `ev` (optional) receives per-codec events
+    def step(self, ev=None):
+        from weight_dequantization_b200 import lt_decode as L
+
+        torch = self.torch
+        hw = self.hw
+        s = torch.cuda.current_stream()
+
+        def mark(key):
+            if ev is not None:
+                e = torch.cuda.Event(enable_timing=True)
+                e.record(s)
+                ev.setdefault(key, []).append(e)
+
+        c1, c2, c3, c4 = hw["C1"], hw["C2"], hw["C3"], hw["C4"]
+        mark("C1.start")
+        L.lt_dequant_int4(self.c1["packed"], self.c1["scales"], self.c1["zeros"], c1["rows"], c1["cols"],
+                          c1["group_size"], self.c1_out, s)
+        mark("C1.end")
+        L.lt_dequant_int8(self.c2["q"], self.c2["scales"], None, L.LT_SCALE_PER_ROW, c2["rows"], c2["cols"],
+                          self.c2_out, s)
+        mark("C2.end")
+        L.lt_zrle_decode(self.c3["enc"], int(c3["enc"].size), self.c3["offsets"], c3["n"], c3["chunk_elems"],
+                         self.c3_out, self.status, s)
+        mark("C3.end")
+        L.lt_lz4_int4_decode(self.c4["comp"], int(c4["comp"].size), self.c4["offsets"], c4["block_bytes"],
+                             self.c4["scales"], self.c4["zeros"], c4["rows"], c4["cols"], c4["group_size"],
+                             self.c4_out, self.status, s)
+        mark("C4.end")
+        for i, descs in enumerate(self.c5):
+            L.lt_lz4_int4_decode_batch(descs, self.status, s)
+            mark("C5.layer")
+        return 4 + len(self.c5)  # kernel launches of this step
+
+    def upload_inputs(self):
+        for ph, d in self.h2d:
+            d.copy_(ph, non_blocking=True)
+
+    def download_status(self):
+        self.status_host.copy_(self.status, non_blocking=True)
+
+
+def launches_per_step(hw) -> int:
+    # every call takes its vector path (no scalar tail launch): all element
+    # counts are multiples of 8, groups multiples of 8, buffers 256-byte aligned
+    c1, c2 = hw["C1"], hw["C2"]
+    assert (c1["rows"] * c1["cols"]) % 8 == 0 and c1["group_size"] % 8 == 0
+    assert (c2["rows"] * c2["cols"]) % 8 == 0 and c2["cols"] % 8 == 0
+    return 4 + len(hw["C5"])
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ----------------------------------------------------------------------------
+
+def oracle_sample_step(hw, frac: float):
+    """Run the oracle on the first `frac` of every workload's units; returns
+    (decoded bytes, seconds)."""
+    import numpy as np
+
+    import oracle
+
+    t0 = time.perf_counter()
+    dec = 0
+    c1 = hw["C1"]
+    r1 = max(1, int(c1["rows"] * frac))
+    n1 = r1 * c1["cols"]
+    g1 = n1 // c1["group_size"]
+    oracle.dequant_int4(c1["packed"][: n1 // 2], c1["scales"][:g1], c1["zeros"][:g1], r1, c1["cols"],
+                        c1["group_size"])
+    dec += 2 * n1
+    c2 = hw["C2"]
+    r2 = max(1, int(c2["rows"] * frac))
+    oracle.dequant_int8(c2["q"][: r2 * c2["cols"]], c2["scales"][:r2], None, True, r2, c2["cols"])
+    dec += 2 * r2 * c2["cols"]
+    c3 = hw["C3"]
+    nch = max(1, int((len(c3["offsets"]) - 1) * frac))
+    n3 = min(c3["n"], nch * c3["chunk_elems"])
+    oracle.zrle_decode(c3["enc"], c3["offsets"][: nch + 1], n3, c3["chunk_elems"])
+    dec += 2 * n3
+
+    def lz4_part(m):
+        nb = max(1, int((len(m["offsets"]) - 1) * frac))
+        s1 = int(m["offsets"][nb])
+        codes = min(m["rows"] * m["cols"], nb * 2 * m["block_bytes"])
+        g = codes // m["group_size"]
+        oracle.lz4_int4_decode(m["comp"][:s1], m["offsets"][: nb + 1], m["block_bytes"], m["scales"][:g],
+                               m["zeros"][:g], 1, codes, m["group_size"])
+        return 2 * codes
+
+    dec += lz4_part(hw["C4"])
+    for mats in hw["C5"]:
+        for m in mats:
+            dec += lz4_part(m)
+    return dec, time.perf_counter() - t0
+
+
+def cpu_baseline(hw, budget_s: float = 15.0):
+    frac = 1.0 / 512
+    dec, dt = oracle_sample_step(hw, frac)
+    # scale the sample to the time budget (bounded)
+    frac2 = min(0.25, frac * max(1.0, budget_s / max(dt, 1e-3)))
+    if frac2 > frac * 1.5:
+        frac = frac2
+        dec, dt = oracle_sample_step(hw, frac)
+    return {
+        "value": dec / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+        "sample": f"first {frac:.4%} of the units (rows, chunks, 64 KB blocks) of every workload of one step "
+                  f"({dec / 1e6:.1f} MB decoded in {dt:.1f} s, single-threaded plain C oracle)",
+    }
+
+
+# ----------------------------------------------------------------------------
+# arms
+# ----------------------------------------------------------------------------
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_config(hw, layers):
+    c5_codes = sum(m["rows"] * m["cols"] for mats in hw["C5"] for m in mats)
+    return {
+        "workload": "decode suite: C1 INT4 1M codes G256 + C2 INT8 8192x8192 per-row + C3 zero-run 8x2048x11008 "
+                    f"+ C4 LZ4+INT4 4096x14336 G128 + C5 {layers}-layer Llama-2-70B-shaped LZ4+INT4 G128 sweep "
+                    "(64 KB LZ4 blocks, one reused layer buffer)",
+        "c5_codes": c5_codes,
+        "l2": "inputs larger than L2 (each step touches ~16 GB; no flush)",
+    }
+
+
+def run_lt(args, rank, world, local):
+    import torch
+
+    torch.cuda.set_device(local)
+    dist = dist_init(world)
+    from weight_dequantization_b200 import lt_decode as L
+
+    L.load_library()
+    hw = build_host_workload(rank, args.layers)
+    (alg, layer_alg) = algorithmic_bytes(hw)
+    dw = DeviceWorkload(hw, pinned=True)
+    nlaunch = launches_per_step(hw)
+    torch.cuda.synchronize()
+
+    # warm-up
+    for _ in range(max(args.warmup, 0)):
+        dw.step()
+    torch.cuda.synchronize()
+    if int(dw.status.item()) != 0:
+        raise RuntimeError(f"decode reported status {int(dw.status.item())} on the benchmark input")
+
+    # timed region: K steps, device time by CUDA events on the launching stream
+    clocks = ClockSampler(gpu_id_for(local))
+    clocks.start()
+    time.sleep(0.3)
+    ev = {}
+    s = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(s)
+    for _ in range(args.steps):
+        dw.step(ev)
+    e1.record(s)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ck = clocks.stop()
+    elapsed = e0.elapsed_time(e1) / 1e3
+    elapsed = max_over_ranks(elapsed, dist)
+
+    # per codec (device time of the launches, summed over steps)
+    K = args.steps
+    t_c = {"C1": 0.0, "C2": 0.0, "C3": 0.0, "C4": 0.0, "C5": 0.0}
+    layer_t = []
+    L5 = len(dw.c5)
+    for k in range(K):
+        t_c["C1"] += ev["C1.start"][k].elapsed_time(ev["C1.end"][k])
+        t_c["C2"] += ev["C1.end"][k].elapsed_time(ev["C2.end"][k])
+        t_c["C3"] += ev["C2.end"][k].elapsed_time(ev["C3.end"][k])
+        t_c["C4"] += ev["C3.end"][k].elapsed_time(ev["C4.end"][k])
+        prev = ev["C4.end"][k]
+        for li in range(L5):
+            cur = ev["C5.layer"][k * L5 + li]
+            dt = prev.elapsed_time(cur)
+            layer_t.append(dt)
+            t_c["C5"] += dt
+            prev = cur
+    peak, peak_kind = read_peaks()
+    per_codec = {}
+    for c, (rd, wr) in alg.items():
+        t = t_c[c] / 1e3 / K
+        per_codec[c] = {"decoded_GBps": wr / t / 1e9, "us_per_call": t * 1e6 / (L5 if c == "C5" else 1),
+                        "bytes_read": rd, "bytes_written": wr,
+                        "hbm_frac_of_measured": (rd + wr) / t / 1e9 / peak,
+                        "hbm_frac_of_8TBps": (rd + wr) / t / 1e9 / NOMINAL_HBM_GBS}
+    decoded = sum(wr for _, wr in alg.values())
+    total_decoded = sum_over_ranks(decoded * K, dist)
+    value = total_decoded / elapsed / 1e9
+
+    # roofline of the dominant kernel: the fused LZ4 decode, one launch per C5 layer
+    avg_layer_s = statistics.mean(layer_t) / 1e3
+    layer_bytes = statistics.mean([rd + wr for rd, wr in layer_alg])
+    achieved = layer_bytes / avg_layer_s / 1e9
+    traffic = None
+    if NCU_TRAFFIC["sources_sha256"] == kernel_sources_sha() and NCU_TRAFFIC["bytes_per_launch"]:
+        traffic = NCU_TRAFFIC["bytes_per_launch"]
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": traffic, "kernel": "k_lz4<fused> (C5 layer, 7 matrices per launch)",
+                "peak_kind": peak_kind, "algorithmic_bytes_per_launch": layer_bytes,
+                "frac_of_8TBps": achieved / NOMINAL_HBM_GBS}
+
+    # end-to-end: inputs copied from pinned host memory every step, status read back
+    torch.cuda.synchronize()
+    dw.upload_inputs()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    KE = max(1, args.e2e_steps)
+    f0.record(s)
+    for _ in range(KE):
+        dw.upload_inputs()
+        dw.step()
+        dw.download_status()
+    f1.record(s)
+    torch.cuda.synchronize()
+    e2e_t = max_over_ranks(f0.elapsed_time(f1) / 1e3, dist)
+    e2e_total = sum_over_ranks(decoded * KE, dist)
+    e2e = {"value": e2e_total / e2e_t / 1e9, "unit": "GB/s", "h2d_bytes_per_step": dw.h2d_bytes,
+           "d2h_bytes_per_step": 4, "steps": KE}
+    if int(dw.status_host.item()) != 0:
+        raise RuntimeError("decode reported an error in the end-to-end run")
+
+    result = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(hw)
+        result = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": elapsed / K * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16", "data": "synthetic (seeded generators; value laws of the workloads)",
+            "config": workload_config(hw, args.layers), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": nlaunch * K, "clocks": {"sm_mhz": ck["sm_mhz"], "sm_max_mhz": ck["sm_max_mhz"],
+                                                     "reasons": ck["reasons"], "samples": ck["samples"]},
+            "per_codec": per_codec, "impl": "lt",
+        }
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def run_reference(args, rank, world):
+    """The oracle (plain C, single thread) as the reference arm: each step is
+    a bounded sample of the same workload, sized so the whole run stays
+    within a few minutes."""
+    if rank != 0:
+        return None
+    hw = build_host_workload(0, args.layers)
+    steps = args.steps + args.warmup
+    # calibrate: aim at ~90 s for all steps together
+    dec, dt = oracle_sample_step(hw, 1.0 / 4096)
+    per_step_budget = max(0.05, 90.0 / max(steps, 1))
+    frac = min(0.25, (1.0 / 4096) * per_step_budget / max(dt, 1e-4))
+    for _ in range(args.warmup):
+        oracle_sample_step(hw, frac)
+    tot_dec, tot_t = 0, 0.0
+    for _ in range(args.steps):
+        d, t = oracle_sample_step(hw, frac)
+        tot_dec += d
+        tot_t += t
+    value = tot_dec / tot_t / 1e9
+    sample = (f"first {frac:.5%} of the units of every workload per step, single-threaded plain C oracle "
+              f"on the host ({tot_dec / max(args.steps, 1) / 1e6:.2f} MB decoded per step)")
+    return {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": tot_t / max(args.steps, 1) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(hw, args.layers), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+    else:
+        res = run_lt(args, rank, world, local)
+    if res is not None and rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

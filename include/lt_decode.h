@@ -1,0 +1,194 @@
+/*
+ * lt_decode.h -- C ABI of liblt_decode.so: on-device decoding of compressed
+ * tensors on NVIDIA B200 (sm_100a).
+ *
+ * Operations (sources are web pages, cited by title and section):
+ *   INT4 group dequantization   "GPU Compression Pipeline - TDD Roadmap",
+ *                               Phase 1.1 INT4 Dequantization
+ *   INT8 dequantization         same page, Phase 1.2 INT8 Dequantization
+ *   zero-run decoding           "LoreToken-powered GPU memory layer",
+ *                               compression strategies (zero-run encoding of
+ *                               mostly-zero ReLU activations)
+ *   fused LZ4 -> INT4 -> fp16   "GPU Compression Pipeline - TDD Roadmap",
+ *                               Phase 2.1 LZ4 + INT4 Fused Kernel, with the
+ *                               64 KB blocks of Phase 3.1 / Phase 6.1
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every data pointer is a DEVICE pointer owned by the caller (except the
+ *    descriptor array of lt_lz4_int4_decode_batch, a host array read during
+ *    the call). The library allocates no memory, frees nothing, never
+ *    synchronizes and keeps no pointer after it returns.
+ *  - All work is enqueued on `stream` (NULL = the legacy default stream).
+ *    A call returns as soon as its kernel is enqueued.
+ *  - lt_half is an IEEE 754 binary16 bit pattern (the storage of __half /
+ *    torch.float16). lt_half pointers must be 2-byte aligned and
+ *    uint64_t pointers 8-byte aligned, else LT_ERR_MISALIGNED. Wider
+ *    alignment (16 bytes) of the large buffers selects vectorized kernels;
+ *    any other alignment is still decoded correctly, just more slowly.
+ *  - Dequantized values are (q - z) * s rounded once to binary16: round to
+ *    nearest, ties to even, subnormals kept, overflow to infinity. |q - z|
+ *    is at most 255, so the product is exact before that single rounding.
+ *  - Host-checkable argument errors are returned synchronously and nothing is
+ *    enqueued. Launch failures return LT_ERR_CUDA.
+ *  - Data-dependent errors of the stream decoders (a corrupt stream, a
+ *    decoded size that differs from the declared one) are asynchronous: if
+ *    `d_status` is not NULL the first error code is stored there (the caller
+ *    zeroes it beforehand and reads it after synchronizing the stream).
+ *    After such an error the output content is unspecified, but every write
+ *    stays inside the output buffer. Decoders never trap, assert or loop
+ *    unboundedly on corrupt input.
+ *  - Sizes of zero are valid and enqueue nothing.
+ */
+#ifndef LT_DECODE_H_
+#define LT_DECODE_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LT_ABI_VERSION 1
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *lt_stream_t;
+
+/* IEEE 754 binary16 bit pattern. */
+typedef uint16_t lt_half;
+
+typedef enum {
+  LT_OK = 0,
+  LT_ERR_INVALID_ARG = 1,    /* NULL pointer with a non-zero size, negative size, bad shape */
+  LT_ERR_MISALIGNED = 2,     /* pointer not aligned to its element type */
+  LT_ERR_UNSUPPORTED = 3,    /* valid request outside what the kernels implement */
+  LT_ERR_CORRUPT_STREAM = 4, /* (device status) malformed LZ4 / zero-run data */
+  LT_ERR_SIZE_MISMATCH = 5,  /* (device status) stream decodes to a different length */
+  LT_ERR_CUDA = 6            /* a CUDA launch failed */
+} lt_status;
+
+typedef enum { LT_SCALE_PER_TENSOR = 0, LT_SCALE_PER_ROW = 1 } lt_scale_mode;
+
+/*
+ * INT4 group dequantization ("GPU Compression Pipeline - TDD Roadmap",
+ * Phase 1.1; block-level, GPTQ/AWQ-style groups).
+ *
+ *   packed  ceil(rows*cols/2) bytes: code k = rows-major element index k is
+ *           the low nibble of byte k/2 when k is even, the high nibble when
+ *           odd (the page's example: bytes 0x10,0x32,0x54,0x76 are codes
+ *           0..7). An odd element count ignores the last high nibble.
+ *   scales  rows*cols/group_size binary16 scales, group g covers codes
+ *           [g*group_size, (g+1)*group_size): groups run along each row of a
+ *           row-major [rows, cols] tensor and never cross a row.
+ *   zeros   one uint8 zero point per group, or NULL for zero point 0.
+ *   out     rows*cols binary16 values, out[k] = fp16_rn((q[k] - z[g]) * s[g]).
+ *   group_size >= 1 and divides cols, else LT_ERR_INVALID_ARG.
+ */
+lt_status lt_dequant_int4(const uint8_t *packed, const lt_half *scales, const uint8_t *zeros, int64_t rows,
+                          int64_t cols, int32_t group_size, lt_half *out, lt_stream_t stream);
+
+/*
+ * INT8 dequantization ("GPU Compression Pipeline - TDD Roadmap", Phase 1.2:
+ * "values * scale", per-tensor and per-channel scales).
+ *
+ *   q           rows*cols int8 values, row-major [rows, cols].
+ *   scales      1 binary16 scale (LT_SCALE_PER_TENSOR) or one per row
+ *               (LT_SCALE_PER_ROW, the output channel).
+ *   zeros       int8 zero points laid out like scales, or NULL for 0.
+ *   out         rows*cols binary16, out[r, c] = fp16_rn((q[r, c] - z) * s).
+ */
+lt_status lt_dequant_int8(const int8_t *q, const lt_half *scales, const int8_t *zeros, int32_t scale_mode,
+                          int64_t rows, int64_t cols, lt_half *out, lt_stream_t stream);
+
+/*
+ * Zero-run decoding of mostly-zero activations ("LoreToken-powered GPU
+ * memory layer", compression strategies: zero-run encoding).
+ *
+ *   enc, enc_bytes   the encoded stream.
+ *   chunk_offsets    n_chunks + 1 byte offsets into enc (uint64, device),
+ *                    n_chunks = ceil(n_elements / chunk_elems). Chunk c
+ *                    covers elements [c*chunk_elems, min(n, (c+1)*chunk_elems))
+ *                    and its bytes are enc[offsets[c], offsets[c+1]).
+ *   Chunk bytes: records (u16 zero_run, u16 literal_count, literal_count
+ *   binary16 literals), little-endian; each record emits zero_run elements
+ *   equal to +0 (0x0000), then the literals bit for bit. Decoding of a chunk
+ *   stops once it is full; bytes after that are padding. Offsets may be any
+ *   byte position; 16-byte-aligned offsets (the generator pads chunks to 16
+ *   bytes) take the fast path.
+ *   Device status: LT_ERR_CORRUPT_STREAM if a record overruns its chunk or
+ *   its bytes, or an offset pair lies outside enc; LT_ERR_SIZE_MISMATCH if a
+ *   chunk's bytes end before the chunk is full.
+ *   chunk_elems in [1, 65535], else LT_ERR_UNSUPPORTED.
+ */
+lt_status lt_zrle_decode(const uint8_t *enc, uint64_t enc_bytes, const uint64_t *chunk_offsets, int64_t n_elements,
+                         int32_t chunk_elems, lt_half *out, int32_t *d_status, lt_stream_t stream);
+
+/*
+ * Fused LZ4 block decompression -> INT4 unpack -> scale -> binary16
+ * ("GPU Compression Pipeline - TDD Roadmap", Phase 2.1: decompress
+ * directly to dequantized F16 with no intermediate buffer).
+ *
+ *   comp, comp_bytes   raw LZ4 blocks (block format, no frame), independent
+ *                      (no block refers to another).
+ *   block_offsets      n_blocks + 1 byte offsets into comp (uint64, device).
+ *   block_bytes        decompressed bytes per block, in [16, 65536] and a
+ *                      multiple of 16 (65536 in the workloads); the last
+ *                      block holds the remainder of ceil(rows*cols/2).
+ *                      n_blocks = ceil(ceil(rows*cols/2) / block_bytes).
+ *   The decompressed bytes are the `packed` array of lt_dequant_int4, and
+ *   scales / zeros / rows / cols / group_size / out mean what they mean
+ *   there. Decompressed bytes live only in on-chip shared memory.
+ *   Device status: LT_ERR_CORRUPT_STREAM for a malformed block (offset 0 or
+ *   before the block start, literal or match past the block end, input
+ *   overrun, an offset pair outside comp), LT_ERR_SIZE_MISMATCH for a block
+ *   that decodes to fewer bytes than it must.
+ */
+lt_status lt_lz4_int4_decode(const uint8_t *comp, uint64_t comp_bytes, const uint64_t *block_offsets,
+                             int32_t block_bytes, const lt_half *scales, const uint8_t *zeros, int64_t rows,
+                             int64_t cols, int32_t group_size, lt_half *out, int32_t *d_status, lt_stream_t stream);
+
+/*
+ * Several fused LZ4 -> INT4 decodes in one launch (the weight matrices of a
+ * transformer layer decoded into one reused buffer). Each descriptor has
+ * the meaning of the lt_lz4_int4_decode arguments of the same name. The
+ * descriptor array itself is a HOST array, read during the call.
+ * 1 <= n_desc <= LT_LZ4_BATCH_MAX, else LT_ERR_INVALID_ARG / UNSUPPORTED.
+ */
+#define LT_LZ4_BATCH_MAX 16
+typedef struct {
+  const uint8_t *comp;
+  uint64_t comp_bytes;
+  const uint64_t *block_offsets;
+  const lt_half *scales;
+  const uint8_t *zeros;
+  lt_half *out;
+  int64_t rows;
+  int64_t cols;
+  int32_t group_size;
+  int32_t block_bytes;
+} lt_lz4_int4_desc;
+
+lt_status lt_lz4_int4_decode_batch(const lt_lz4_int4_desc *descs, int32_t n_desc, int32_t *d_status,
+                                   lt_stream_t stream);
+
+/*
+ * Plain LZ4 block decompression to bytes (the same on-chip decoder as the
+ * fused path, writing the decompressed bytes instead of dequantizing them).
+ * Used to check the LZ4 stage bit for bit, and as a general decoder.
+ *   out        out_bytes bytes; block b fills [b*block_bytes, ...).
+ *   block_bytes in [16, 65536], a multiple of 16.
+ */
+lt_status lt_lz4_decode(const uint8_t *comp, uint64_t comp_bytes, const uint64_t *block_offsets, int32_t block_bytes,
+                        uint8_t *out, uint64_t out_bytes, int32_t *d_status, lt_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char *lt_status_string(lt_status s);
+
+/* LT_ABI_VERSION of the built library. */
+int32_t lt_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LT_DECODE_H_ */

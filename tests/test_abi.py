@@ -1,0 +1,80 @@
+"""The C-ABI library loads and exports what include/lt_decode.h declares.
+
+Runs without a GPU: only symbol lookup and host-side argument checks, which
+return before any CUDA call.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from weight_dequantization_b200 import _build
+from weight_dequantization_b200 import lt_decode as L
+
+HEADER = os.path.join(_build.ROOT, "include", "lt_decode.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build_decode()
+    return L.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lt_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    assert set(names) == set(L.EXPORTED), names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_abi_version_and_status_strings(lib):
+    assert L.abi_version() == 1
+    for code in range(7):
+        s = L.status_string(code)
+        assert s and s != "unknown status"
+    assert L.status_string(99) == "unknown status"
+
+
+def test_host_argument_errors_return_synchronously(lib):
+    # each of these is rejected before anything touches a device
+    P = 0x1000  # never dereferenced
+    assert lib.lt_dequant_int4(P, P, None, -1, 8, 8, P, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_dequant_int4(P, P, None, 2, 12, 8, P, None) == L.LT_ERR_INVALID_ARG  # 8 does not divide 12
+    assert lib.lt_dequant_int4(P, P, None, 2, 8, 0, P, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_dequant_int4(None, P, None, 2, 8, 8, P, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_dequant_int4(P, P + 1, None, 2, 8, 8, P, None) == L.LT_ERR_MISALIGNED
+    assert lib.lt_dequant_int4(P, P, None, 0, 8, 8, P, None) == L.LT_OK  # empty: nothing enqueued
+    assert lib.lt_dequant_int8(P, P, None, 2, 4, 4, P, None) == L.LT_ERR_INVALID_ARG  # bad scale mode
+    assert lib.lt_dequant_int8(P, P, None, 1, 4, 4, P + 1, None) == L.LT_ERR_MISALIGNED
+    assert lib.lt_zrle_decode(P, 16, P, 100, 0, P, None, None) == L.LT_ERR_UNSUPPORTED
+    assert lib.lt_zrle_decode(P, 16, P, 100, 65536, P, None, None) == L.LT_ERR_UNSUPPORTED
+    assert lib.lt_zrle_decode(P, 16, P + 4, 100, 4096, P, None, None) == L.LT_ERR_MISALIGNED
+    assert lib.lt_zrle_decode(P, 16, P, -1, 4096, P, None, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_lz4_int4_decode(P, 16, P, 65537, P, None, 1, 8, 8, P, None, None) == L.LT_ERR_UNSUPPORTED
+    assert lib.lt_lz4_int4_decode(P, 16, P, 1000, P, None, 1, 8, 8, P, None, None) == L.LT_ERR_UNSUPPORTED
+    assert lib.lt_lz4_int4_decode(P, 16, P, 65536, P, None, 1, 8, 3, P, None, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_lz4_int4_decode(P, 16, P + 2, 65536, P, None, 1, 8, 8, P, None, None) == L.LT_ERR_MISALIGNED
+    assert lib.lt_lz4_decode(P, 16, P, 8, P, 100, None, None) == L.LT_ERR_UNSUPPORTED
+    arr = (L.LtLz4Int4Desc * 17)()
+    assert lib.lt_lz4_int4_decode_batch(arr, 17, None, None) == L.LT_ERR_UNSUPPORTED
+    assert lib.lt_lz4_int4_decode_batch(arr, 0, None, None) == L.LT_ERR_INVALID_ARG
+
+
+def test_binding_rejects_host_tensors():
+    torch = pytest.importorskip("torch")
+    x = torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(TypeError):
+        L.lt_dequant_int4(x, x, None, 1, 32, 32, x, stream=0)

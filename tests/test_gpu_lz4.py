@@ -1,0 +1,277 @@
+"""GPU parity: LZ4 block decoding (raw bytes, bit-exact) and the fused
+LZ4 -> INT4 -> fp16 decode (vs the oracle's decompress-then-dequantize)."""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from tests._gpu import assert_f16_parity, dev, f16_out, host_bits, need_gpu, status_buf, torch
+from tests._pins import hexbytes, liblz4, lz4_lib_compress
+from weight_dequantization_b200 import lt_decode as L
+from weight_dequantization_b200.synth import (fp16_uniform, int4_gauss_groups_packed, int4_uniform_packed,
+                                              lz4_compress_block, lz4_compress_blocks, u8_uniform)
+from weight_dequantization_b200.synth import workloads as W
+
+pytestmark = pytest.mark.gpu
+RNG = np.random.default_rng(13)
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    need_gpu()
+
+
+def run_raw(comp, offsets, block_bytes, out_bytes):
+    out = torch.full((out_bytes + 16,), 0xEE, dtype=torch.uint8, device="cuda")
+    stat = status_buf()
+    L.lt_lz4_decode(dev(comp) if comp.size else None, int(comp.size), dev(offsets), block_bytes, out, out_bytes,
+                    stat)
+    torch.cuda.synchronize()
+    o = out.cpu().numpy()
+    assert np.all(o[out_bytes:] == 0xEE), "write past the end of the output"
+    return o[:out_bytes], int(stat.item())
+
+
+def run_fused(d, zeros="use", out_offset=0):
+    z = d["zeros"] if zeros == "use" else None
+    n = d["rows"] * d["cols"]
+    out = f16_out(n, out_offset)
+    stat = status_buf()
+    L.lt_lz4_int4_decode(dev(d["comp"]), int(d["comp"].size), dev(d["offsets"]), d["block_bytes"], dev(d["scales"]),
+                         dev(z), d["rows"], d["cols"], d["group_size"], out, stat)
+    torch.cuda.synchronize()
+    return host_bits(out), int(stat.item())
+
+
+def oracle_fused(d, zeros="use"):
+    z = d["zeros"] if zeros == "use" else None
+    return oracle.lz4_int4_decode(d["comp"], d["offsets"], d["block_bytes"], d["scales"], z, d["rows"], d["cols"],
+                                  d["group_size"])
+
+
+def make_matrix(rows, cols, G, block_bytes, seed=1, law="gauss"):
+    n = rows * cols
+    packed = int4_gauss_groups_packed(seed, n) if law == "gauss" else int4_uniform_packed(seed, n)
+    comp, offs = lz4_compress_blocks(packed, block_bytes)
+    return dict(rows=rows, cols=cols, group_size=G, block_bytes=block_bytes, comp=comp, offsets=offs,
+                packed=packed, scales=fp16_uniform(seed, n // G, 0.001, 0.1, stream=1),
+                zeros=u8_uniform(seed, n // G, 0, 15, stream=2))
+
+
+# --------------------------------------------------------------------------- raw LZ4
+
+def test_lz4_handmade_blocks(golden_dir):
+    cases = json.load(open(os.path.join(golden_dir, "lz4_handmade.json")))["cases"]
+    for c in cases:
+        comp = np.frombuffer(hexbytes(c["comp"]), np.uint8)
+        if "out" in c:
+            want = hexbytes(c["out"])
+        elif "out_repeat" in c:
+            r = c["out_repeat"]
+            want = hexbytes(r["unit"]) * r["count"] + hexbytes(r["extra"]) + hexbytes(r["tail"])
+        else:
+            want = None
+        out_len = len(want) if want is not None else c["out_len"]
+        offs = np.array([0, comp.size], np.uint64)
+        bb = max(16, (out_len + 15) // 16 * 16)
+        got, st = run_raw(comp, offs, bb, out_len)
+        _, st_o = oracle.lz4_block_decode(comp, out_len)
+        assert st == st_o == c["status"], c["name"]
+        if want is not None:
+            assert got.tobytes() == want, c["name"]
+
+
+def test_lz4_raw_c4_full_size_bit_exact():
+    d = W.c4_lz4_int4(keep_packed=True)
+    got, st = run_raw(d["comp"], d["offsets"], d["block_bytes"], d["packed_bytes"])
+    assert st == 0
+    assert np.array_equal(got, d["packed"])
+
+
+@pytest.mark.parametrize("kind", ["0xab", "random_literals", "zeros", "max_offset"])
+def test_lz4_roadmap_64k_blocks(kind):
+    if kind == "0xab":          # the roadmap's 64 KB block of 0xAB
+        data = np.full(65536, 0xAB, np.uint8)
+        comp = lz4_compress_block(data)
+    elif kind == "random_literals":  # a block stored as literals only
+        data = RNG.integers(0, 256, 65536, dtype=np.uint8)
+        comp = lz4_compress_block(data, force_literals=True)
+    elif kind == "zeros":
+        data = np.zeros(65536, np.uint8)
+        comp = lz4_compress_block(data)
+    else:                        # the farthest match a 64 KB block can hold: offset 65500
+        head = RNG.integers(0, 256, 65500, dtype=np.uint8)
+        lit_ext = bytes([255] * ((65500 - 15) // 255)) + bytes([(65500 - 15) % 255])
+        comp = np.frombuffer(bytes([0xFF]) + lit_ext + head.tobytes() + (65500).to_bytes(2, "little")
+                             + bytes([31 - 4 - 15]) + bytes([0x50]) + b"tail!", np.uint8).copy()
+        data = np.concatenate([head, head[:31], np.frombuffer(b"tail!", np.uint8)])
+        assert data.size == 65536
+        want, st_o = oracle.lz4_block_decode(comp, data.size)
+        assert st_o == 0 and np.array_equal(want, data)
+    got, st = run_raw(comp, np.array([0, comp.size], np.uint64), 65536, data.size)
+    assert st == 0 and np.array_equal(got, data)
+
+
+@pytest.mark.skipif(liblz4() is None, reason="system liblz4 not present")
+def test_lz4_decodes_blocks_from_the_system_lz4_library():
+    blocks, raw = [], []
+    for i in range(24):
+        if i % 3 == 0:
+            data = int4_gauss_groups_packed(i, 131072).tobytes()
+        elif i % 3 == 1:
+            data = RNG.integers(0, 4, 65536, dtype=np.uint8).tobytes()
+        else:
+            words = [b"lz4", b"block", b"decode", b"b200", b"nibble"]
+            data = b"".join(words[j] for j in RNG.integers(0, 5, 20000))[:65536]
+        blocks.append(lz4_lib_compress(data))
+        raw.append(data)
+    comp = np.frombuffer(b"".join(blocks), np.uint8)
+    offs = np.concatenate([[0], np.cumsum([len(b) for b in blocks])]).astype(np.uint64)
+    got, st = run_raw(comp, offs, 65536, 24 * 65536)
+    assert st == 0
+    assert got.tobytes() == b"".join(raw)
+
+
+@pytest.mark.parametrize("n_bytes,block_bytes", [(1, 16), (100, 16), (5000, 4096), (200_001, 65536),
+                                                 (300_000, 16384), (65536 * 3, 65536)])
+def test_lz4_raw_ragged_sizes(n_bytes, block_bytes):
+    data = int4_gauss_groups_packed(n_bytes, 2 * n_bytes)[:n_bytes]
+    comp, offs = lz4_compress_blocks(data, block_bytes)
+    got, st = run_raw(comp, offs, block_bytes, n_bytes)
+    assert st == 0 and np.array_equal(got, data)
+
+
+def test_lz4_corrupt_blocks_match_oracle_status():
+    data = int4_gauss_groups_packed(77, 131072)
+    comp = lz4_compress_block(data)
+    seen = set()
+    for trial in range(80):
+        c = comp.copy()
+        if trial % 4 == 3:
+            c = c[: int(RNG.integers(1, c.size))]
+        else:
+            for _ in range(1 + trial % 3):
+                c[int(RNG.integers(0, c.size))] ^= np.uint8(1 << int(RNG.integers(0, 8)))
+        want, st_o = oracle.lz4_block_decode(c, data.size)
+        got, st_g = run_raw(c, np.array([0, c.size], np.uint64), 65536, data.size)
+        assert st_g == st_o, trial
+        seen.add(st_o)
+        if st_o == 0:
+            assert np.array_equal(got, want)
+    assert 4 in seen
+    # offsets outside the stream
+    got, st = run_raw(comp, np.array([0, comp.size + 10], np.uint64), 65536, data.size)
+    assert st == L.LT_ERR_CORRUPT_STREAM
+    got, st = run_raw(comp, np.array([10, 5], np.uint64), 65536, data.size)
+    assert st == L.LT_ERR_CORRUPT_STREAM
+
+
+# --------------------------------------------------------------------------- fused
+
+def test_fused_c4_full_size():
+    d = W.c4_lz4_int4()
+    want, st = oracle_fused(d)
+    assert st == 0
+    got, st_g = run_fused(d)
+    assert st_g == 0
+    assert_f16_parity(got, want, what="C4")
+
+
+@pytest.mark.parametrize("rows,cols,G,block_bytes,law,zeros,out_offset", [
+    (16, 8192, 128, 65536, "gauss", "use", 0),
+    (16, 8192, 128, 65536, "gauss", None, 0),
+    (8, 4096, 256, 16384, "uniform", "use", 0),
+    (3, 4000, 8, 4096, "gauss", "use", 0),
+    (5, 4002, 6, 4096, "gauss", "use", 0),        # groups not a multiple of 8: scalar epilogue
+    (7, 4001, 4001, 16, "uniform", "use", 0),     # odd element count, tiny blocks
+    (4, 4096, 128, 65536, "gauss", "use", 3),     # unaligned output
+    (33, 2048, 64, 32768, "gauss", "use", 0),     # ragged last block
+])
+def test_fused_shapes(rows, cols, G, block_bytes, law, zeros, out_offset):
+    d = make_matrix(rows, cols, G, block_bytes, seed=rows * cols, law=law)
+    want, st = oracle_fused(d, zeros)
+    assert st == 0
+    got, st_g = run_fused(d, zeros, out_offset)
+    assert st_g == 0
+    assert_f16_parity(got, want, what=f"{rows}x{cols}/G{G}/B{block_bytes}")
+
+
+def test_fused_corrupt_stream_reports_and_stays_in_bounds():
+    d = make_matrix(16, 8192, 128, 65536, seed=3)
+    d["comp"] = d["comp"].copy()
+    d["comp"][100] ^= 0xFF
+    d["comp"][5000] ^= 0x5A
+    n = d["rows"] * d["cols"]
+    buf = torch.full((n + 64,), 7.0, dtype=torch.float16, device="cuda")
+    out = buf[:n]
+    stat = status_buf()
+    L.lt_lz4_int4_decode(dev(d["comp"]), int(d["comp"].size), dev(d["offsets"]), 65536, dev(d["scales"]),
+                         dev(d["zeros"]), d["rows"], d["cols"], 128, out, stat)
+    torch.cuda.synchronize()
+    _, st_o = oracle_fused(d)
+    assert int(stat.item()) == st_o != 0
+    assert torch.all(buf[n:] == 7.0)
+
+
+def test_fused_batch_matches_per_matrix_oracle():
+    # a Llama-shaped layer at 1/64 of the rows, one launch for all matrices
+    mats = W.c5_layers(layers=1, scale=1 / 64)[0]
+    outs, descs = [], []
+    dev_refs = []
+    for m in mats:
+        n = m["rows"] * m["cols"]
+        out = f16_out(n)
+        refs = [dev(m["comp"]), dev(m["offsets"]), dev(m["scales"]), dev(m["zeros"])]
+        dev_refs.append(refs)
+        descs.append(dict(comp=refs[0], comp_bytes=int(m["comp"].size), block_offsets=refs[1], scales=refs[2],
+                          zeros=refs[3], out=out, rows=m["rows"], cols=m["cols"], group_size=m["group_size"],
+                          block_bytes=m["block_bytes"]))
+        outs.append(out)
+    stat = status_buf()
+    L.lt_lz4_int4_decode_batch(descs, stat)
+    torch.cuda.synchronize()
+    assert int(stat.item()) == 0
+    for m, out in zip(mats, outs):
+        want, st = oracle_fused(m)
+        assert st == 0
+        assert_f16_parity(host_bits(out), want, what=m["name"])
+
+
+def test_fused_full_c5_layer_sampled_blocks():
+    # one full-size layer in one launch (as the benchmark runs it); the oracle
+    # checks a random sample of 64 KB blocks of every matrix one by one
+    mats = W.c5_layers(layers=1)[0]
+    total = sum(m["rows"] * m["cols"] for m in mats)
+    buf = torch.empty(total, dtype=torch.float16, device="cuda")
+    descs, keep, base = [], [], 0
+    for m in mats:
+        n = m["rows"] * m["cols"]
+        refs = [dev(m["comp"]), dev(m["offsets"]), dev(m["scales"]), dev(m["zeros"])]
+        keep.append(refs)
+        descs.append(dict(comp=refs[0], comp_bytes=int(m["comp"].size), block_offsets=refs[1], scales=refs[2],
+                          zeros=refs[3], out=buf[base:base + n], rows=m["rows"], cols=m["cols"],
+                          group_size=m["group_size"], block_bytes=m["block_bytes"]))
+        m["base"] = base
+        base += n
+    stat = status_buf()
+    L.lt_lz4_int4_decode_batch(descs, stat)
+    torch.cuda.synchronize()
+    assert int(stat.item()) == 0
+    codes_per_block = 2 * 65536
+    for m in mats:
+        n_blocks = len(m["offsets"]) - 1
+        for b in RNG.choice(n_blocks, size=min(12, n_blocks), replace=False):
+            s0, s1 = int(m["offsets"][b]), int(m["offsets"][b + 1])
+            g0 = b * codes_per_block // 128
+            sub = dict(comp=m["comp"][s0:s1], offsets=np.array([0, s1 - s0], np.uint64), block_bytes=65536,
+                       scales=m["scales"][g0:g0 + 1024], zeros=m["zeros"][g0:g0 + 1024], rows=1,
+                       cols=codes_per_block, group_size=128)
+            want, st = oracle_fused(sub)
+            assert st == 0
+            k0 = m["base"] + b * codes_per_block
+            got = host_bits(buf[k0:k0 + codes_per_block])
+            assert_f16_parity(got, want, what=f"{m['name']} block {b}")

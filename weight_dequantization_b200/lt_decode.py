@@ -1,0 +1,160 @@
+"""Python binding of liblt_decode.so (ctypes; argument marshalling only).
+
+Every function has the name and the arguments of the C entry point declared
+in ``include/lt_decode.h``. Tensor arguments are CUDA tensors (their device
+pointers are passed) or raw integer device addresses; ``None`` is NULL. The
+stream defaults to PyTorch's current stream on the output's device. A non-OK
+status raises :class:`LtError`. There is no CPU path: CPU tensors are
+rejected, and a missing or unloadable library raises at import of this
+module's first call.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblt_decode.so")
+
+LT_OK = 0
+LT_ERR_INVALID_ARG = 1
+LT_ERR_MISALIGNED = 2
+LT_ERR_UNSUPPORTED = 3
+LT_ERR_CORRUPT_STREAM = 4
+LT_ERR_SIZE_MISMATCH = 5
+LT_ERR_CUDA = 6
+LT_SCALE_PER_TENSOR = 0
+LT_SCALE_PER_ROW = 1
+LT_LZ4_BATCH_MAX = 16
+
+EXPORTED = (
+    "lt_dequant_int4", "lt_dequant_int8", "lt_zrle_decode", "lt_lz4_int4_decode",
+    "lt_lz4_int4_decode_batch", "lt_lz4_decode", "lt_status_string", "lt_abi_version",
+)
+
+
+class LtError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class LtLz4Int4Desc(ctypes.Structure):
+    _fields_ = [
+        ("comp", ctypes.c_void_p), ("comp_bytes", ctypes.c_uint64), ("block_offsets", ctypes.c_void_p),
+        ("scales", ctypes.c_void_p), ("zeros", ctypes.c_void_p), ("out", ctypes.c_void_p),
+        ("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("group_size", ctypes.c_int32),
+        ("block_bytes", ctypes.c_int32),
+    ]
+
+
+_lib = None
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load liblt_decode.so (no compute; works without a GPU)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"{p} is not built: run __graft_entry__.build() (the decoders have no CPU fallback)")
+    lib = ctypes.CDLL(p)
+    P, U64, I64, I32 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int64, ctypes.c_int32
+    lib.lt_dequant_int4.argtypes = [P, P, P, I64, I64, I32, P, P]
+    lib.lt_dequant_int8.argtypes = [P, P, P, I32, I64, I64, P, P]
+    lib.lt_zrle_decode.argtypes = [P, U64, P, I64, I32, P, P, P]
+    lib.lt_lz4_int4_decode.argtypes = [P, U64, P, I32, P, P, I64, I64, I32, P, P, P]
+    lib.lt_lz4_int4_decode_batch.argtypes = [ctypes.POINTER(LtLz4Int4Desc), I32, P, P]
+    lib.lt_lz4_decode.argtypes = [P, U64, P, I32, P, U64, P, P]
+    for f in ("lt_dequant_int4", "lt_dequant_int8", "lt_zrle_decode", "lt_lz4_int4_decode",
+              "lt_lz4_int4_decode_batch", "lt_lz4_decode"):
+        getattr(lib, f).restype = ctypes.c_int
+    lib.lt_status_string.argtypes = [ctypes.c_int]
+    lib.lt_status_string.restype = ctypes.c_char_p
+    lib.lt_abi_version.argtypes = []
+    lib.lt_abi_version.restype = I32
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().lt_status_string(int(status)).decode()
+
+
+def abi_version() -> int:
+    return int(load_library().lt_abi_version())
+
+
+def _ptr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    dev = getattr(x, "device", None)
+    if dev is None or dev.type != "cuda":
+        raise TypeError("liblt_decode takes CUDA tensors or device addresses (there is no CPU path)")
+    if not x.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return x.data_ptr()
+
+
+def _stream(stream, like) -> int | None:
+    if stream is None:
+        import torch
+
+        dev = getattr(like, "device", None)
+        s = torch.cuda.current_stream(dev if dev is not None and dev.type == "cuda" else None)
+        return s.cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str) -> None:
+    if status != LT_OK:
+        raise LtError(status, where)
+
+
+def lt_dequant_int4(packed, scales, zeros, rows: int, cols: int, group_size: int, out, stream=None) -> None:
+    _check(load_library().lt_dequant_int4(_ptr(packed), _ptr(scales), _ptr(zeros), rows, cols, group_size,
+                                          _ptr(out), _stream(stream, out)), "lt_dequant_int4")
+
+
+def lt_dequant_int8(q, scales, zeros, scale_mode: int, rows: int, cols: int, out, stream=None) -> None:
+    _check(load_library().lt_dequant_int8(_ptr(q), _ptr(scales), _ptr(zeros), scale_mode, rows, cols, _ptr(out),
+                                          _stream(stream, out)), "lt_dequant_int8")
+
+
+def lt_zrle_decode(enc, enc_bytes: int, chunk_offsets, n_elements: int, chunk_elems: int, out, d_status=None,
+                   stream=None) -> None:
+    _check(load_library().lt_zrle_decode(_ptr(enc), enc_bytes, _ptr(chunk_offsets), n_elements, chunk_elems,
+                                         _ptr(out), _ptr(d_status), _stream(stream, out)), "lt_zrle_decode")
+
+
+def lt_lz4_int4_decode(comp, comp_bytes: int, block_offsets, block_bytes: int, scales, zeros, rows: int, cols: int,
+                       group_size: int, out, d_status=None, stream=None) -> None:
+    _check(load_library().lt_lz4_int4_decode(_ptr(comp), comp_bytes, _ptr(block_offsets), block_bytes,
+                                             _ptr(scales), _ptr(zeros), rows, cols, group_size, _ptr(out),
+                                             _ptr(d_status), _stream(stream, out)), "lt_lz4_int4_decode")
+
+
+def lt_lz4_int4_decode_batch(descs: Sequence[dict], d_status=None, stream=None) -> None:
+    """``descs``: dicts with the keys of lt_lz4_int4_desc (tensors or addresses)."""
+    n = len(descs)
+    arr = (LtLz4Int4Desc * max(n, 1))()
+    for i, d in enumerate(descs):
+        arr[i] = LtLz4Int4Desc(_ptr(d["comp"]), d["comp_bytes"], _ptr(d["block_offsets"]), _ptr(d["scales"]),
+                               _ptr(d.get("zeros")), _ptr(d["out"]), d["rows"], d["cols"], d["group_size"],
+                               d["block_bytes"])
+    like = descs[0]["out"] if n else None
+    _check(load_library().lt_lz4_int4_decode_batch(arr, n, _ptr(d_status), _stream(stream, like)),
+           "lt_lz4_int4_decode_batch")
+
+
+def lt_lz4_decode(comp, comp_bytes: int, block_offsets, block_bytes: int, out, out_bytes: int, d_status=None,
+                  stream=None) -> None:
+    _check(load_library().lt_lz4_decode(_ptr(comp), comp_bytes, _ptr(block_offsets), block_bytes, _ptr(out),
+                                        out_bytes, _ptr(d_status), _stream(stream, out)), "lt_lz4_decode")
