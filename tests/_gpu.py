@@ -20,7 +20,7 @@ def dev(a: np.ndarray | None):
     """numpy -> contiguous CUDA tensor with the same bytes (None stays None)."""
     if a is None:
         return None
-    a = np.ascontiguousarray(a)
+    a = np.array(a, copy=True, order="C")
     if a.dtype == np.uint16:
         a = a.view(np.int16)
     elif a.dtype == np.uint64:
