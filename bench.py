@@ -61,6 +61,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=8, help="C5 layers (8 is the workload)")
+    ap.add_argument("--only", default="C1,C2,C3,C4,C5",
+                    help="comma-separated subset of the workloads to run (profiling); the bench line uses all")
     return ap.parse_args()
 
 
@@ -176,18 +178,19 @@ def gpu_id_for(dev_index: int) -> str:
 # workloads
 # ----------------------------------------------------------------------------
 
-def build_host_workload(rank: int, layers: int):
+def build_host_workload(rank: int, layers: int, only=("C1", "C2", "C3", "C4", "C5")):
     """Seeded host inputs; each rank gets its own seeds (weak scaling)."""
     from weight_dequantization_b200.synth import workloads as W
 
     off = 1000 * rank
-    return {
-        "C1": W.c1_int4(seed=1 + off),
-        "C2": W.c2_int8(seed=2 + off),
-        "C3": W.c3_zrle(seed=3 + off),
-        "C4": W.c4_lz4_int4(seed=4 + off),
-        "C5": W.c5_layers(layers=layers, seed=5 + off),
+    make = {
+        "C1": lambda: W.c1_int4(seed=1 + off),
+        "C2": lambda: W.c2_int8(seed=2 + off),
+        "C3": lambda: W.c3_zrle(seed=3 + off),
+        "C4": lambda: W.c4_lz4_int4(seed=4 + off),
+        "C5": lambda: W.c5_layers(layers=layers, seed=5 + off),
     }
+    return {k: make[k]() for k in ("C1", "C2", "C3", "C4", "C5") if k in only}
 
 
 def nbytes(a) -> int:
@@ -196,22 +199,28 @@ def nbytes(a) -> int:
 
 def algorithmic_bytes(hw):
     """Bytes the method must read + write per codec (actual buffers)."""
-    c1, c2, c3, c4 = hw["C1"], hw["C2"], hw["C3"], hw["C4"]
-    n1 = c1["rows"] * c1["cols"]
-    n2 = c2["rows"] * c2["cols"]
-    out = {
-        "C1": (nbytes(c1["packed"]) + nbytes(c1["scales"]) + nbytes(c1["zeros"]), 2 * n1),
-        "C2": (nbytes(c2["q"]) + nbytes(c2["scales"]) + nbytes(c2["zeros"]), 2 * n2),
-        "C3": (nbytes(c3["enc"]) + nbytes(c3["offsets"]), 2 * c3["n"]),
-        "C4": (nbytes(c4["comp"]) + nbytes(c4["offsets"]) + nbytes(c4["scales"]) + nbytes(c4["zeros"]),
-               2 * c4["rows"] * c4["cols"]),
-    }
+    out = {}
+    if "C1" in hw:
+        c1 = hw["C1"]
+        out["C1"] = (nbytes(c1["packed"]) + nbytes(c1["scales"]) + nbytes(c1["zeros"]), 2 * c1["rows"] * c1["cols"])
+    if "C2" in hw:
+        c2 = hw["C2"]
+        out["C2"] = (nbytes(c2["q"]) + nbytes(c2["scales"]) + nbytes(c2["zeros"]), 2 * c2["rows"] * c2["cols"])
+    if "C3" in hw:
+        c3 = hw["C3"]
+        out["C3"] = (nbytes(c3["enc"]) + nbytes(c3["offsets"]), 2 * c3["n"])
+    if "C4" in hw:
+        c4 = hw["C4"]
+        out["C4"] = (nbytes(c4["comp"]) + nbytes(c4["offsets"]) + nbytes(c4["scales"]) + nbytes(c4["zeros"]),
+                     2 * c4["rows"] * c4["cols"])
     layer = []
-    for mats in hw["C5"]:
-        rd = sum(nbytes(m["comp"]) + nbytes(m["offsets"]) + nbytes(m["scales"]) + nbytes(m["zeros"]) for m in mats)
-        wr = sum(2 * m["rows"] * m["cols"] for m in mats)
-        layer.append((rd, wr))
-    out["C5"] = (sum(r for r, _ in layer), sum(w for _, w in layer))
+    if "C5" in hw:
+        for mats in hw["C5"]:
+            rd = sum(nbytes(m["comp"]) + nbytes(m["offsets"]) + nbytes(m["scales"]) + nbytes(m["zeros"])
+                     for m in mats)
+            wr = sum(2 * m["rows"] * m["cols"] for m in mats)
+            layer.append((rd, wr))
+        out["C5"] = (sum(r for r, _ in layer), sum(w for _, w in layer))
     return out, layer
 
 
@@ -243,29 +252,37 @@ class DeviceWorkload:
                 self.h2d.append((ph, d))
             return d
 
-        c1, c2, c3, c4 = hw["C1"], hw["C2"], hw["C3"], hw["C4"]
-        self.c1 = dict(packed=put(c1["packed"]), scales=put(c1["scales"]), zeros=put(c1["zeros"]))
-        self.c1_out = torch.empty(c1["rows"] * c1["cols"], dtype=torch.float16, device="cuda")
-        self.c2 = dict(q=put(c2["q"]), scales=put(c2["scales"]))
-        self.c2_out = torch.empty(c2["rows"] * c2["cols"], dtype=torch.float16, device="cuda")
-        self.c3 = dict(enc=put(c3["enc"]), offsets=put(c3["offsets"]))
-        self.c3_out = torch.empty(c3["n"], dtype=torch.float16, device="cuda")
-        self.c4 = dict(comp=put(c4["comp"]), offsets=put(c4["offsets"]), scales=put(c4["scales"]),
-                       zeros=put(c4["zeros"]))
-        self.c4_out = torch.empty(c4["rows"] * c4["cols"], dtype=torch.float16, device="cuda")
-        layer_elems = max(sum(m["rows"] * m["cols"] for m in mats) for mats in hw["C5"])
-        self.c5_out = torch.empty(layer_elems, dtype=torch.float16, device="cuda")  # one reused layer buffer
+        if "C1" in hw:
+            c1 = hw["C1"]
+            self.c1 = dict(packed=put(c1["packed"]), scales=put(c1["scales"]), zeros=put(c1["zeros"]))
+            self.c1_out = torch.empty(c1["rows"] * c1["cols"], dtype=torch.float16, device="cuda")
+        if "C2" in hw:
+            c2 = hw["C2"]
+            self.c2 = dict(q=put(c2["q"]), scales=put(c2["scales"]))
+            self.c2_out = torch.empty(c2["rows"] * c2["cols"], dtype=torch.float16, device="cuda")
+        if "C3" in hw:
+            c3 = hw["C3"]
+            self.c3 = dict(enc=put(c3["enc"]), offsets=put(c3["offsets"]))
+            self.c3_out = torch.empty(c3["n"], dtype=torch.float16, device="cuda")
+        if "C4" in hw:
+            c4 = hw["C4"]
+            self.c4 = dict(comp=put(c4["comp"]), offsets=put(c4["offsets"]), scales=put(c4["scales"]),
+                           zeros=put(c4["zeros"]))
+            self.c4_out = torch.empty(c4["rows"] * c4["cols"], dtype=torch.float16, device="cuda")
         self.c5 = []
-        for mats in hw["C5"]:
-            descs, base = [], 0
-            for m in mats:
-                n = m["rows"] * m["cols"]
-                descs.append(dict(comp=put(m["comp"]), comp_bytes=int(m["comp"].size), block_offsets=put(m["offsets"]),
-                                  scales=put(m["scales"]), zeros=put(m["zeros"]), out=self.c5_out[base:base + n],
-                                  rows=m["rows"], cols=m["cols"], group_size=m["group_size"],
-                                  block_bytes=m["block_bytes"]))
-                base += n
-            self.c5.append(descs)
+        if "C5" in hw:
+            layer_elems = max(sum(m["rows"] * m["cols"] for m in mats) for mats in hw["C5"])
+            self.c5_out = torch.empty(layer_elems, dtype=torch.float16, device="cuda")  # one reused layer buffer
+            for mats in hw["C5"]:
+                descs, base = [], 0
+                for m in mats:
+                    n = m["rows"] * m["cols"]
+                    descs.append(dict(comp=put(m["comp"]), comp_bytes=int(m["comp"].size),
+                                      block_offsets=put(m["offsets"]), scales=put(m["scales"]),
+                                      zeros=put(m["zeros"]), out=self.c5_out[base:base + n], rows=m["rows"],
+                                      cols=m["cols"], group_size=m["group_size"], block_bytes=m["block_bytes"]))
+                    base += n
+                self.c5.append(descs)
         self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
         self.status_host = torch.zeros(1, dtype=torch.int32).pin_memory() if pinned else None
         self.h2d_bytes = sum(int(p.numel() * p.element_size()) for p, _ in self.h2d)
@@ -284,25 +301,38 @@ class DeviceWorkload:
                 e.record(s)
                 ev.setdefault(key, []).append(e)
 
-        c1, c2, c3, c4 = hw["C1"], hw["C2"], hw["C3"], hw["C4"]
-        mark("C1.start")
-        L.lt_dequant_int4(self.c1["packed"], self.c1["scales"], self.c1["zeros"], c1["rows"], c1["cols"],
-                          c1["group_size"], self.c1_out, s)
-        mark("C1.end")
-        L.lt_dequant_int8(self.c2["q"], self.c2["scales"], None, L.LT_SCALE_PER_ROW, c2["rows"], c2["cols"],
-                          self.c2_out, s)
-        mark("C2.end")
-        L.lt_zrle_decode(self.c3["enc"], int(c3["enc"].size), self.c3["offsets"], c3["n"], c3["chunk_elems"],
-                         self.c3_out, self.status, s)
-        mark("C3.end")
-        L.lt_lz4_int4_decode(self.c4["comp"], int(c4["comp"].size), self.c4["offsets"], c4["block_bytes"],
-                             self.c4["scales"], self.c4["zeros"], c4["rows"], c4["cols"], c4["group_size"],
-                             self.c4_out, self.status, s)
-        mark("C4.end")
-        for i, descs in enumerate(self.c5):
+        mark("start")
+        n = 0
+        if "C1" in hw:
+            c1 = hw["C1"]
+            L.lt_dequant_int4(self.c1["packed"], self.c1["scales"], self.c1["zeros"], c1["rows"], c1["cols"],
+                              c1["group_size"], self.c1_out, s)
+            mark("C1")
+            n += 1
+        if "C2" in hw:
+            c2 = hw["C2"]
+            L.lt_dequant_int8(self.c2["q"], self.c2["scales"], None, L.LT_SCALE_PER_ROW, c2["rows"], c2["cols"],
+                              self.c2_out, s)
+            mark("C2")
+            n += 1
+        if "C3" in hw:
+            c3 = hw["C3"]
+            L.lt_zrle_decode(self.c3["enc"], int(c3["enc"].size), self.c3["offsets"], c3["n"], c3["chunk_elems"],
+                             self.c3_out, self.status, s)
+            mark("C3")
+            n += 1
+        if "C4" in hw:
+            c4 = hw["C4"]
+            L.lt_lz4_int4_decode(self.c4["comp"], int(c4["comp"].size), self.c4["offsets"], c4["block_bytes"],
+                                 self.c4["scales"], self.c4["zeros"], c4["rows"], c4["cols"], c4["group_size"],
+                                 self.c4_out, self.status, s)
+            mark("C4")
+            n += 1
+        for descs in self.c5:
             L.lt_lz4_int4_decode_batch(descs, self.status, s)
-            mark("C5.layer")
-        return 4 + len(self.c5)  # kernel launches of this step
+            mark("C5")
+            n += 1
+        return n  # kernel launches of this step
 
     def upload_inputs(self):
         for ph, d in self.h2d:
@@ -315,10 +345,17 @@ class DeviceWorkload:
 def launches_per_step(hw) -> int:
     # every call takes its vector path (no scalar tail launch): all element
     # counts are multiples of 8, groups multiples of 8, buffers 256-byte aligned
-    c1, c2 = hw["C1"], hw["C2"]
-    assert (c1["rows"] * c1["cols"]) % 8 == 0 and c1["group_size"] % 8 == 0
-    assert (c2["rows"] * c2["cols"]) % 8 == 0 and c2["cols"] % 8 == 0
-    return 4 + len(hw["C5"])
+    n = 0
+    if "C1" in hw:
+        c1 = hw["C1"]
+        assert (c1["rows"] * c1["cols"]) % 8 == 0 and c1["group_size"] % 8 == 0
+        n += 1
+    if "C2" in hw:
+        c2 = hw["C2"]
+        assert (c2["rows"] * c2["cols"]) % 8 == 0 and c2["cols"] % 8 == 0
+        n += 1
+    n += ("C3" in hw) + ("C4" in hw) + len(hw.get("C5", []))
+    return n
 
 
 # ----------------------------------------------------------------------------
@@ -334,22 +371,25 @@ def oracle_sample_step(hw, frac: float):
 
     t0 = time.perf_counter()
     dec = 0
-    c1 = hw["C1"]
-    r1 = max(1, int(c1["rows"] * frac))
-    n1 = r1 * c1["cols"]
-    g1 = n1 // c1["group_size"]
-    oracle.dequant_int4(c1["packed"][: n1 // 2], c1["scales"][:g1], c1["zeros"][:g1], r1, c1["cols"],
-                        c1["group_size"])
-    dec += 2 * n1
-    c2 = hw["C2"]
-    r2 = max(1, int(c2["rows"] * frac))
-    oracle.dequant_int8(c2["q"][: r2 * c2["cols"]], c2["scales"][:r2], None, True, r2, c2["cols"])
-    dec += 2 * r2 * c2["cols"]
-    c3 = hw["C3"]
-    nch = max(1, int((len(c3["offsets"]) - 1) * frac))
-    n3 = min(c3["n"], nch * c3["chunk_elems"])
-    oracle.zrle_decode(c3["enc"], c3["offsets"][: nch + 1], n3, c3["chunk_elems"])
-    dec += 2 * n3
+    if "C1" in hw:
+        c1 = hw["C1"]
+        r1 = max(1, int(c1["rows"] * frac))
+        n1 = r1 * c1["cols"]
+        g1 = n1 // c1["group_size"]
+        oracle.dequant_int4(c1["packed"][: n1 // 2], c1["scales"][:g1], c1["zeros"][:g1], r1, c1["cols"],
+                            c1["group_size"])
+        dec += 2 * n1
+    if "C2" in hw:
+        c2 = hw["C2"]
+        r2 = max(1, int(c2["rows"] * frac))
+        oracle.dequant_int8(c2["q"][: r2 * c2["cols"]], c2["scales"][:r2], None, True, r2, c2["cols"])
+        dec += 2 * r2 * c2["cols"]
+    if "C3" in hw:
+        c3 = hw["C3"]
+        nch = max(1, int((len(c3["offsets"]) - 1) * frac))
+        n3 = min(c3["n"], nch * c3["chunk_elems"])
+        oracle.zrle_decode(c3["enc"], c3["offsets"][: nch + 1], n3, c3["chunk_elems"])
+        dec += 2 * n3
 
     def lz4_part(m):
         nb = max(1, int((len(m["offsets"]) - 1) * frac))
@@ -360,8 +400,9 @@ def oracle_sample_step(hw, frac: float):
                                m["zeros"][:g], 1, codes, m["group_size"])
         return 2 * codes
 
-    dec += lz4_part(hw["C4"])
-    for mats in hw["C5"]:
+    if "C4" in hw:
+        dec += lz4_part(hw["C4"])
+    for mats in hw.get("C5", []):
         for m in mats:
             dec += lz4_part(m)
     return dec, time.perf_counter() - t0
@@ -396,14 +437,20 @@ def read_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def workload_config(hw, layers):
-    c5_codes = sum(m["rows"] * m["cols"] for mats in hw["C5"] for m in mats)
+def workload_config(hw, layers, only=("C1", "C2", "C3", "C4", "C5")):
+    c5_codes = sum(m["rows"] * m["cols"] for mats in hw.get("C5", []) for m in mats)
+    parts = {
+        "C1": "C1 INT4 1M codes G256",
+        "C2": "C2 INT8 8192x8192 per-row",
+        "C3": "C3 zero-run 8x2048x11008",
+        "C4": "C4 LZ4+INT4 4096x14336 G128",
+        "C5": f"C5 {layers}-layer Llama-2-70B-shaped LZ4+INT4 G128 sweep (one reused layer buffer)",
+    }
     return {
-        "workload": "decode suite: C1 INT4 1M codes G256 + C2 INT8 8192x8192 per-row + C3 zero-run 8x2048x11008 "
-                    f"+ C4 LZ4+INT4 4096x14336 G128 + C5 {layers}-layer Llama-2-70B-shaped LZ4+INT4 G128 sweep "
-                    "(64 KB LZ4 blocks, one reused layer buffer)",
+        "workload": "decode suite: " + " + ".join(parts[c] for c in parts if c in only) + " (64 KB LZ4 blocks)",
         "c5_codes": c5_codes,
-        "l2": "inputs larger than L2 (each step touches ~16 GB; no flush)",
+        "l2": "inputs larger than L2 (each step touches ~16 GB; no flush)" if "C5" in only else
+              "subset run: inputs may stay in L2 between steps",
     }
 
 
@@ -415,7 +462,8 @@ def run_lt(args, rank, world, local):
     from weight_dequantization_b200 import lt_decode as L
 
     L.load_library()
-    hw = build_host_workload(rank, args.layers)
+    only = tuple(x.strip() for x in args.only.split(",") if x.strip())
+    hw = build_host_workload(rank, args.layers, only)
     (alg, layer_alg) = algorithmic_bytes(hw)
     dw = DeviceWorkload(hw, pinned=True)
     nlaunch = launches_per_step(hw)
@@ -450,23 +498,24 @@ def run_lt(args, rank, world, local):
     elapsed = e0.elapsed_time(e1) / 1e3
     elapsed = max_over_ranks(elapsed, dist)
 
-    # per codec (device time of the launches, summed over steps)
+    # per codec (device time of the launches, summed over steps): events are
+    # recorded at the step start and after every launch, in launch order
     K = args.steps
-    t_c = {"C1": 0.0, "C2": 0.0, "C3": 0.0, "C4": 0.0, "C5": 0.0}
+    order = [c for c in ("C1", "C2", "C3", "C4") if c in hw] + ["C5"] * len(dw.c5)
+    t_c = {c: 0.0 for c in alg}
     layer_t = []
-    L5 = len(dw.c5)
+    idx = {c: 0 for c in set(order)}
     for k in range(K):
-        t_c["C1"] += ev["C1.start"][k].elapsed_time(ev["C1.end"][k])
-        t_c["C2"] += ev["C1.end"][k].elapsed_time(ev["C2.end"][k])
-        t_c["C3"] += ev["C2.end"][k].elapsed_time(ev["C3.end"][k])
-        t_c["C4"] += ev["C3.end"][k].elapsed_time(ev["C4.end"][k])
-        prev = ev["C4.end"][k]
-        for li in range(L5):
-            cur = ev["C5.layer"][k * L5 + li]
+        prev = ev["start"][k]
+        for c in order:
+            cur = ev[c][idx[c]]
+            idx[c] += 1
             dt = prev.elapsed_time(cur)
-            layer_t.append(dt)
-            t_c["C5"] += dt
+            t_c[c] += dt
+            if c == "C5":
+                layer_t.append(dt)
             prev = cur
+    L5 = max(1, len(dw.c5))
     peak, peak_kind = read_peaks()
     per_codec = {}
     for c, (rd, wr) in alg.items():
@@ -479,16 +528,28 @@ def run_lt(args, rank, world, local):
     total_decoded = sum_over_ranks(decoded * K, dist)
     value = total_decoded / elapsed / 1e9
 
-    # roofline of the dominant kernel: the fused LZ4 decode, one launch per C5 layer
-    avg_layer_s = statistics.mean(layer_t) / 1e3
-    layer_bytes = statistics.mean([rd + wr for rd, wr in layer_alg])
-    achieved = layer_bytes / avg_layer_s / 1e9
+    # roofline of the dominant kernel: the fused LZ4 decode, one launch per
+    # C5 layer (the C4 launch when C5 is not run)
+    if layer_t:
+        avg_s = statistics.mean(layer_t) / 1e3
+        launch_bytes = statistics.mean([rd + wr for rd, wr in layer_alg])
+        kname = "k_lz4<fused> (C5 layer, 7 matrices per launch)"
+    elif "C4" in alg:
+        avg_s = t_c["C4"] / 1e3 / K
+        launch_bytes = sum(alg["C4"])
+        kname = "k_lz4<fused> (C4)"
+    else:
+        c0 = next(iter(alg))
+        avg_s = t_c[c0] / 1e3 / K
+        launch_bytes = sum(alg[c0])
+        kname = c0
+    achieved = launch_bytes / avg_s / 1e9
     traffic = None
-    if NCU_TRAFFIC["sources_sha256"] == kernel_sources_sha() and NCU_TRAFFIC["bytes_per_launch"]:
+    if NCU_TRAFFIC["sources_sha256"] == kernel_sources_sha() and NCU_TRAFFIC["bytes_per_launch"] and layer_t:
         traffic = NCU_TRAFFIC["bytes_per_launch"]
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": traffic, "kernel": "k_lz4<fused> (C5 layer, 7 matrices per launch)",
-                "peak_kind": peak_kind, "algorithmic_bytes_per_launch": layer_bytes,
+                "traffic": traffic, "kernel": kname,
+                "peak_kind": peak_kind, "algorithmic_bytes_per_launch": launch_bytes,
                 "frac_of_8TBps": achieved / NOMINAL_HBM_GBS}
 
     # end-to-end: inputs copied from pinned host memory every step, status read back
@@ -523,7 +584,7 @@ def run_lt(args, rank, world, local):
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": elapsed / K * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f16", "data": "synthetic (seeded generators; value laws of the workloads)",
-            "config": workload_config(hw, args.layers), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "config": workload_config(hw, args.layers, only), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": nlaunch * K, "clocks": {"sm_mhz": ck["sm_mhz"], "sm_max_mhz": ck["sm_max_mhz"],
                                                      "reasons": ck["reasons"], "samples": ck["samples"]},
             "per_codec": per_codec, "impl": "lt",
@@ -540,7 +601,8 @@ def run_reference(args, rank, world):
     within a few minutes."""
     if rank != 0:
         return None
-    hw = build_host_workload(0, args.layers)
+    only = tuple(x.strip() for x in args.only.split(",") if x.strip())
+    hw = build_host_workload(0, args.layers, only)
     steps = args.steps + args.warmup
     # calibrate: aim at ~90 s for all steps together
     dec, dt = oracle_sample_step(hw, 1.0 / 4096)
@@ -560,7 +622,7 @@ def run_reference(args, rank, world):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": tot_t / max(args.steps, 1) * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(hw, args.layers), "impl": "reference",
+        "config": workload_config(hw, args.layers, only), "impl": "reference",
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

@@ -64,7 +64,8 @@ typedef enum {
   LT_ERR_UNSUPPORTED = 3,    /* valid request outside what the kernels implement */
   LT_ERR_CORRUPT_STREAM = 4, /* (device status) malformed LZ4 / zero-run data */
   LT_ERR_SIZE_MISMATCH = 5,  /* (device status) stream decodes to a different length */
-  LT_ERR_CUDA = 6            /* a CUDA launch failed */
+  LT_ERR_CUDA = 6,           /* a CUDA launch failed */
+  LT_ERR_TIMEOUT = 7         /* (device status) an internal on-chip wait ran out; never expected */
 } lt_status;
 
 typedef enum { LT_SCALE_PER_TENSOR = 0, LT_SCALE_PER_ROW = 1 } lt_scale_mode;

@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_abi_version_and_status_strings(lib):
     assert L.abi_version() == 1
-    for code in range(7):
+    for code in range(8):
         s = L.status_string(code)
         assert s and s != "unknown status"
     assert L.status_string(99) == "unknown status"

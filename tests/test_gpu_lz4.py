@@ -283,3 +283,39 @@ def test_fused_full_c5_layer_sampled_blocks():
             k0 = m["base"] + b * codes_per_block
             got = host_bits(buf[k0:k0 + codes_per_block])
             assert_f16_parity(got, want, what=f"{m['name']} block {b}")
+
+
+@pytest.mark.parametrize("seed,n_blocks,block_bytes,last", [(1, 40, 65536, None), (2, 7, 65536, 12345),
+                                                             (3, 30, 16384, 999), (4, 300, 4096, None)])
+def test_lz4_random_sequence_blocks(seed, n_blocks, block_bytes, last):
+    # every match regime: offset 1, periodic 2..15, overlapping >= 16,
+    # non-overlapping and far offsets; literal runs of every length class
+    from tests._lz4gen import random_blocks
+    comp, offs, raw = random_blocks(seed, n_blocks, block_bytes, last)
+    got, st = run_raw(comp, offs, block_bytes, raw.size)
+    assert st == 0
+    assert np.array_equal(got, raw)
+    # and through the fused path: raw bytes are the packed codes
+    n = 2 * raw.size
+    G = 64 if n % 64 == 0 else 2
+    d = dict(rows=1, cols=n, group_size=G, block_bytes=block_bytes, comp=comp, offsets=offs,
+             scales=fp16_uniform(seed, n // G, -0.5, 0.5, stream=1), zeros=u8_uniform(seed, n // G, 0, 15, stream=2))
+    want, st_o = oracle_fused(d)
+    assert st_o == 0
+    got, st_g = run_fused(d)
+    assert st_g == 0
+    assert_f16_parity(got, want, what="random blocks fused")
+
+
+@pytest.mark.parametrize("shift", [1, 3, 8, 13])
+def test_lz4_compressed_stream_not_16_byte_aligned(shift):
+    from tests._lz4gen import random_blocks
+    comp, offs, raw = random_blocks(9 + shift, 5, 65536, last=5000)
+    dbuf = dev(np.concatenate([np.zeros(shift, np.uint8), comp]))
+    out = torch.full((raw.size + 16,), 0xEE, dtype=torch.uint8, device="cuda")
+    stat = status_buf()
+    L.lt_lz4_decode(dbuf[shift:], int(comp.size), dev(offs), 65536, out, raw.size, stat)
+    torch.cuda.synchronize()
+    assert int(stat.item()) == 0
+    o = out.cpu().numpy()
+    assert np.array_equal(o[:raw.size], raw) and np.all(o[raw.size:] == 0xEE)

@@ -410,3 +410,17 @@ def test_lz4_corrupt_block_is_reported_not_crashing():
     for cut in (1, 2, 10, comp.size // 2):
         _, st = oracle.lz4_block_decode(comp[:-cut], data.size)
         assert st != 0
+
+
+def test_lz4_random_sequence_blocks_match_direct_simulation():
+    # blocks assembled sequence by sequence in every match regime; expected
+    # bytes from a direct simulation of the format, and the system library
+    from tests._lz4gen import random_blocks
+    comp, offs, raw = random_blocks(101, 12, 65536, last=40000)
+    out, st = oracle.lz4_decode_blocks(comp, offs, 65536, raw.size)
+    assert st == 0 and np.array_equal(out, raw)
+    if liblz4() is not None:
+        for b in range(len(offs) - 1):
+            c = comp[int(offs[b]):int(offs[b + 1])].tobytes()
+            want = raw[b * 65536:(b + 1) * 65536].tobytes()
+            assert lz4_lib_decompress(c, len(want)) == want

@@ -63,6 +63,8 @@ LT_API const char *lt_status_string(lt_status s) {
       return "decoded size differs from the declared size";
     case LT_ERR_CUDA:
       return "CUDA launch failed";
+    case LT_ERR_TIMEOUT:
+      return "an on-chip wait ran out (internal error)";
   }
   return "unknown status";
 }

@@ -24,6 +24,7 @@ LT_ERR_UNSUPPORTED = 3
 LT_ERR_CORRUPT_STREAM = 4
 LT_ERR_SIZE_MISMATCH = 5
 LT_ERR_CUDA = 6
+LT_ERR_TIMEOUT = 7
 LT_SCALE_PER_TENSOR = 0
 LT_SCALE_PER_ROW = 1
 LT_LZ4_BATCH_MAX = 16
