@@ -283,6 +283,13 @@ class DeviceWorkload:
                                       cols=m["cols"], group_size=m["group_size"], block_bytes=m["block_bytes"]))
                     base += n
                 self.c5.append(descs)
+        # LZ4 workspace (sequence index), sized for the largest single call
+        from weight_dequantization_b200 import lt_decode as L
+
+        nblk = [len(hw["C4"]["offsets"]) - 1] if "C4" in hw else []
+        nblk += [sum(len(m["offsets"]) - 1 for m in mats) for mats in hw.get("C5", [])]
+        self.ws = torch.empty(max([L.lt_lz4_workspace_bytes(n) for n in nblk] + [16]), dtype=torch.uint8,
+                              device="cuda")
         self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
         self.status_host = torch.zeros(1, dtype=torch.int32).pin_memory() if pinned else None
         self.h2d_bytes = sum(int(p.numel() * p.element_size()) for p, _ in self.h2d)
@@ -325,11 +332,11 @@ class DeviceWorkload:
             c4 = hw["C4"]
             L.lt_lz4_int4_decode(self.c4["comp"], int(c4["comp"].size), self.c4["offsets"], c4["block_bytes"],
                                  self.c4["scales"], self.c4["zeros"], c4["rows"], c4["cols"], c4["group_size"],
-                                 self.c4_out, self.status, s)
+                                 self.c4_out, self.ws, self.status, s)
             mark("C4")
             n += 1
         for descs in self.c5:
-            L.lt_lz4_int4_decode_batch(descs, self.status, s)
+            L.lt_lz4_int4_decode_batch(descs, self.ws, self.status, s)
             mark("C5")
             n += 1
         return n  # kernel launches of this step

@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define LT_ABI_VERSION 1
+#define LT_ABI_VERSION 2
 
 /* Same type as cudaStream_t. */
 typedef struct CUstream_st *lt_stream_t;
@@ -125,6 +125,21 @@ lt_status lt_zrle_decode(const uint8_t *enc, uint64_t enc_bytes, const uint64_t 
                          int32_t chunk_elems, lt_half *out, int32_t *d_status, lt_stream_t stream);
 
 /*
+ * Workspace of the LZ4 decoders. The serial part of LZ4 -- walking the
+ * sequence headers of a block -- runs as a separate pass, one thread per
+ * block, that writes a small sequence index (16 bytes per sequence, at most
+ * 512 sequences per block) into a caller-provided device workspace; the
+ * expansion then runs with the index in hand. lt_lz4_workspace_bytes(n)
+ * is the size needed for n blocks in one call (the sum over a batch). A
+ * call given NULL or a smaller workspace still decodes correctly, each
+ * block walked by the expanding CTA itself (much slower), and so is a block
+ * with more than 512 sequences. The workspace must be 16-byte aligned, is
+ * owned by the caller, and may be reused by the next call on the same
+ * stream; calls that run concurrently need their own.
+ */
+uint64_t lt_lz4_workspace_bytes(int64_t n_blocks);
+
+/*
  * Fused LZ4 block decompression -> INT4 unpack -> scale -> binary16
  * ("GPU Compression Pipeline - TDD Roadmap", Phase 2.1: decompress
  * directly to dequantized F16 with no intermediate buffer).
@@ -138,21 +153,25 @@ lt_status lt_zrle_decode(const uint8_t *enc, uint64_t enc_bytes, const uint64_t 
  *                      n_blocks = ceil(ceil(rows*cols/2) / block_bytes).
  *   The decompressed bytes are the `packed` array of lt_dequant_int4, and
  *   scales / zeros / rows / cols / group_size / out mean what they mean
- *   there. Decompressed bytes live only in on-chip shared memory.
+ *   there. Decompressed bytes live only in on-chip shared memory; the
+ *   workspace holds the sequence index (see lt_lz4_workspace_bytes).
  *   Device status: LT_ERR_CORRUPT_STREAM for a malformed block (offset 0 or
  *   before the block start, literal or match past the block end, input
  *   overrun, an offset pair outside comp), LT_ERR_SIZE_MISMATCH for a block
- *   that decodes to fewer bytes than it must.
+ *   that decodes to fewer bytes than it must. A malformed block's output is
+ *   left unspecified (possibly unwritten).
  */
 lt_status lt_lz4_int4_decode(const uint8_t *comp, uint64_t comp_bytes, const uint64_t *block_offsets,
                              int32_t block_bytes, const lt_half *scales, const uint8_t *zeros, int64_t rows,
-                             int64_t cols, int32_t group_size, lt_half *out, int32_t *d_status, lt_stream_t stream);
+                             int64_t cols, int32_t group_size, lt_half *out, void *workspace,
+                             uint64_t workspace_bytes, int32_t *d_status, lt_stream_t stream);
 
 /*
  * Several fused LZ4 -> INT4 decodes in one launch (the weight matrices of a
  * transformer layer decoded into one reused buffer). Each descriptor has
  * the meaning of the lt_lz4_int4_decode arguments of the same name. The
- * descriptor array itself is a HOST array, read during the call.
+ * descriptor array itself is a HOST array, read during the call; the
+ * workspace covers the blocks of all descriptors together.
  * 1 <= n_desc <= LT_LZ4_BATCH_MAX, else LT_ERR_INVALID_ARG / UNSUPPORTED.
  */
 #define LT_LZ4_BATCH_MAX 16
@@ -169,18 +188,19 @@ typedef struct {
   int32_t block_bytes;
 } lt_lz4_int4_desc;
 
-lt_status lt_lz4_int4_decode_batch(const lt_lz4_int4_desc *descs, int32_t n_desc, int32_t *d_status,
-                                   lt_stream_t stream);
+lt_status lt_lz4_int4_decode_batch(const lt_lz4_int4_desc *descs, int32_t n_desc, void *workspace,
+                                   uint64_t workspace_bytes, int32_t *d_status, lt_stream_t stream);
 
 /*
- * Plain LZ4 block decompression to bytes (the same on-chip decoder as the
- * fused path, writing the decompressed bytes instead of dequantizing them).
- * Used to check the LZ4 stage bit for bit, and as a general decoder.
+ * Plain LZ4 block decompression to bytes (the same decoder as the fused
+ * path, writing the decompressed bytes instead of dequantizing them). Used
+ * to check the LZ4 stage bit for bit, and as a general decoder.
  *   out        out_bytes bytes; block b fills [b*block_bytes, ...).
  *   block_bytes in [16, 65536], a multiple of 16.
  */
 lt_status lt_lz4_decode(const uint8_t *comp, uint64_t comp_bytes, const uint64_t *block_offsets, int32_t block_bytes,
-                        uint8_t *out, uint64_t out_bytes, int32_t *d_status, lt_stream_t stream);
+                        uint8_t *out, uint64_t out_bytes, void *workspace, uint64_t workspace_bytes,
+                        int32_t *d_status, lt_stream_t stream);
 
 /* Static, human-readable name of a status code. */
 const char *lt_status_string(lt_status s);

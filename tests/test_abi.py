@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert L.abi_version() == 1
+    assert L.abi_version() == 2
     for code in range(8):
         s = L.status_string(code)
         assert s and s != "unknown status"
@@ -63,14 +63,19 @@ def test_host_argument_errors_return_synchronously(lib):
     assert lib.lt_zrle_decode(P, 16, P, 100, 65536, P, None, None) == L.LT_ERR_UNSUPPORTED
     assert lib.lt_zrle_decode(P, 16, P + 4, 100, 4096, P, None, None) == L.LT_ERR_MISALIGNED
     assert lib.lt_zrle_decode(P, 16, P, -1, 4096, P, None, None) == L.LT_ERR_INVALID_ARG
-    assert lib.lt_lz4_int4_decode(P, 16, P, 65537, P, None, 1, 8, 8, P, None, None) == L.LT_ERR_UNSUPPORTED
-    assert lib.lt_lz4_int4_decode(P, 16, P, 1000, P, None, 1, 8, 8, P, None, None) == L.LT_ERR_UNSUPPORTED
-    assert lib.lt_lz4_int4_decode(P, 16, P, 65536, P, None, 1, 8, 3, P, None, None) == L.LT_ERR_INVALID_ARG
-    assert lib.lt_lz4_int4_decode(P, 16, P + 2, 65536, P, None, 1, 8, 8, P, None, None) == L.LT_ERR_MISALIGNED
-    assert lib.lt_lz4_decode(P, 16, P, 8, P, 100, None, None) == L.LT_ERR_UNSUPPORTED
+    assert lib.lt_lz4_int4_decode(P, 16, P, 65537, P, None, 1, 8, 8, P, None, 0, None, None) == L.LT_ERR_UNSUPPORTED
+    assert lib.lt_lz4_int4_decode(P, 16, P, 1000, P, None, 1, 8, 8, P, None, 0, None, None) == L.LT_ERR_UNSUPPORTED
+    assert lib.lt_lz4_int4_decode(P, 16, P, 65536, P, None, 1, 8, 3, P, None, 0, None, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_lz4_int4_decode(P, 16, P + 2, 65536, P, None, 1, 8, 8, P, None, 0, None, None) == L.LT_ERR_MISALIGNED
+    assert lib.lt_lz4_int4_decode(P, 16, P, 65536, P, None, 1, 8, 8, P, P + 4, 1 << 20, None, None) == \
+        L.LT_ERR_MISALIGNED
+    assert lib.lt_lz4_decode(P, 16, P, 8, P, 100, None, 0, None, None) == L.LT_ERR_UNSUPPORTED
     arr = (L.LtLz4Int4Desc * 17)()
-    assert lib.lt_lz4_int4_decode_batch(arr, 17, None, None) == L.LT_ERR_UNSUPPORTED
-    assert lib.lt_lz4_int4_decode_batch(arr, 0, None, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_lz4_int4_decode_batch(arr, 17, None, 0, None, None) == L.LT_ERR_UNSUPPORTED
+    assert lib.lt_lz4_int4_decode_batch(arr, 0, None, 0, None, None) == L.LT_ERR_INVALID_ARG
+    # workspace sizing: a 16-byte index header plus 512 descriptors per block
+    assert lib.lt_lz4_workspace_bytes(0) == 0
+    assert lib.lt_lz4_workspace_bytes(448) >= 448 * (16 + 16 * 512)
 
 
 def test_binding_rejects_host_tensors():

@@ -25,24 +25,33 @@ def _gpu():
     need_gpu()
 
 
-def run_raw(comp, offsets, block_bytes, out_bytes):
+def workspace(n_blocks, mode="ws"):
+    """The decoders' workspace: "ws" = enough for the sequence index,
+    "none" = no workspace (every block walked by the expanding CTA)."""
+    if mode == "none":
+        return None
+    return torch.empty(L.lt_lz4_workspace_bytes(n_blocks), dtype=torch.uint8, device="cuda")
+
+
+def run_raw(comp, offsets, block_bytes, out_bytes, ws="ws"):
     out = torch.full((out_bytes + 16,), 0xEE, dtype=torch.uint8, device="cuda")
     stat = status_buf()
     L.lt_lz4_decode(dev(comp) if comp.size else None, int(comp.size), dev(offsets), block_bytes, out, out_bytes,
-                    stat)
+                    workspace(len(offsets) - 1, ws), stat)
     torch.cuda.synchronize()
     o = out.cpu().numpy()
     assert np.all(o[out_bytes:] == 0xEE), "write past the end of the output"
     return o[:out_bytes], int(stat.item())
 
 
-def run_fused(d, zeros="use", out_offset=0):
+def run_fused(d, zeros="use", out_offset=0, ws="ws"):
     z = d["zeros"] if zeros == "use" else None
     n = d["rows"] * d["cols"]
     out = f16_out(n, out_offset)
     stat = status_buf()
     L.lt_lz4_int4_decode(dev(d["comp"]), int(d["comp"].size), dev(d["offsets"]), d["block_bytes"], dev(d["scales"]),
-                         dev(z), d["rows"], d["cols"], d["group_size"], out, stat)
+                         dev(z), d["rows"], d["cols"], d["group_size"], out, workspace(len(d["offsets"]) - 1, ws),
+                         stat)
     torch.cuda.synchronize()
     return host_bits(out), int(stat.item())
 
@@ -64,7 +73,8 @@ def make_matrix(rows, cols, G, block_bytes, seed=1, law="gauss"):
 
 # --------------------------------------------------------------------------- raw LZ4
 
-def test_lz4_handmade_blocks(golden_dir):
+@pytest.mark.parametrize("ws", ["ws", "none"])
+def test_lz4_handmade_blocks(golden_dir, ws):
     cases = json.load(open(os.path.join(golden_dir, "lz4_handmade.json")))["cases"]
     for c in cases:
         comp = np.frombuffer(hexbytes(c["comp"]), np.uint8)
@@ -78,22 +88,24 @@ def test_lz4_handmade_blocks(golden_dir):
         out_len = len(want) if want is not None else c["out_len"]
         offs = np.array([0, comp.size], np.uint64)
         bb = max(16, (out_len + 15) // 16 * 16)
-        got, st = run_raw(comp, offs, bb, out_len)
+        got, st = run_raw(comp, offs, bb, out_len, ws)
         _, st_o = oracle.lz4_block_decode(comp, out_len)
         assert st == st_o == c["status"], c["name"]
         if want is not None:
             assert got.tobytes() == want, c["name"]
 
 
-def test_lz4_raw_c4_full_size_bit_exact():
+@pytest.mark.parametrize("ws", ["ws", "none"])
+def test_lz4_raw_c4_full_size_bit_exact(ws):
     d = W.c4_lz4_int4(keep_packed=True)
-    got, st = run_raw(d["comp"], d["offsets"], d["block_bytes"], d["packed_bytes"])
+    got, st = run_raw(d["comp"], d["offsets"], d["block_bytes"], d["packed_bytes"], ws)
     assert st == 0
     assert np.array_equal(got, d["packed"])
 
 
+@pytest.mark.parametrize("ws", ["ws", "none"])
 @pytest.mark.parametrize("kind", ["0xab", "random_literals", "zeros", "max_offset"])
-def test_lz4_roadmap_64k_blocks(kind):
+def test_lz4_roadmap_64k_blocks(kind, ws):
     if kind == "0xab":          # the roadmap's 64 KB block of 0xAB
         data = np.full(65536, 0xAB, np.uint8)
         comp = lz4_compress_block(data)
@@ -112,7 +124,7 @@ def test_lz4_roadmap_64k_blocks(kind):
         assert data.size == 65536
         want, st_o = oracle.lz4_block_decode(comp, data.size)
         assert st_o == 0 and np.array_equal(want, data)
-    got, st = run_raw(comp, np.array([0, comp.size], np.uint64), 65536, data.size)
+    got, st = run_raw(comp, np.array([0, comp.size], np.uint64), 65536, data.size, ws)
     assert st == 0 and np.array_equal(got, data)
 
 
@@ -145,7 +157,8 @@ def test_lz4_raw_ragged_sizes(n_bytes, block_bytes):
     assert st == 0 and np.array_equal(got, data)
 
 
-def test_lz4_corrupt_blocks_match_oracle_status():
+@pytest.mark.parametrize("ws", ["ws", "none"])
+def test_lz4_corrupt_blocks_match_oracle_status(ws):
     data = int4_gauss_groups_packed(77, 131072)
     comp = lz4_compress_block(data)
     seen = set()
@@ -157,7 +170,7 @@ def test_lz4_corrupt_blocks_match_oracle_status():
             for _ in range(1 + trial % 3):
                 c[int(RNG.integers(0, c.size))] ^= np.uint8(1 << int(RNG.integers(0, 8)))
         want, st_o = oracle.lz4_block_decode(c, data.size)
-        got, st_g = run_raw(c, np.array([0, c.size], np.uint64), 65536, data.size)
+        got, st_g = run_raw(c, np.array([0, c.size], np.uint64), 65536, data.size, ws)
         assert st_g == st_o, trial
         seen.add(st_o)
         if st_o == 0:
@@ -172,11 +185,12 @@ def test_lz4_corrupt_blocks_match_oracle_status():
 
 # --------------------------------------------------------------------------- fused
 
-def test_fused_c4_full_size():
+@pytest.mark.parametrize("ws", ["ws", "none"])
+def test_fused_c4_full_size(ws):
     d = W.c4_lz4_int4()
     want, st = oracle_fused(d)
     assert st == 0
-    got, st_g = run_fused(d)
+    got, st_g = run_fused(d, ws=ws)
     assert st_g == 0
     assert_f16_parity(got, want, what="C4")
 
@@ -213,7 +227,7 @@ def test_fused_corrupt_stream_reports_and_stays_in_bounds():
     out = buf[:n]
     stat = status_buf()
     L.lt_lz4_int4_decode(dev(d["comp"]), int(d["comp"].size), dev(d["offsets"]), 65536, dev(d["scales"]),
-                         dev(d["zeros"]), d["rows"], d["cols"], 128, out, stat)
+                         dev(d["zeros"]), d["rows"], d["cols"], 128, out, workspace(4), stat)
     torch.cuda.synchronize()
     _, st_o = oracle_fused(d)
     assert st_o != 0
@@ -240,7 +254,8 @@ def test_fused_batch_matches_per_matrix_oracle():
                           block_bytes=m["block_bytes"]))
         outs.append(out)
     stat = status_buf()
-    L.lt_lz4_int4_decode_batch(descs, stat)
+    nb = sum(len(m["offsets"]) - 1 for m in mats)
+    L.lt_lz4_int4_decode_batch(descs, workspace(nb), stat)
     torch.cuda.synchronize()
     assert int(stat.item()) == 0
     for m, out in zip(mats, outs):
@@ -266,7 +281,8 @@ def test_fused_full_c5_layer_sampled_blocks():
         m["base"] = base
         base += n
     stat = status_buf()
-    L.lt_lz4_int4_decode_batch(descs, stat)
+    nb = sum(len(m["offsets"]) - 1 for m in mats)
+    L.lt_lz4_int4_decode_batch(descs, workspace(nb), stat)
     torch.cuda.synchronize()
     assert int(stat.item()) == 0
     codes_per_block = 2 * 65536
@@ -285,14 +301,15 @@ def test_fused_full_c5_layer_sampled_blocks():
             assert_f16_parity(got, want, what=f"{m['name']} block {b}")
 
 
+@pytest.mark.parametrize("ws", ["ws", "none"])
 @pytest.mark.parametrize("seed,n_blocks,block_bytes,last", [(1, 40, 65536, None), (2, 7, 65536, 12345),
                                                              (3, 30, 16384, 999), (4, 300, 4096, None)])
-def test_lz4_random_sequence_blocks(seed, n_blocks, block_bytes, last):
+def test_lz4_random_sequence_blocks(seed, n_blocks, block_bytes, last, ws):
     # every match regime: offset 1, periodic 2..15, overlapping >= 16,
     # non-overlapping and far offsets; literal runs of every length class
     from tests._lz4gen import random_blocks
     comp, offs, raw = random_blocks(seed, n_blocks, block_bytes, last)
-    got, st = run_raw(comp, offs, block_bytes, raw.size)
+    got, st = run_raw(comp, offs, block_bytes, raw.size, ws)
     assert st == 0
     assert np.array_equal(got, raw)
     # and through the fused path: raw bytes are the packed codes
@@ -302,9 +319,40 @@ def test_lz4_random_sequence_blocks(seed, n_blocks, block_bytes, last):
              scales=fp16_uniform(seed, n // G, -0.5, 0.5, stream=1), zeros=u8_uniform(seed, n // G, 0, 15, stream=2))
     want, st_o = oracle_fused(d)
     assert st_o == 0
-    got, st_g = run_fused(d)
+    got, st_g = run_fused(d, ws=ws)
     assert st_g == 0
     assert_f16_parity(got, want, what="random blocks fused")
+
+
+def test_lz4_blocks_with_more_sequences_than_the_index_holds():
+    # short literals and short matches: thousands of sequences per 64 KB
+    # block, beyond the workspace index; such blocks are walked by the CTA
+    from tests._lz4gen import _sequence
+    rng = np.random.default_rng(5)
+    comps, raws = [], []
+    for blk in range(6):
+        out, comp = bytearray(), bytearray()
+        while len(out) < 65536 - 40:
+            lits = rng.integers(0, 256, int(rng.integers(1, 6)), dtype=np.uint8).tobytes()
+            op = len(out) + len(lits)
+            d = int(rng.integers(1, min(op, 2000) + 1))
+            m = int(rng.integers(4, 12))
+            comp += _sequence(lits, d, m)
+            out += lits
+            for _ in range(m):
+                out.append(out[-d])
+        tail = rng.integers(0, 256, 65536 - len(out), dtype=np.uint8).tobytes()
+        comp += _sequence(tail, 0, 0)
+        out += tail
+        comps.append(bytes(comp))
+        raws.append(bytes(out))
+    comp = np.frombuffer(b"".join(comps), np.uint8).copy()
+    offs = np.concatenate([[0], np.cumsum([len(c) for c in comps])]).astype(np.uint64)
+    raw = np.frombuffer(b"".join(raws), np.uint8)
+    want, st = oracle.lz4_decode_blocks(comp, offs, 65536, raw.size)
+    assert st == 0 and np.array_equal(want, raw)
+    got, st = run_raw(comp, offs, 65536, raw.size, "ws")
+    assert st == 0 and np.array_equal(got, raw)
 
 
 @pytest.mark.parametrize("shift", [1, 3, 8, 13])
@@ -314,7 +362,7 @@ def test_lz4_compressed_stream_not_16_byte_aligned(shift):
     dbuf = dev(np.concatenate([np.zeros(shift, np.uint8), comp]))
     out = torch.full((raw.size + 16,), 0xEE, dtype=torch.uint8, device="cuda")
     stat = status_buf()
-    L.lt_lz4_decode(dbuf[shift:], int(comp.size), dev(offs), 65536, out, raw.size, stat)
+    L.lt_lz4_decode(dbuf[shift:], int(comp.size), dev(offs), 65536, out, raw.size, workspace(len(offs) - 1), stat)
     torch.cuda.synchronize()
     assert int(stat.item()) == 0
     o = out.cpu().numpy()

@@ -31,7 +31,7 @@ LT_LZ4_BATCH_MAX = 16
 
 EXPORTED = (
     "lt_dequant_int4", "lt_dequant_int8", "lt_zrle_decode", "lt_lz4_int4_decode",
-    "lt_lz4_int4_decode_batch", "lt_lz4_decode", "lt_status_string", "lt_abi_version",
+    "lt_lz4_int4_decode_batch", "lt_lz4_decode", "lt_lz4_workspace_bytes", "lt_status_string", "lt_abi_version",
 )
 
 
@@ -66,9 +66,11 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.lt_dequant_int4.argtypes = [P, P, P, I64, I64, I32, P, P]
     lib.lt_dequant_int8.argtypes = [P, P, P, I32, I64, I64, P, P]
     lib.lt_zrle_decode.argtypes = [P, U64, P, I64, I32, P, P, P]
-    lib.lt_lz4_int4_decode.argtypes = [P, U64, P, I32, P, P, I64, I64, I32, P, P, P]
-    lib.lt_lz4_int4_decode_batch.argtypes = [ctypes.POINTER(LtLz4Int4Desc), I32, P, P]
-    lib.lt_lz4_decode.argtypes = [P, U64, P, I32, P, U64, P, P]
+    lib.lt_lz4_int4_decode.argtypes = [P, U64, P, I32, P, P, I64, I64, I32, P, P, U64, P, P]
+    lib.lt_lz4_int4_decode_batch.argtypes = [ctypes.POINTER(LtLz4Int4Desc), I32, P, U64, P, P]
+    lib.lt_lz4_decode.argtypes = [P, U64, P, I32, P, U64, P, U64, P, P]
+    lib.lt_lz4_workspace_bytes.argtypes = [I64]
+    lib.lt_lz4_workspace_bytes.restype = U64
     for f in ("lt_dequant_int4", "lt_dequant_int8", "lt_zrle_decode", "lt_lz4_int4_decode",
               "lt_lz4_int4_decode_batch", "lt_lz4_decode"):
         getattr(lib, f).restype = ctypes.c_int
@@ -135,14 +137,29 @@ def lt_zrle_decode(enc, enc_bytes: int, chunk_offsets, n_elements: int, chunk_el
                                          _ptr(out), _ptr(d_status), _stream(stream, out)), "lt_zrle_decode")
 
 
+def lt_lz4_workspace_bytes(n_blocks: int) -> int:
+    return int(load_library().lt_lz4_workspace_bytes(int(n_blocks)))
+
+
+def _ws(workspace):
+    if workspace is None:
+        return None, 0
+    if isinstance(workspace, tuple):
+        return workspace
+    return _ptr(workspace), workspace.numel() * workspace.element_size()
+
+
 def lt_lz4_int4_decode(comp, comp_bytes: int, block_offsets, block_bytes: int, scales, zeros, rows: int, cols: int,
-                       group_size: int, out, d_status=None, stream=None) -> None:
+                       group_size: int, out, workspace=None, d_status=None, stream=None) -> None:
+    """``workspace``: a CUDA tensor (its bytes), an (address, bytes) pair, or
+    None (correct but slow decode)."""
+    wp, wb = _ws(workspace)
     _check(load_library().lt_lz4_int4_decode(_ptr(comp), comp_bytes, _ptr(block_offsets), block_bytes,
-                                             _ptr(scales), _ptr(zeros), rows, cols, group_size, _ptr(out),
+                                             _ptr(scales), _ptr(zeros), rows, cols, group_size, _ptr(out), wp, wb,
                                              _ptr(d_status), _stream(stream, out)), "lt_lz4_int4_decode")
 
 
-def lt_lz4_int4_decode_batch(descs: Sequence[dict], d_status=None, stream=None) -> None:
+def lt_lz4_int4_decode_batch(descs: Sequence[dict], workspace=None, d_status=None, stream=None) -> None:
     """``descs``: dicts with the keys of lt_lz4_int4_desc (tensors or addresses)."""
     n = len(descs)
     arr = (LtLz4Int4Desc * max(n, 1))()
@@ -151,11 +168,18 @@ def lt_lz4_int4_decode_batch(descs: Sequence[dict], d_status=None, stream=None) 
                                _ptr(d.get("zeros")), _ptr(d["out"]), d["rows"], d["cols"], d["group_size"],
                                d["block_bytes"])
     like = descs[0]["out"] if n else None
-    _check(load_library().lt_lz4_int4_decode_batch(arr, n, _ptr(d_status), _stream(stream, like)),
+    wp, wb = _ws(workspace)
+    _check(load_library().lt_lz4_int4_decode_batch(arr, n, wp, wb, _ptr(d_status), _stream(stream, like)),
            "lt_lz4_int4_decode_batch")
 
 
-def lt_lz4_decode(comp, comp_bytes: int, block_offsets, block_bytes: int, out, out_bytes: int, d_status=None,
-                  stream=None) -> None:
+def lt_lz4_decode(comp, comp_bytes: int, block_offsets, block_bytes: int, out, out_bytes: int, workspace=None,
+                  d_status=None, stream=None) -> None:
+    wp, wb = _ws(workspace)
     _check(load_library().lt_lz4_decode(_ptr(comp), comp_bytes, _ptr(block_offsets), block_bytes, _ptr(out),
-                                        out_bytes, _ptr(d_status), _stream(stream, out)), "lt_lz4_decode")
+                                        out_bytes, wp, wb, _ptr(d_status), _stream(stream, out)), "lt_lz4_decode")
+
+
+def lz4_blocks(n_bytes: int, block_bytes: int) -> int:
+    """Number of LZ4 blocks of ``block_bytes`` covering ``n_bytes``."""
+    return (int(n_bytes) + block_bytes - 1) // block_bytes
