@@ -89,23 +89,15 @@ def dist_init(world):
 
 
 def max_over_ranks(x: float, dist) -> float:
-    if dist is None:
-        return x
-    import torch
+    from weight_dequantization_b200.shard import reduce_max
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return reduce_max(x, device="cuda") if dist is not None else x
 
 
 def sum_over_ranks(x: float, dist) -> float:
-    if dist is None:
-        return x
-    import torch
+    from weight_dequantization_b200.shard import reduce_sum
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return reduce_sum(x, device="cuda") if dist is not None else x
 
 
 # ----------------------------------------------------------------------------
