@@ -202,6 +202,42 @@ lt_status lt_lz4_decode(const uint8_t *comp, uint64_t comp_bytes, const uint64_t
                         uint8_t *out, uint64_t out_bytes, void *workspace, uint64_t workspace_bytes,
                         int32_t *d_status, lt_stream_t stream);
 
+/*
+ * The fused decode of lt_lz4_int4_decode for callers that cannot allocate
+ * device memory. (No counterpart on the pages: this entry point exists for
+ * how the library is called, not for what it computes.)
+ *
+ * Some callers may not allocate device memory at the time they decode: a
+ * plugin running inside an inference engine or server that hands out a fixed
+ * device-memory budget at start-up and forbids allocations afterwards, or
+ * any code whose device allocator belongs to another component. They cannot
+ * provide the workspace the other LZ4 entry points take. This entry point
+ * keeps that workspace in a scratch array built into the library instead:
+ * every GPU that loads the library holds LT_NOALLOC_MAX_BLOCKS blocks'
+ * worth of it (about 4 MiB) until the process exits, and the call itself
+ * allocates and frees nothing.
+ *
+ * Arguments, results and device status are those of lt_lz4_int4_decode,
+ * without the workspace. Limits and rules:
+ *  - At most LT_NOALLOC_MAX_BLOCKS LZ4 blocks per call
+ *    (ceil(ceil(rows*cols/2) / block_bytes)); larger requests return
+ *    LT_ERR_UNSUPPORTED and enqueue nothing.
+ *  - The first call on each device looks up the scratch array's device
+ *    address (cudaGetSymbolAddress) with that device current; make that
+ *    first call before any stream capture. A failed lookup returns
+ *    LT_ERR_CUDA.
+ *  - All calls on a device share the one scratch array and it keeps the
+ *    last call's contents (nothing in it needs to start at zero). Calls whose
+ *    work overlaps on the GPU -- on different streams, or from different host
+ *    threads -- race on it and may decode wrongly: run them one after
+ *    another, e.g. on one stream.
+ */
+#define LT_NOALLOC_MAX_BLOCKS 512
+lt_status lt_lz4_int4_decode_noalloc(const uint8_t *comp, uint64_t comp_bytes, const uint64_t *block_offsets,
+                                     int32_t block_bytes, const lt_half *scales, const uint8_t *zeros, int64_t rows,
+                                     int64_t cols, int32_t group_size, lt_half *out, int32_t *d_status,
+                                     lt_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 const char *lt_status_string(lt_status s);
 

@@ -26,6 +26,8 @@
 // Blocks with more than kCap sequences, and calls without a workspace, are
 // decoded by warp 0 walking the block itself (slower, same result).
 
+#include <mutex>
+
 #include "lt_common.cuh"
 
 namespace lt {
@@ -616,4 +618,61 @@ LT_API lt_status lt_lz4_decode(const uint8_t *comp, uint64_t comp_bytes, const u
   if (workspace && !aligned(workspace, 16)) return LT_ERR_MISALIGNED;
   batch.max_block_bytes = block_bytes;
   return launch(batch, false, workspace, workspace_bytes, d_status, (cudaStream_t)stream);
+}
+
+// ---------------------------------------------------------------------------
+// Entry point that allocates nothing: the fused decode with its sequence
+// index kept in a fixed scratch array compiled into this library, for
+// callers that may not allocate device memory themselves (see the header).
+// ---------------------------------------------------------------------------
+namespace lt {
+namespace {
+
+constexpr uint64_t kNoAllocBytes = (uint64_t)LT_NOALLOC_MAX_BLOCKS * (16ull + 16ull * kCap) + 256;
+
+// One copy per GPU that loads the library, resident until the process
+// exits. Host code only ever sees its address through the lookup below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[64] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the first call on a device does it).
+lt_status noalloc_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LT_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return LT_ERR_CUDA;
+    }
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return LT_OK;
+}
+
+}  // namespace
+}  // namespace lt
+
+LT_API lt_status lt_lz4_int4_decode_noalloc(const uint8_t *comp, uint64_t comp_bytes, const uint64_t *block_offsets,
+                                            int32_t block_bytes, const lt_half *scales, const uint8_t *zeros,
+                                            int64_t rows, int64_t cols, int32_t group_size, lt_half *out,
+                                            int32_t *d_status, lt_stream_t stream) {
+  if (!aligned(d_status, 4)) return LT_ERR_MISALIGNED;
+  Batch batch = empty_batch();
+  lt_status s = add_fused_job(batch, comp, comp_bytes, block_offsets, block_bytes, scales, zeros, rows, cols,
+                              group_size, out);
+  if (s != LT_OK) return s;
+  if (batch.total_blocks > LT_NOALLOC_MAX_BLOCKS) return LT_ERR_UNSUPPORTED;  // larger than the built-in scratch
+  if (batch.total_blocks == 0) return LT_OK;
+  void *scratch = nullptr;
+  s = noalloc_scratch(&scratch);
+  if (s != LT_OK) return s;
+  // the parse pass writes every index entry the expand pass reads, so the
+  // scratch needs no clearing between calls
+  return launch(batch, true, scratch, kNoAllocBytes, d_status, (cudaStream_t)stream);
 }

@@ -31,8 +31,10 @@ LT_LZ4_BATCH_MAX = 16
 
 EXPORTED = (
     "lt_dequant_int4", "lt_dequant_int8", "lt_zrle_decode", "lt_lz4_int4_decode",
-    "lt_lz4_int4_decode_batch", "lt_lz4_decode", "lt_lz4_workspace_bytes", "lt_status_string", "lt_abi_version",
+    "lt_lz4_int4_decode_batch", "lt_lz4_decode", "lt_lz4_workspace_bytes", "lt_lz4_int4_decode_noalloc",
+    "lt_status_string", "lt_abi_version",
 )
+LT_NOALLOC_MAX_BLOCKS = 512
 
 
 class LtError(RuntimeError):
@@ -69,6 +71,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.lt_lz4_int4_decode.argtypes = [P, U64, P, I32, P, P, I64, I64, I32, P, P, U64, P, P]
     lib.lt_lz4_int4_decode_batch.argtypes = [ctypes.POINTER(LtLz4Int4Desc), I32, P, U64, P, P]
     lib.lt_lz4_decode.argtypes = [P, U64, P, I32, P, U64, P, U64, P, P]
+    lib.lt_lz4_int4_decode_noalloc.argtypes = [P, U64, P, I32, P, P, I64, I64, I32, P, P, P]
+    lib.lt_lz4_int4_decode_noalloc.restype = ctypes.c_int
     lib.lt_lz4_workspace_bytes.argtypes = [I64]
     lib.lt_lz4_workspace_bytes.restype = U64
     for f in ("lt_dequant_int4", "lt_dequant_int8", "lt_zrle_decode", "lt_lz4_int4_decode",
@@ -178,6 +182,18 @@ def lt_lz4_decode(comp, comp_bytes: int, block_offsets, block_bytes: int, out, o
     wp, wb = _ws(workspace)
     _check(load_library().lt_lz4_decode(_ptr(comp), comp_bytes, _ptr(block_offsets), block_bytes, _ptr(out),
                                         out_bytes, wp, wb, _ptr(d_status), _stream(stream, out)), "lt_lz4_decode")
+
+
+def lt_lz4_int4_decode_noalloc(comp, comp_bytes: int, block_offsets, block_bytes: int, scales, zeros, rows: int,
+                               cols: int, group_size: int, out, d_status=None, stream=None) -> None:
+    """lt_lz4_int4_decode without a workspace argument, for callers that may
+    not allocate device memory: the sequence index lives in a scratch array
+    built into the library (at most LT_NOALLOC_MAX_BLOCKS blocks per call;
+    calls that overlap on the GPU race on it)."""
+    _check(load_library().lt_lz4_int4_decode_noalloc(_ptr(comp), comp_bytes, _ptr(block_offsets), block_bytes,
+                                                     _ptr(scales), _ptr(zeros), rows, cols, group_size, _ptr(out),
+                                                     _ptr(d_status), _stream(stream, out)),
+           "lt_lz4_int4_decode_noalloc")
 
 
 def lz4_blocks(n_bytes: int, block_bytes: int) -> int:
