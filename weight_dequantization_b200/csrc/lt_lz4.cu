@@ -42,7 +42,6 @@ constexpr uint32_t kStep = 512;          // window bytes per dequantizer-warp st
 constexpr uint32_t kCap = 512;           // sequence descriptors per block in the workspace
 constexpr uint32_t kOverflow = 0x100;    // parse status: more than kCap sequences
 constexpr uint32_t kNoIndex = 0x101;     // no workspace: every block takes the fallback
-constexpr int kParseThreads = 32;
 constexpr long kSpinLimit = 1L << 23;    // ~0.5 s of polling, then give up
 
 struct Job {
@@ -91,7 +90,6 @@ __device__ __forceinline__ void st_release_shared(uint32_t *p, uint32_t v) {
   asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"((uint32_t)__cvta_generic_to_shared(p)), "r"(v)
                : "memory");
 }
-__device__ __forceinline__ void prefetch_l1(const void *p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
 __device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
 // Wait (whole warp) until *c >= target. Lane 0 polls; the value is
@@ -195,91 +193,198 @@ __device__ __forceinline__ void copy_match(uint8_t *win, uint32_t op, uint32_t d
 }
 
 // ---------------------------------------------------------------------------
-// 1. parse: one thread walks one block
+// 1. parse: one warp walks one block
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t ldb(const uint8_t *g, uint32_t i, uint32_t n) { return i < n ? __ldg(g + i) : 0u; }
+// One warp walks one block: its compressed bytes stream through a 2 KB
+// shared-memory ring (cp.async, one 16-byte copy per lane = one 512-byte
+// chunk per instruction, four chunks in flight ahead of the walk) and every
+// lane reads the same header bytes from there (broadcast), so the walk is
+// warp-uniform -- no divergence -- at two dependent shared-memory reads per
+// sequence. 64 warps per SM walk 64 blocks side by side.
+constexpr int kParseWarps = 4;
+constexpr uint32_t kPRing = 2048;
+constexpr uint32_t kPChunk = 512;
+constexpr uint32_t kPChunks = kPRing / kPChunk;
 
-// Walk LZ4 block g[0, n_in) that must decode to exactly olen bytes; write
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+               "l"(gmem), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+struct WarpRing {
+  uint8_t *buf;        // this warp's kPRing bytes
+  const uint8_t *a0;   // rel 0: the block's first byte rounded down to 16 bytes
+  const uint8_t *beg;  // the block's first byte
+  const uint8_t *end;  // one past its last byte
+  uint32_t total;      // chunks covering [a0, end)
+  uint32_t issued;     // chunks issued (each one cp.async group, in order)
+  uint32_t done;       // chunks known landed and visible to the warp
+  int lane;
+
+  // copies of chunk `issued`, 16 bytes per lane; only bytes of [beg, end)
+  // are read from HBM (a piece starting before `beg` is copied byte by byte)
+  __device__ __forceinline__ void issue() {
+    const uint32_t rel = issued * kPChunk + 16u * (uint32_t)lane;
+    const uint8_t *src = a0 + rel;
+    uint8_t *dst = buf + (rel & (kPRing - 1));
+    if (src >= beg) {
+      const uint32_t nb = src < end ? (uint32_t)((end - src) < 16 ? (end - src) : 16) : 0u;
+      cp_async16(dst, nb ? (const void *)src : (const void *)beg, nb);
+    } else {
+      for (uint32_t i = 0; i < 16; ++i)
+        if (src + i >= beg && src + i < end) dst[i] = __ldg(src + i);
+    }
+    cp_async_commit();
+    ++issued;
+  }
+  // wait until every chunk up to c (< issued) has landed
+  __device__ __forceinline__ void wait_for(uint32_t c) {
+    if (c < done) return;
+    switch (issued - 1 - c) {  // groups allowed to stay in flight
+      case 0: cp_async_wait<0>(); break;
+      case 1: cp_async_wait<1>(); break;
+      case 2: cp_async_wait<2>(); break;
+      default: cp_async_wait<3>(); break;
+    }
+    done = c + 1;
+    __syncwarp();  // every lane's copies are visible to every lane
+  }
+  // keep kPChunks chunks in flight ahead of rel position `pos`. A slot is
+  // refilled only after the chunk it held has landed: copies of different
+  // groups may complete in any order.
+  __device__ __forceinline__ void top_up(uint32_t pos) {
+    const uint32_t lim = pos / kPChunk + kPChunks;
+    while (issued < total && issued < lim) {
+      if (issued >= kPChunks) wait_for(issued - kPChunks);
+      issue();
+    }
+  }
+  // make rel bytes [pos, q) readable (q - pos <= 8)
+  __device__ __forceinline__ void need(uint32_t pos, uint32_t q) {
+    const uint32_t c = (q - 1) / kPChunk;
+    if (c < done) return;
+    const uint32_t cmin = pos / kPChunk;
+    if (cmin > issued) {  // the walk skipped everything fetched (a long literal run): restart there
+      cp_async_wait<0>();
+      issued = done = cmin;
+    }
+    top_up(pos);
+    wait_for(c);
+  }
+  __device__ __forceinline__ uint32_t at(uint32_t rel) const { return buf[rel & (kPRing - 1)]; }
+};
+
+// Walk LZ4 block [beg, end) that must decode to exactly olen bytes; write
 // descriptors {literal source, output position, literal length,
 // match offset | (match length - 4) << 16} (offset 0: no match). Returns 0,
-// a stream status, or kOverflow.
-__device__ uint32_t parse_block(const uint8_t *__restrict__ g, uint64_t ilen, uint32_t olen, uint4 *__restrict__ out,
-                                uint32_t &n_out) {
+// a stream status, or kOverflow. Every step checks the bounds the oracle
+// checks, in the same order, so statuses agree. Warp-uniform.
+__device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint4 *__restrict__ out,
+                                                uint32_t &n_out) {
   n_out = 0;
+  const uint64_t ilen = (uint64_t)(r.end - r.beg);
   if (ilen == 0) return olen == 0 ? 0u : (uint32_t)LT_ERR_SIZE_MISMATCH;
   if (ilen > 0x7FFFFFFFull) return LT_ERR_CORRUPT_STREAM;  // no valid block of <= 64 KB is this long
-  const uint32_t n_in = (uint32_t)ilen;
-  uint32_t ip = 0, op = 0, n = 0, pf = 0;
-  uint32_t st = 0;
+  const uint32_t lead = (uint32_t)(r.beg - r.a0);
+  const uint32_t iend = lead + (uint32_t)ilen;
+  uint32_t ip = lead, op = 0, n = 0, st = 0;
   for (;;) {
-    while (pf < n_in && pf < ip + 1024) {  // keep ~1 KB of the stream in L1 ahead of the walk
-      prefetch_l1(g + pf);
-      pf += 128;
-    }
-    if (ip >= n_in) { st = LT_ERR_CORRUPT_STREAM; break; }
-    const uint32_t token = ldb(g, ip, n_in);
-    uint32_t b1 = ldb(g, ip + 1, n_in);
+    if (ip >= iend) { st = LT_ERR_CORRUPT_STREAM; break; }
+    r.need(ip, ip + 2 < iend ? ip + 2 : iend);
+    const uint32_t token = r.at(ip);
+    uint32_t b = ip + 1 < iend ? r.at(ip + 1) : 0u;
     ip += 1;
     uint32_t lit = token >> 4;
     if (lit == 15) {
       for (;;) {
-        if (ip >= n_in || lit > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
+        if (ip >= iend || lit > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
         ip += 1;
-        lit += b1;
-        if (b1 != 255) break;
-        b1 = ldb(g, ip, n_in);
+        lit += b;
+        if (b != 255) break;
+        if (ip < iend) {
+          r.need(ip, ip + 1);
+          b = r.at(ip);
+        }
       }
       if (st) break;
     }
-    if ((uint64_t)ip + lit > n_in || (uint64_t)op + lit > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
-    const uint32_t ls = ip;
+    if ((uint64_t)ip + lit > iend || (uint64_t)op + lit > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
+    const uint32_t ls = ip - lead;
     ip += lit;
-    if (ip == n_in) {  // the last sequence has literals only
+    if (ip == iend) {  // the last sequence has literals only
       if (n >= kCap) { st = kOverflow; break; }
-      out[n++] = make_uint4(ls, op, lit, 0u);
+      if (r.lane == 0) out[n] = make_uint4(ls, op, lit, 0u);
+      ++n;
       op += lit;
       if (op != olen) st = LT_ERR_SIZE_MISMATCH;
       break;
     }
-    if (ip + 2 > n_in) { st = LT_ERR_CORRUPT_STREAM; break; }
-    const uint32_t d = ldb(g, ip, n_in) | (ldb(g, ip + 1, n_in) << 8);
-    uint32_t b2 = ldb(g, ip + 2, n_in);
+    if (ip + 2 > iend) { st = LT_ERR_CORRUPT_STREAM; break; }
+    r.need(ip, ip + 3 < iend ? ip + 3 : iend);
+    const uint32_t d = r.at(ip) | (r.at(ip + 1) << 8);
+    b = ip + 2 < iend ? r.at(ip + 2) : 0u;
     ip += 2;
     if (d == 0 || d > op + lit) { st = LT_ERR_CORRUPT_STREAM; break; }
     uint32_t mlen = (token & 15u) + 4;
     if ((token & 15u) == 15u) {
       for (;;) {
-        if (ip >= n_in || mlen > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
+        if (ip >= iend || mlen > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
         ip += 1;
-        mlen += b2;
-        if (b2 != 255) break;
-        b2 = ldb(g, ip, n_in);
+        mlen += b;
+        if (b != 255) break;
+        if (ip < iend) {
+          r.need(ip, ip + 1);
+          b = r.at(ip);
+        }
       }
       if (st) break;
     }
     if ((uint64_t)op + lit + mlen > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
     if (n >= kCap) { st = kOverflow; break; }
-    out[n++] = make_uint4(ls, op, lit, d | ((mlen - 4) << 16));
+    if (r.lane == 0) out[n] = make_uint4(ls, op, lit, d | ((mlen - 4) << 16));
+    ++n;
     op += lit + mlen;
+    r.top_up(ip);
   }
+  cp_async_wait<0>();  // nothing may land in the ring after this block
+  __syncwarp();
   n_out = n;
   return st;
 }
 
-__global__ void __launch_bounds__(kParseThreads) k_lz4_parse(const __grid_constant__ Batch batch,
-                                                             uint4 *__restrict__ hdr, uint4 *__restrict__ desc) {
-  for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < batch.total_blocks;
-       blk += (int64_t)gridDim.x * blockDim.x) {
+__global__ void __launch_bounds__(kParseWarps * 32) k_lz4_parse(const __grid_constant__ Batch batch,
+                                                                uint4 *__restrict__ hdr, uint4 *__restrict__ desc) {
+  __shared__ __align__(16) uint8_t rings[kParseWarps][kPRing];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t blk = (int64_t)blockIdx.x * kParseWarps + warp; blk < batch.total_blocks;
+       blk += (int64_t)gridDim.x * kParseWarps) {
     int64_t b;
     const Job &jb = find_job(batch, blk, b);
     const uint32_t olen = block_len(jb, b);
     const uint64_t s0 = jb.offsets[b], s1 = jb.offsets[b + 1];
     uint32_t n = 0, st;
-    if (s1 < s0 || s1 > jb.comp_bytes)
+    if (s1 < s0 || s1 > jb.comp_bytes) {
       st = LT_ERR_CORRUPT_STREAM;
-    else
-      st = parse_block(jb.comp + s0, s1 - s0, olen, desc + blk * kCap, n);
-    hdr[blk] = make_uint4(n, st, 0u, 0u);
+    } else {
+      WarpRing r;
+      r.buf = rings[warp];
+      r.lane = lane;
+      r.beg = jb.comp + s0;
+      r.end = jb.comp + s1;
+      r.a0 = reinterpret_cast<const uint8_t *>(reinterpret_cast<uintptr_t>(r.beg) & ~uintptr_t(15));
+      r.total = (uint32_t)((r.end - r.a0 + kPChunk - 1) / kPChunk);
+      r.issued = 0;
+      r.done = 0;
+      r.top_up(0);
+      st = parse_block(r, olen, desc + blk * kCap, n);
+    }
+    if (lane == 0) hdr[blk] = make_uint4(n, st, 0u, 0u);
   }
 }
 
@@ -496,9 +601,9 @@ lt_status launch(const Batch &batch, bool fused, void *workspace, uint64_t works
     uintptr_t p = (reinterpret_cast<uintptr_t>(workspace) + 255) & ~uintptr_t(255);
     hdr = reinterpret_cast<uint4 *>(p);
     desc = hdr + batch.total_blocks;
-    const int64_t need = (batch.total_blocks + kParseThreads - 1) / kParseThreads;
-    const int64_t cap = (int64_t)num_sms() * 16;
-    k_lz4_parse<<<(int)(need < cap ? need : cap), kParseThreads, 0, st>>>(batch, hdr, desc);
+    const int64_t need = (batch.total_blocks + kParseWarps - 1) / kParseWarps;
+    const int64_t cap = (int64_t)num_sms() * blocks_per_sm((const void *)k_lz4_parse, kParseWarps * 32, 0);
+    k_lz4_parse<<<(int)(need < cap ? need : cap), kParseWarps * 32, 0, st>>>(batch, hdr, desc);
   }
   const size_t smem = (size_t)((batch.max_block_bytes + 15) / 16 * 16) + 2 * kPad;
   const void *k = fused ? (const void *)k_lz4_expand<true> : (const void *)k_lz4_expand<false>;
