@@ -35,14 +35,22 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kMaxWindow = 65536;
+constexpr uint32_t kMaxWindow = 65536;
 constexpr int kPad = 16;                 // guard bytes before and after the window
-constexpr uint32_t kPublishBytes = 2048;
-constexpr uint32_t kStep = 512;          // window bytes per dequantizer-warp step (4 words per lane)
-constexpr uint32_t kCap = 512;           // sequence descriptors per block in the workspace
+constexpr uint32_t kCap = 2 * kThreads; // sequence descriptors per block in the workspace (two per thread)
 constexpr uint32_t kOverflow = 0x100;    // parse status: more than kCap sequences
 constexpr uint32_t kNoIndex = 0x101;     // no workspace: every block takes the fallback
-constexpr long kSpinLimit = 1L << 23;    // ~0.5 s of polling, then give up
+constexpr uint32_t kNoInPlace = 0x102;   // parse status: the block cannot be staged in its window
+constexpr uint32_t kWinSlack = 512;      // window bytes past the largest block, for in-place staging
+constexpr int kMatchRounds = 24;         // parallel match rounds before the rest is replayed in order
+constexpr uint32_t kScanMax = 8;         // sequences a match source may span and still be checked one by one
+constexpr uint32_t kSerialTail = 24;     // unresolved matches left when warp 0 takes over
+
+// Window bytes a CTA holds for blocks of up to max_block_bytes: the block
+// plus room to stage its compressed bytes at the end.
+__host__ __device__ constexpr uint32_t win_cap(int32_t max_block_bytes) {
+  return ((uint32_t)max_block_bytes + 15u) / 16u * 16u + kWinSlack;
+}
 
 struct Job {
   const uint8_t *comp;
@@ -78,60 +86,7 @@ __device__ __forceinline__ uint32_t block_len(const Job &jb, int64_t b) {
   return (uint32_t)((jb.packed_bytes - d0) < jb.block_bytes ? (jb.packed_bytes - d0) : jb.block_bytes);
 }
 
-__device__ __forceinline__ uint32_t ld_acquire_shared(const uint32_t *p) {
-  uint32_t v;
-  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];"
-               : "=r"(v)
-               : "r"((uint32_t)__cvta_generic_to_shared(p))
-               : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_shared(uint32_t *p, uint32_t v) {
-  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"((uint32_t)__cvta_generic_to_shared(p)), "r"(v)
-               : "memory");
-}
 __device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
-
-// Wait (whole warp) until *c >= target. Lane 0 polls; the value is
-// broadcast. Returns false if the wait ran out (the status records it).
-__device__ __forceinline__ bool wait_ge(const uint32_t *c, uint32_t target, uint32_t &seen, int lane,
-                                        int32_t *d_status) {
-  uint32_t v = 0, ok = 1;
-  if (lane == 0) {
-    v = ld_acquire_shared(c);
-    long spins = 0;
-    while (v < target) {
-      if (++spins > kSpinLimit) {
-        report(d_status, LT_ERR_TIMEOUT);
-        ok = 0;
-        break;
-      }
-      if (spins > 32) __nanosleep(64);
-      v = ld_acquire_shared(c);
-    }
-  }
-  v = __shfl_sync(0xFFFFFFFFu, v, 0);
-  ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-  __syncwarp();
-  seen = v;
-  return ok != 0;
-}
-
-// 4 bytes at a (little-endian) from global memory, touching nothing outside
-// [lo, hi); bytes outside read as 0.
-__device__ __forceinline__ uint32_t gather4_global(const uint8_t *a, const uint8_t *lo, const uint8_t *hi) {
-  const uint8_t *al = reinterpret_cast<const uint8_t *>(reinterpret_cast<uintptr_t>(a) & ~uintptr_t(3));
-  if (al >= lo && al + 8 <= hi) {
-    const uint32_t u0 = __ldg(reinterpret_cast<const uint32_t *>(al));
-    const uint32_t u1 = __ldg(reinterpret_cast<const uint32_t *>(al) + 1);
-    return __funnelshift_r(u0, u1, 8u * (uint32_t)(reinterpret_cast<uintptr_t>(a) & 3));
-  }
-  uint32_t v = 0;
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    if (a + j >= lo && a + j < hi) v |= (uint32_t)__ldg(a + j) << (8 * j);
-  return v;
-}
 
 // 4 bytes at window byte index s (may be slightly negative or past the end:
 // the window has kPad guard bytes on both sides)
@@ -161,30 +116,33 @@ __device__ __forceinline__ void write_span(uint8_t *win, uint32_t a, uint32_t b,
   }
 }
 
-// Replay one match (warp-wide): window bytes [op, op + M) from [op - d, ...).
-__device__ __forceinline__ void copy_match(uint8_t *win, uint32_t op, uint32_t d, uint32_t M, int lane) {
+// Replay one match with NL cooperating lanes (lid in [0, NL), syncing with
+// `mask`): window bytes [op, op + M) from [op - d, ...).
+template <int NL>
+__device__ __forceinline__ void copy_match(uint8_t *win, uint32_t op, uint32_t d, uint32_t M, int lid,
+                                           unsigned mask) {
   if (d >= M) {
-    write_span<32>(
-        win, op, op + M, lane, [&](uint32_t x) { return win[x - d]; },
+    write_span<NL>(
+        win, op, op + M, lid, [&](uint32_t x) { return win[x - d]; },
         [&](uint32_t x) { return gather4_window(win, (int32_t)x - (int32_t)d); });
   } else if (d == 1) {
     const uint32_t bv = win[op - 1];
     const uint32_t v = 0x01010101u * bv;
-    write_span<32>(
-        win, op, op + M, lane, [&](uint32_t) { return (uint8_t)bv; }, [&](uint32_t) { return v; });
+    write_span<NL>(
+        win, op, op + M, lid, [&](uint32_t) { return (uint8_t)bv; }, [&](uint32_t) { return v; });
   } else if (d >= 16) {
     for (uint32_t done = 0; done < M; done += d) {  // rounds of d bytes: each round's source precedes it
       const uint32_t n = (M - done) < d ? (M - done) : d;
-      write_span<32>(
-          win, op + done, op + done + n, lane, [&](uint32_t x) { return win[x - d]; },
+      write_span<NL>(
+          win, op + done, op + done + n, lid, [&](uint32_t x) { return win[x - d]; },
           [&](uint32_t x) { return gather4_window(win, (int32_t)x - (int32_t)d); });
-      __syncwarp();
+      __syncwarp(mask);
     }
   } else {
     const uint32_t src0 = op - d;
-    uint32_t rr = (uint32_t)lane % d;
-    const uint32_t step = 32u % d;
-    for (uint32_t i = lane; i < M; i += 32) {
+    uint32_t rr = (uint32_t)lid % d;
+    const uint32_t step = (uint32_t)NL % d;
+    for (uint32_t i = lid; i < M; i += NL) {
       win[op + i] = win[src0 + rr];
       rr += step;
       if (rr >= d) rr -= d;
@@ -285,7 +243,7 @@ struct WarpRing {
 // match offset | (match length - 4) << 16} (offset 0: no match). Returns 0,
 // a stream status, or kOverflow. Every step checks the bounds the oracle
 // checks, in the same order, so statuses agree. Warp-uniform.
-__device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint4 *__restrict__ out,
+__device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint32_t wcap, uint4 *__restrict__ out,
                                                 uint32_t &n_out) {
   n_out = 0;
   const uint64_t ilen = (uint64_t)(r.end - r.beg);
@@ -293,6 +251,11 @@ __device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint
   if (ilen > 0x7FFFFFFFull) return LT_ERR_CORRUPT_STREAM;  // no valid block of <= 64 KB is this long
   const uint32_t lead = (uint32_t)(r.beg - r.a0);
   const uint32_t iend = lead + (uint32_t)ilen;
+  // In-place staging: the expanding CTA puts rel byte p at window index
+  // so16 + p. That works if no literal byte's output position lies past its
+  // staged position (checked per run below).
+  bool inplace = iend <= wcap;
+  const uint32_t so16 = inplace ? (wcap - iend) & ~15u : 0u;
   uint32_t ip = lead, op = 0, n = 0, st = 0;
   for (;;) {
     if (ip >= iend) { st = LT_ERR_CORRUPT_STREAM; break; }
@@ -315,6 +278,7 @@ __device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint
       if (st) break;
     }
     if ((uint64_t)ip + lit > iend || (uint64_t)op + lit > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
+    if (lit && op > so16 + ip) inplace = false;
     const uint32_t ls = ip - lead;
     ip += lit;
     if (ip == iend) {  // the last sequence has literals only
@@ -355,6 +319,7 @@ __device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint
   cp_async_wait<0>();  // nothing may land in the ring after this block
   __syncwarp();
   n_out = n;
+  if (st == 0 && !inplace) st = kNoInPlace;
   return st;
 }
 
@@ -382,7 +347,7 @@ __global__ void __launch_bounds__(kParseWarps * 32) k_lz4_parse(const __grid_con
       r.issued = 0;
       r.done = 0;
       r.top_up(0);
-      st = parse_block(r, olen, desc + blk * kCap, n);
+      st = parse_block(r, olen, win_cap(batch.max_block_bytes), desc + blk * kCap, n);
     }
     if (lane == 0) hdr[blk] = make_uint4(n, st, 0u, 0u);
   }
@@ -429,7 +394,7 @@ __device__ int walk_block_warp(const uint8_t *__restrict__ src, uint64_t ilen, u
       } while (bb == 255);
     }
     if ((uint64_t)op + mlen > olen) return LT_ERR_CORRUPT_STREAM;
-    copy_match(win, op, d, (uint32_t)mlen, lane);
+    copy_match<32>(win, op, d, (uint32_t)mlen, lane, 0xFFFFFFFFu);
     __syncwarp();
     op += (uint32_t)mlen;
   }
@@ -439,13 +404,248 @@ __device__ int walk_block_warp(const uint8_t *__restrict__ src, uint64_t ilen, u
 // ---------------------------------------------------------------------------
 // 2. expand
 // ---------------------------------------------------------------------------
+
+// first k in [0, n) with a[k] > v (n if none); a non-decreasing
+__device__ __forceinline__ uint32_t upper_bound(const uint32_t *a, uint32_t n, int64_t v) {
+  uint32_t lo = 0, hi = n;
+  while (lo < hi) {
+    const uint32_t mid = (lo + hi) >> 1;
+    if ((int64_t)a[mid] > v) hi = mid;
+    else lo = mid + 1;
+  }
+  return lo;
+}
+
+// Per-block state of the expansion, in shared memory.
+struct Seqs {
+  uint32_t op[kCap + 1];  // output position of sequence k's literals; op[n] = block length
+  uint32_t md[kCap];      // output position of its match (op[k + 1] is the match's end)
+  uint32_t le[kCap];      // literals: end of k's literal run in the block; matches: kf | kl << 16
+  uint16_t dist[kCap];    // its match offset (0: no match)
+  uint16_t rnd[kCap];     // round after which its match is final (0: no match; 0xFFFF: not yet)
+  union {
+    uint16_t seg[kMaxWindow / 256];  // literals: last sequence starting at or before byte 256 s
+    uint16_t list[2][kCap];          // matches: unresolved sequences, by round parity
+  } u;
+  uint32_t first[3];  // first unresolved sequence, one slot per round mod 3
+  uint32_t cnt[3];    // length of the unresolved list, one slot per round mod 3
+};
+
+// Append (warp-wide) the lanes' sequences with `take` set to list `dst`,
+// counting in *cnt, and fold them into the minimum *first.
+__device__ __forceinline__ void append_pending(uint16_t *dst, uint32_t *cnt, uint32_t *first, bool take, uint32_t j,
+                                               int lane) {
+  const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
+  if (!m) return;
+  uint32_t base = 0;
+  if (lane == 0) base = atomicAdd(cnt, (uint32_t)__popc(m));
+  base = __shfl_sync(0xFFFFFFFFu, base, 0);
+  if (take) dst[base + __popc(m & ((1u << lane) - 1u))] = (uint16_t)j;
+  const uint32_t wmin = __reduce_min_sync(0xFFFFFFFFu, take ? j : 0xFFFFFFFFu);
+  if (lane == 0) atomicMin(first, wmin);
+}
+
+// Rebuild one block whose sequence index is in the workspace (n <= kCap
+// sequences, staged in place by the parse's rule). All threads of the CTA.
+//  a. stage: the compressed bytes go to the end of the window (16-byte
+//     cp.async copies), the index into Seqs;
+//  b. literals: in rounds of 16 output bytes per thread, in output order.
+//     Each thread reads the staged literal bytes of its four output words
+//     (one 4-byte gather per word), the CTA syncs, and the thread stores
+//     them as one aligned 16-byte word (bytes of a match are written too,
+//     with junk: the matches overwrite them).
+//     The parse checked that a literal's output position never lies past
+//     its staged position, so a round's stores only hit staged bytes whose
+//     output lies in this round or earlier ones -- bytes already read;
+//  c. matches: round r copies every unresolved match whose source bytes
+//     are all final after round r - 1 -- literal bytes, or bytes of matches
+//     resolved earlier -- four at a time per warp, 8 lanes each. The
+//     unresolved matches are kept in a compact list, so a round costs in
+//     proportion to what is left. The first unresolved match is always
+//     ready, so every round makes progress; once few are left (or after
+//     kMatchRounds rounds) warp 0 replays the rest in order.
+// Returns false before any output byte is written if the index is not one
+// the parse can have written (the caller then walks the block itself).
+__device__ __forceinline__ bool resolve_block(uint8_t *win, Seqs &S, const uint8_t *beg, uint32_t ilen, uint32_t olen,
+                                              uint32_t n, uint32_t wcap, const uint4 *__restrict__ dsc) {
+  const uint32_t tid = threadIdx.x;
+  const int lane = tid & 31;
+  // a. stage
+  const uint32_t lead = (uint32_t)(reinterpret_cast<uintptr_t>(beg) & 15);
+  const uint32_t iend = lead + ilen;
+  const uint32_t so16 = (wcap - iend) & ~15u;
+  const uint32_t S0 = so16 + lead;  // window index of staged block byte 0
+  const uint8_t *a0 = beg - lead;
+  const uint8_t *end = beg + ilen;
+  const uint32_t nch = (iend + 15) / 16;
+  for (uint32_t c = tid; c < nch; c += kThreads) {
+    const uint8_t *src = a0 + 16 * c;
+    uint8_t *dst = win + so16 + 16 * c;
+    if (src >= beg) {
+      const uint32_t nb = (uint32_t)((end - src) < 16 ? (end - src) : 16);
+      cp_async16(dst, src, nb);  // the rest of the 16 bytes is zero-filled
+    } else {
+      for (uint32_t i = 0; i < 16; ++i)
+        if (src + i >= beg && src + i < end) dst[i] = __ldg(src + i);
+    }
+  }
+  cp_async_commit();
+  // every index the expansion reads or writes stays inside the window if,
+  // for all k: op[k] <= md[k] <= op[k + 1] <= olen, the literal run lies in
+  // the block, and a match's offset reaches no further back than byte 0
+  bool bad = false;
+  for (uint32_t j = tid; j < n; j += kThreads) {
+    const uint4 e = dsc[j];
+    const uint32_t d = e.w & 0xFFFFu;
+    const uint32_t md = e.y + e.z;
+    if (e.y > olen || e.z > olen - e.y || e.x > ilen || e.z > ilen - e.x || d > md) bad = true;
+    S.op[j] = e.y;
+    S.md[j] = md;
+    S.le[j] = e.x + e.z;
+    S.dist[j] = (uint16_t)d;
+    S.rnd[j] = d ? (uint16_t)0xFFFF : (uint16_t)0;
+  }
+  if (tid == 0) S.op[n] = olen;
+  __syncthreads();
+  for (uint32_t j = tid; j < n; j += kThreads)
+    if (S.md[j] > S.op[j + 1]) bad = true;
+  const uint32_t nseg = (olen + 255) / 256;
+  for (uint32_t sg = tid; sg < nseg; sg += kThreads) {
+    const uint32_t u = upper_bound(S.op, n, 256 * sg);
+    S.u.seg[sg] = (uint16_t)(u ? u - 1 : 0u);
+  }
+  cp_async_wait<0>();
+  if (__syncthreads_or(bad)) return false;
+
+  // b. literals. A 4-byte output word holds literals of at most one run
+  // (two runs are separated by a match of at least 4 bytes), so each word
+  // is one 4-byte gather from the staged bytes at that run's offset.
+  for (uint32_t r0 = 0; r0 < olen; r0 += 16 * kThreads) {
+    const uint32_t p0 = r0 + 16 * tid;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    bool any = false;
+    if (p0 < olen) {
+      uint32_t k = S.u.seg[p0 >> 8];
+      uint32_t o = S.op[k], m = S.md[k], nx = S.op[k + 1];
+      int32_t delta = (int32_t)(S0 + S.le[k] - m);  // staged index of output byte p is p + delta (within k's literals)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t p = p0 + 4 * q;
+        if (p < olen) {
+          while (nx <= p + 3 && k + 1 < n) {  // k: the last sequence starting at or before the word's last byte
+            ++k;
+            o = nx;
+            m = S.md[k];
+            nx = S.op[k + 1];
+            delta = (int32_t)(S0 + S.le[k] - m);
+          }
+          if (p < m && p + 4 > o) {
+            w[q] = gather4_window(win, (int32_t)p + delta);
+            any = true;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    if (any) {
+      if (p0 + 16 <= olen) {
+        *reinterpret_cast<uint4 *>(win + p0) = make_uint4(w[0], w[1], w[2], w[3]);
+      } else {
+#pragma unroll
+        for (uint32_t i = 0; i < 16; ++i)
+          if (p0 + i < olen) win[p0 + i] = (uint8_t)(w[i >> 2] >> (8 * (i & 3)));
+      }
+    }
+  }
+
+  // c. matches: the initial list holds every sequence with a match
+  for (uint32_t j0 = 0; j0 < n; j0 += kThreads) {
+    const uint32_t j = j0 + tid;
+    bool take = false;
+    if (j < n && S.dist[j]) {
+      const uint32_t md = S.md[j], d = S.dist[j], M = S.op[j + 1] - md;
+      const uint32_t lo = md - d, hi = lo + (d < M ? d : M);
+      const uint32_t uf = upper_bound(S.op, n, lo), ul = upper_bound(S.op, n, hi - 1);
+      S.le[j] = (uf ? uf - 1 : 0u) | ((ul ? ul - 1 : 0u) << 16);  // sequences holding the source's ends
+      take = true;
+    }
+    append_pending(S.u.list[0], &S.cnt[0], &S.first[0], take, j, lane);
+  }
+  __syncthreads();
+  for (int r = 0;; ++r) {
+    const uint32_t P = S.cnt[r % 3];
+    if (P == 0) break;
+    const uint32_t F = S.first[r % 3];
+    if (r >= kMatchRounds || P <= kSerialTail) {  // few left or long chains: finish in order
+      if (tid < 32) {
+        for (uint32_t j0 = F; j0 < n; j0 += 32) {
+          const uint32_t jl = j0 + (uint32_t)lane;
+          unsigned pm = __ballot_sync(0xFFFFFFFFu, jl < n && S.rnd[jl] == 0xFFFF);
+          while (pm) {
+            const uint32_t j = j0 + (uint32_t)(__ffs(pm) - 1);
+            pm &= pm - 1;
+            const uint32_t md = S.md[j], d = S.dist[j], M = S.op[j + 1] - md;
+            copy_match<32>(win, md, d, M, lane, 0xFFFFFFFFu);
+            __syncwarp();
+          }
+        }
+      }
+      break;
+    }
+    if (tid == 0) {
+      S.first[(r + 2) % 3] = 0xFFFFFFFFu;
+      S.cnt[(r + 2) % 3] = 0;
+    }
+    const uint16_t *cur = S.u.list[r & 1];
+    uint16_t *nxt = S.u.list[(r + 1) & 1];
+    for (uint32_t i0 = 32 * (tid >> 5); i0 < P; i0 += kThreads) {  // warp-uniform
+      const uint32_t i = i0 + (uint32_t)lane;
+      uint32_t j = 0, md = 0, d = 0, M = 0;
+      bool ready = false, live = i < P;
+      if (live) {
+        j = cur[i];
+        md = S.md[j];
+        d = S.dist[j];
+        M = S.op[j + 1] - md;
+        const uint32_t lo = md - d, hi = lo + (d < M ? d : M);
+        const uint32_t kf = S.le[j] & 0xFFFFu, kl = S.le[j] >> 16;
+        ready = kl < F;
+        if (!ready) {
+          const uint32_t k0 = kf > F ? kf : F;
+          ready = kl - k0 < kScanMax;
+          for (uint32_t k = k0; ready && k <= kl; ++k)
+            if (S.rnd[k] > (uint32_t)r && S.md[k] < hi && S.op[k + 1] > lo) ready = false;
+        }
+      }
+      // the ready matches, four at a time: 8 lanes copy each
+      const unsigned rm = __ballot_sync(0xFFFFFFFFu, ready);
+      const int nr = __popc(rm);
+      const int sub = lane >> 3;
+      for (int g = 0; g < nr; g += 4) {
+        const int which = g + sub;
+        const int src = which < nr ? (int)__fns(rm, 0, which + 1) : 0;
+        const uint32_t bd = __shfl_sync(0xFFFFFFFFu, md, src), bo = __shfl_sync(0xFFFFFFFFu, d, src);
+        const uint32_t bm = __shfl_sync(0xFFFFFFFFu, M, src);
+        if (which < nr) copy_match<8>(win, bd, bo, bm, lane & 7, 0xFFu << (8 * sub));
+        __syncwarp();
+      }
+      if (ready) S.rnd[j] = (uint16_t)(r + 1);
+      append_pending(nxt, &S.cnt[(r + 1) % 3], &S.first[(r + 1) % 3], live && !ready, j, lane);
+    }
+    __syncthreads();
+  }
+  return true;
+}
+
 template <bool FUSED>
 __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constant__ Batch batch,
                                                           const uint4 *__restrict__ hdr,
                                                           const uint4 *__restrict__ desc, int32_t *d_status) {
   extern __shared__ uint4 smem_u4[];
   uint8_t *win = reinterpret_cast<uint8_t *>(smem_u4) + kPad;
-  __shared__ uint32_t progress, s_n, s_st;
+  __shared__ Seqs S;
+  __shared__ uint32_t s_n, s_st;
+  const uint32_t wcap = win_cap(batch.max_block_bytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   for (int64_t blk = blockIdx.x; blk < batch.total_blocks; blk += gridDim.x) {
@@ -465,126 +665,86 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
       }
     }
     if (threadIdx.x == 0) {
-      progress = 0;
       const uint4 h = hdr ? hdr[blk] : make_uint4(0u, kNoIndex, 0u, 0u);
       s_n = h.x;
       s_st = h.y;
+      S.first[0] = S.first[1] = S.first[2] = 0xFFFFFFFFu;
+      S.cnt[0] = S.cnt[1] = S.cnt[2] = 0;
     }
     __syncthreads();
-    const uint32_t n = s_n, st = s_st;
-    if (st != 0 && st != kOverflow && st != kNoIndex) {
+    const uint32_t n = s_n;
+    uint32_t st = s_st;
+    if (st != 0 && st != kOverflow && st != kNoIndex && st != kNoInPlace) {
       // the parse found a malformed block: report it; its output stays unwritten
       if (threadIdx.x == 0) report(d_status, (int32_t)st);
       __syncthreads();
       continue;
     }
     const uint64_t s0 = jb.offsets[b], s1 = jb.offsets[b + 1];
-    if (st == 0) {
-      // literal runs: 16 half-warps, sequence i by half-warp i mod 16
-      const uint4 *dsc = desc + blk * kCap;
-      const uint8_t *lo = jb.comp, *hi = jb.comp + jb.comp_bytes;
-      const uint8_t *g = jb.comp + s0;
-      const uint32_t hw = threadIdx.x >> 4, hl = threadIdx.x & 15;
-      for (uint32_t i = hw; i < n; i += 2 * kWarps) {
-        const uint4 e = dsc[i];
-        if (e.z) {
-          const uint8_t *sb = g + e.x - e.y;  // global source of window byte x is sb[x]
-          write_span<16>(
-              win, e.y, e.y + e.z, (int)hl, [&](uint32_t x) { return (uint8_t)__ldg(sb + x); },
-              [&](uint32_t x) { return gather4_global(sb + x, lo, hi); });
-        }
-      }
-      __syncthreads();
+    const uint32_t lead = (uint32_t)(reinterpret_cast<uintptr_t>(jb.comp + s0) & 15);
+    if (st == 0 && (n > kCap || s1 < s0 || s1 > jb.comp_bytes || s1 - s0 + lead > wcap))
+      st = kNoIndex;  // never from the parse
+    if (st == 0 && !resolve_block(win, S, jb.comp + s0, (uint32_t)(s1 - s0), olen, n, wcap, desc + blk * kCap))
+      st = kNoIndex;
+    if (st != 0 && warp == 0) {
+      int err = LT_ERR_CORRUPT_STREAM;
+      if (s0 <= s1 && s1 <= jb.comp_bytes) err = walk_block_warp(jb.comp + s0, s1 - s0, win, olen, lane);
+      if (err && lane == 0) report(d_status, err);  // content unspecified after an error
     }
-    if (warp == 0) {
-      if (st == 0) {
-        // matches, in order
-        const uint4 *dsc = desc + blk * kCap;
-        uint32_t published = 0;
-        for (uint32_t base = 0; base < n; base += 32) {
-          const uint4 mine = (base + lane < n) ? dsc[base + lane] : make_uint4(0u, 0u, 0u, 0u);
-          const uint32_t cnt = (n - base) < 32 ? (n - base) : 32;
-          for (uint32_t k = 0; k < cnt; ++k) {
-            const uint32_t pos = __shfl_sync(0xFFFFFFFFu, mine.y + mine.z, k);
-            const uint32_t dm = __shfl_sync(0xFFFFFFFFu, mine.w, k);
-            const uint32_t d = dm & 0xFFFFu;
-            if (d) {
-              copy_match(win, pos, d, (dm >> 16) + 4, lane);
-              __syncwarp();
-              const uint32_t end = pos + (dm >> 16) + 4;
-              if (end - published >= kPublishBytes) {
-                st_release_shared(&progress, end);
-                published = end;
-              }
+    __syncthreads();
+    if (FUSED) {
+      uint16_t *out = reinterpret_cast<uint16_t *>(jb.out);
+      const int64_t k0 = 2 * d0;  // first code of the block
+      const int64_t k_end = (k0 + 2 * (int64_t)olen) < jb.n_codes ? (k0 + 2 * (int64_t)olen) : jb.n_codes;
+      const uint32_t nk = (uint32_t)(k_end - k0);  // codes in this block (<= 131072)
+      const int64_t G = jb.group_size;
+      const int gs = jb.group_shift;
+      const bool vec = (G % 8 == 0) && aligned(out + k0, 16);
+      const int64_t g0 = gs >= 0 ? (k0 >> gs) : 0;
+      const uint32_t koff = gs >= 0 ? (uint32_t)(k0 - (g0 << gs)) : 0u;
+      const uint32_t nw = (nk + 7) / 8;  // window words (8 codes each)
+      for (uint32_t q = threadIdx.x; 4 * q < nw; q += kThreads) {  // 4 words = 32 codes per thread
+        const uint32_t kr = 32 * q;                                // first code
+        if (vec && G % 32 == 0 && kr + 32 <= nk) {
+          const int64_t g = gs >= 0 ? g0 + (int64_t)((koff + kr) >> gs) : (k0 + kr) / G;
+          const uint32_t s2 = bcast_half(__ldg(jb.scales + g));
+          const uint32_t zm = jb.zeros ? int4_zero_magic(__ldg(jb.zeros + g)) : 0x54006400u;
+          const uint4 v = reinterpret_cast<const uint4 *>(win)[q];
+          uint16_t *o = out + k0 + kr;
+          st_u128(o, int4x8_dequant(v.x, zm, s2));
+          st_u128(o + 8, int4x8_dequant(v.y, zm, s2));
+          st_u128(o + 16, int4x8_dequant(v.z, zm, s2));
+          st_u128(o + 24, int4x8_dequant(v.w, zm, s2));
+          continue;
+        }
+        for (uint32_t wi = 4 * q; wi < 4 * q + 4 && wi < nw; ++wi) {
+          const uint32_t kw = 8 * wi;
+          if (vec && kw + 8 <= nk) {
+            const int64_t g = gs >= 0 ? g0 + (int64_t)((koff + kw) >> gs) : (k0 + kw) / G;
+            const uint32_t s2 = bcast_half(__ldg(jb.scales + g));
+            const uint32_t zm = jb.zeros ? int4_zero_magic(__ldg(jb.zeros + g)) : 0x54006400u;
+            st_u128(out + k0 + kw, int4x8_dequant(reinterpret_cast<const uint32_t *>(win)[wi], zm, s2));
+          } else {
+            const uint32_t ke = (kw + 8) < nk ? (kw + 8) : nk;
+            for (uint32_t kk = kw; kk < ke; ++kk) {
+              const uint8_t byte = win[kk >> 1];
+              const int32_t qv = (kk & 1) ? (byte >> 4) : (byte & 0x0F);
+              const int64_t g = (k0 + kk) / G;
+              const int32_t z = jb.zeros ? jb.zeros[g] : 0;
+              out[k0 + kk] = dequant_scalar(qv - z, jb.scales[g]);
             }
           }
         }
-        __syncwarp();
-        st_release_shared(&progress, olen);
-      } else {
-        int err = LT_ERR_CORRUPT_STREAM;
-        if (s0 <= s1 && s1 <= jb.comp_bytes) err = walk_block_warp(jb.comp + s0, s1 - s0, win, olen, lane);
-        __syncwarp();
-        if (err && lane == 0) report(d_status, err);
-        st_release_shared(&progress, olen);  // content unspecified after an error
       }
     } else {
-      const uint32_t dw = (uint32_t)(warp - 1);
-      const uint32_t n_steps = (olen + kStep - 1) / kStep;
-      uint32_t seen = 0;
-      if (FUSED) {
-        uint16_t *out = reinterpret_cast<uint16_t *>(jb.out);
-        const int64_t k0 = 2 * d0;  // first code of the block
-        const int64_t k_end = (k0 + 2 * (int64_t)olen) < jb.n_codes ? (k0 + 2 * (int64_t)olen) : jb.n_codes;
-        const uint32_t nk = (uint32_t)(k_end - k0);  // codes in this block (<= 131072)
-        const int64_t G = jb.group_size;
-        const int gs = jb.group_shift;
-        const bool vec = (G % 8 == 0) && aligned(out + k0, 16);
-        const int64_t g0 = gs >= 0 ? (k0 >> gs) : 0;
-        const uint32_t koff = gs >= 0 ? (uint32_t)(k0 - (g0 << gs)) : 0u;
-        const uint32_t *win32 = reinterpret_cast<const uint32_t *>(win);
-        for (uint32_t u = dw; u < n_steps; u += kWarps - 1) {
-          const uint32_t need = (u + 1) * kStep < olen ? (u + 1) * kStep : olen;
-          if (seen < need && !wait_ge(&progress, need, seen, lane, d_status)) break;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t wi = u * (kStep / 4) + (uint32_t)q * 32 + (uint32_t)lane;  // window word
-            const uint32_t kr = 8 * wi;                                               // its first code
-            if (kr >= nk) continue;
-            if (vec && kr + 8 <= nk) {
-              const int64_t g = gs >= 0 ? g0 + (int64_t)((koff + kr) >> gs) : (k0 + kr) / G;
-              const uint32_t s2 = bcast_half(__ldg(jb.scales + g));
-              const uint32_t zm = jb.zeros ? int4_zero_magic(__ldg(jb.zeros + g)) : 0x54006400u;
-              st_u128(out + k0 + kr, int4x8_dequant(win32[wi], zm, s2));
-            } else {
-              const uint32_t ke = (kr + 8) < nk ? (kr + 8) : nk;
-              for (uint32_t kk = kr; kk < ke; ++kk) {
-                const uint8_t byte = win[kk >> 1];
-                const int32_t qv = (kk & 1) ? (byte >> 4) : (byte & 0x0F);
-                const int64_t g = (k0 + kk) / G;
-                const int32_t z = jb.zeros ? jb.zeros[g] : 0;
-                out[k0 + kk] = dequant_scalar(qv - z, jb.scales[g]);
-              }
-            }
-          }
-        }
+      uint8_t *out = reinterpret_cast<uint8_t *>(jb.out) + d0;
+      if (aligned(out, 16)) {
+        const uint32_t n16 = olen / 16;
+        for (uint32_t i = threadIdx.x; i < n16; i += kThreads)
+          st_u128(reinterpret_cast<uint4 *>(out) + i, reinterpret_cast<const uint4 *>(win)[i]);
+        for (uint32_t i = 16 * n16 + threadIdx.x; i < olen; i += kThreads) out[i] = win[i];
       } else {
-        uint8_t *out = reinterpret_cast<uint8_t *>(jb.out) + d0;
-        const bool vec = aligned(out, 4);
-        for (uint32_t u = dw; u < n_steps; u += kWarps - 1) {
-          const uint32_t need = (u + 1) * kStep < olen ? (u + 1) * kStep : olen;
-          if (seen < need && !wait_ge(&progress, need, seen, lane, d_status)) break;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t x = u * kStep + (uint32_t)q * 128 + 4 * (uint32_t)lane;
-            if (x >= olen) continue;
-            if (vec && x + 4 <= olen) {
-              *reinterpret_cast<uint32_t *>(out + x) = *reinterpret_cast<const uint32_t *>(win + x);
-            } else {
-              for (uint32_t i = x; i < olen && i < x + 4; ++i) out[i] = win[i];
-            }
-          }
-        }
+        for (uint32_t i = threadIdx.x; i < olen; i += kThreads) out[i] = win[i];
       }
     }
     __syncthreads();
@@ -605,13 +765,13 @@ lt_status launch(const Batch &batch, bool fused, void *workspace, uint64_t works
     const int64_t cap = (int64_t)num_sms() * blocks_per_sm((const void *)k_lz4_parse, kParseWarps * 32, 0);
     k_lz4_parse<<<(int)(need < cap ? need : cap), kParseWarps * 32, 0, st>>>(batch, hdr, desc);
   }
-  const size_t smem = (size_t)((batch.max_block_bytes + 15) / 16 * 16) + 2 * kPad;
+  const size_t smem = (size_t)win_cap(batch.max_block_bytes) + 2 * kPad;
   const void *k = fused ? (const void *)k_lz4_expand<true> : (const void *)k_lz4_expand<false>;
   static int attr_set[2][64] = {{0}};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[fused][dev]) {
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxWindow + 2 * kPad);
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)win_cap(kMaxWindow) + 2 * kPad);
     attr_set[fused][dev] = 1;
   }
   const int64_t cap = (int64_t)num_sms() * blocks_per_sm(k, kThreads, smem);
