@@ -42,9 +42,7 @@ constexpr uint32_t kOverflow = 0x100;    // parse status: more than kCap sequenc
 constexpr uint32_t kNoIndex = 0x101;     // no workspace: every block takes the fallback
 constexpr uint32_t kNoInPlace = 0x102;   // parse status: the block cannot be staged in its window
 constexpr uint32_t kWinSlack = 512;      // window bytes past the largest block, for in-place staging
-constexpr int kMatchRounds = 24;         // parallel match rounds before the rest is replayed in order
-constexpr uint32_t kScanMax = 8;         // sequences a match source may span and still be checked one by one
-constexpr uint32_t kSerialTail = 24;     // unresolved matches left when warp 0 takes over
+constexpr uint32_t kLevelCap = 255;      // match levels saturate here (the block is then replayed in order)
 
 // Window bytes a CTA holds for blocks of up to max_block_bytes: the block
 // plus room to stage its compressed bytes at the end.
@@ -223,7 +221,7 @@ struct WarpRing {
       issue();
     }
   }
-  // make rel bytes [pos, q) readable (q - pos <= 8)
+  // make rel bytes [pos, q) readable (pos < q <= pos + 32)
   __device__ __forceinline__ void need(uint32_t pos, uint32_t q) {
     const uint32_t c = (q - 1) / kPChunk;
     if (c < done) return;
@@ -238,14 +236,62 @@ struct WarpRing {
   __device__ __forceinline__ uint32_t at(uint32_t rel) const { return buf[rel & (kPRing - 1)]; }
 };
 
+// Sequence descriptors leave the parse one per lane, 32 at a time.
+struct DescOut {
+  uint4 *out;
+  uint4 held = make_uint4(0u, 0u, 0u, 0u);  // descriptor n with n % 32 == lane
+  uint32_t n = 0;
+  uint32_t lane;
+  __device__ __forceinline__ void push(const uint4 &e) {
+    if (lane == (n & 31)) held = e;
+    ++n;
+    if ((n & 31) == 0) out[n - 32 + lane] = held;
+  }
+  __device__ __forceinline__ void flush() {
+    if (lane < (n & 31)) out[(n & ~31u) + lane] = held;
+  }
+};
+
+// Match levels: a match's level is one more than the highest level of any
+// match that wrote bytes it reads (literals are level 0), tracked per
+// 16-byte output granule in `lmap` (4096 bytes). A granule's level is the
+// highest level of the matches writing into it, so a match that reads a
+// byte another match wrote always has the higher level, and matches of one
+// level never read each other's output: they can be copied in parallel.
+// Levels saturate at kLevelCap (the expansion then replays in order).
+struct Leveler {
+  uint8_t *lmap;
+  uint32_t lane, lmax = 0;
+  // level of the match writing [dst, dst + M) from offset d (warp-wide)
+  __device__ __forceinline__ uint32_t level(uint32_t dst, uint32_t d, uint32_t M) {
+    const uint32_t lo = dst - d, hi = lo + (d < M ? d : M);
+    const uint32_t s0 = lo >> 4, ns = ((hi - 1) >> 4) - s0;  // source granules s0 .. s0 + ns
+    const uint32_t d0 = dst >> 4, nd = ((dst + M - 1) >> 4) - d0;
+    uint32_t mx = lane <= ns ? lmap[s0 + lane] : 0u;
+    const uint32_t old0 = lmap[d0];
+    for (uint32_t g = 32 + lane; g <= ns; g += 32) mx = mx > lmap[s0 + g] ? mx : lmap[s0 + g];  // long sources
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    const uint32_t lvl = mx + 1 < kLevelCap ? mx + 1 : kLevelCap;
+    if (lane <= nd) lmap[d0 + lane] = (uint8_t)(lane == 0 && old0 > lvl ? old0 : lvl);
+    for (uint32_t g = 32 + lane; g <= nd; g += 32) lmap[d0 + g] = (uint8_t)lvl;  // long matches
+    __syncwarp();
+    lmax = lmax > lvl ? lmax : lvl;
+    return lvl;
+  }
+};
+
 // Walk LZ4 block [beg, end) that must decode to exactly olen bytes; write
-// descriptors {literal source, output position, literal length,
-// match offset | (match length - 4) << 16} (offset 0: no match). Returns 0,
-// a stream status, or kOverflow. Every step checks the bounds the oracle
-// checks, in the same order, so statuses agree. Warp-uniform.
-__device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint32_t wcap, uint4 *__restrict__ out,
-                                                uint32_t &n_out) {
+// descriptors {literal source | level << 17, output position, literal
+// length, match offset | (match length - 4) << 16} (offset 0: no match).
+// Returns 0, a stream status, kOverflow or kNoInPlace. Every step checks
+// the bounds the oracle checks, in the same order, so statuses agree.
+// Warp-uniform: every lane reads the same header bytes (broadcast). A
+// match's level is worked out one sequence later, right after the next
+// token is read, so it overlaps that read.
+__device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint32_t wcap, uint8_t *lmap,
+                                                uint4 *__restrict__ out, uint32_t &n_out, uint32_t &lmax_out) {
   n_out = 0;
+  lmax_out = 0;
   const uint64_t ilen = (uint64_t)(r.end - r.beg);
   if (ilen == 0) return olen == 0 ? 0u : (uint32_t)LT_ERR_SIZE_MISMATCH;
   if (ilen > 0x7FFFFFFFull) return LT_ERR_CORRUPT_STREAM;  // no valid block of <= 64 KB is this long
@@ -256,12 +302,28 @@ __device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint
   // staged position (checked per run below).
   bool inplace = iend <= wcap;
   const uint32_t so16 = inplace ? (wcap - iend) & ~15u : 0u;
+  for (uint32_t i = (uint32_t)r.lane; i < kMaxWindow / 16 / 16; i += 32)
+    reinterpret_cast<uint4 *>(lmap)[i] = make_uint4(0u, 0u, 0u, 0u);
+  __syncwarp();
+  DescOut dout;
+  dout.out = out;
+  dout.lane = (uint32_t)r.lane;
+  Leveler lv;
+  lv.lmap = lmap;
+  lv.lane = (uint32_t)r.lane;
+  bool pend = false;  // a match whose level is still to be worked out
+  uint4 pe = make_uint4(0u, 0u, 0u, 0u);
   uint32_t ip = lead, op = 0, n = 0, st = 0;
   for (;;) {
     if (ip >= iend) { st = LT_ERR_CORRUPT_STREAM; break; }
     r.need(ip, ip + 2 < iend ? ip + 2 : iend);
     const uint32_t token = r.at(ip);
     uint32_t b = ip + 1 < iend ? r.at(ip + 1) : 0u;
+    if (pend) {  // the previous match
+      pe.x |= lv.level(pe.y + pe.z, pe.w & 0xFFFFu, (pe.w >> 16) + 4) << 17;
+      dout.push(pe);
+      pend = false;
+    }
     ip += 1;
     uint32_t lit = token >> 4;
     if (lit == 15) {
@@ -283,7 +345,7 @@ __device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint
     ip += lit;
     if (ip == iend) {  // the last sequence has literals only
       if (n >= kCap) { st = kOverflow; break; }
-      if (r.lane == 0) out[n] = make_uint4(ls, op, lit, 0u);
+      dout.push(make_uint4(ls, op, lit, 0u));
       ++n;
       op += lit;
       if (op != olen) st = LT_ERR_SIZE_MISMATCH;
@@ -311,14 +373,17 @@ __device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint
     }
     if ((uint64_t)op + lit + mlen > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
     if (n >= kCap) { st = kOverflow; break; }
-    if (r.lane == 0) out[n] = make_uint4(ls, op, lit, d | ((mlen - 4) << 16));
+    pe = make_uint4(ls, op, lit, d | ((mlen - 4) << 16));
+    pend = true;
     ++n;
     op += lit + mlen;
     r.top_up(ip);
   }
+  if (st == 0) dout.flush();  // (a valid block ends with a literal-only sequence: nothing is pending)
   cp_async_wait<0>();  // nothing may land in the ring after this block
   __syncwarp();
   n_out = n;
+  lmax_out = lv.lmax;
   if (st == 0 && !inplace) st = kNoInPlace;
   return st;
 }
@@ -326,6 +391,7 @@ __device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint
 __global__ void __launch_bounds__(kParseWarps * 32) k_lz4_parse(const __grid_constant__ Batch batch,
                                                                 uint4 *__restrict__ hdr, uint4 *__restrict__ desc) {
   __shared__ __align__(16) uint8_t rings[kParseWarps][kPRing];
+  __shared__ __align__(16) uint8_t lmaps[kParseWarps][kMaxWindow / 16];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int64_t blk = (int64_t)blockIdx.x * kParseWarps + warp; blk < batch.total_blocks;
        blk += (int64_t)gridDim.x * kParseWarps) {
@@ -333,7 +399,7 @@ __global__ void __launch_bounds__(kParseWarps * 32) k_lz4_parse(const __grid_con
     const Job &jb = find_job(batch, blk, b);
     const uint32_t olen = block_len(jb, b);
     const uint64_t s0 = jb.offsets[b], s1 = jb.offsets[b + 1];
-    uint32_t n = 0, st;
+    uint32_t n = 0, st, lmax = 0;
     if (s1 < s0 || s1 > jb.comp_bytes) {
       st = LT_ERR_CORRUPT_STREAM;
     } else {
@@ -347,9 +413,9 @@ __global__ void __launch_bounds__(kParseWarps * 32) k_lz4_parse(const __grid_con
       r.issued = 0;
       r.done = 0;
       r.top_up(0);
-      st = parse_block(r, olen, win_cap(batch.max_block_bytes), desc + blk * kCap, n);
+      st = parse_block(r, olen, win_cap(batch.max_block_bytes), lmaps[warp], desc + blk * kCap, n, lmax);
     }
-    if (lane == 0) hdr[blk] = make_uint4(n, st, 0u, 0u);
+    if (lane == 0) hdr[blk] = make_uint4(n, st, lmax, 0u);
   }
 }
 
@@ -420,30 +486,17 @@ __device__ __forceinline__ uint32_t upper_bound(const uint32_t *a, uint32_t n, i
 struct Seqs {
   uint32_t op[kCap + 1];  // output position of sequence k's literals; op[n] = block length
   uint32_t md[kCap];      // output position of its match (op[k + 1] is the match's end)
-  uint32_t le[kCap];      // literals: end of k's literal run in the block; matches: kf | kl << 16
+  uint32_t le[kCap];      // end of its literal run in the block
   uint16_t dist[kCap];    // its match offset (0: no match)
-  uint16_t rnd[kCap];     // round after which its match is final (0: no match; 0xFFFF: not yet)
+  uint16_t lvl[kCap];     // its match level (0: no match)
   union {
     uint16_t seg[kMaxWindow / 256];  // literals: last sequence starting at or before byte 256 s
-    uint16_t list[2][kCap];          // matches: unresolved sequences, by round parity
+    struct {
+      uint32_t start[kLevelCap + 1];  // matches: first slot of each level in `order` (level counts first)
+      uint16_t order[kCap];           // sequences with a match, by level
+    } m;
   } u;
-  uint32_t first[3];  // first unresolved sequence, one slot per round mod 3
-  uint32_t cnt[3];    // length of the unresolved list, one slot per round mod 3
 };
-
-// Append (warp-wide) the lanes' sequences with `take` set to list `dst`,
-// counting in *cnt, and fold them into the minimum *first.
-__device__ __forceinline__ void append_pending(uint16_t *dst, uint32_t *cnt, uint32_t *first, bool take, uint32_t j,
-                                               int lane) {
-  const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
-  if (!m) return;
-  uint32_t base = 0;
-  if (lane == 0) base = atomicAdd(cnt, (uint32_t)__popc(m));
-  base = __shfl_sync(0xFFFFFFFFu, base, 0);
-  if (take) dst[base + __popc(m & ((1u << lane) - 1u))] = (uint16_t)j;
-  const uint32_t wmin = __reduce_min_sync(0xFFFFFFFFu, take ? j : 0xFFFFFFFFu);
-  if (lane == 0) atomicMin(first, wmin);
-}
 
 // Rebuild one block whose sequence index is in the workspace (n <= kCap
 // sequences, staged in place by the parse's rule). All threads of the CTA.
@@ -457,17 +510,13 @@ __device__ __forceinline__ void append_pending(uint16_t *dst, uint32_t *cnt, uin
 //     The parse checked that a literal's output position never lies past
 //     its staged position, so a round's stores only hit staged bytes whose
 //     output lies in this round or earlier ones -- bytes already read;
-//  c. matches: round r copies every unresolved match whose source bytes
-//     are all final after round r - 1 -- literal bytes, or bytes of matches
-//     resolved earlier -- four at a time per warp, 8 lanes each. The
-//     unresolved matches are kept in a compact list, so a round costs in
-//     proportion to what is left. The first unresolved match is always
-//     ready, so every round makes progress; once few are left (or after
-//     kMatchRounds rounds) warp 0 replays the rest in order.
+//  c. matches, one level at a time (levels come from the parse: a match
+//     reads only literals and matches of lower levels), 8 lanes per match,
+//     a CTA barrier between levels.
 // Returns false before any output byte is written if the index is not one
 // the parse can have written (the caller then walks the block itself).
 __device__ __forceinline__ bool resolve_block(uint8_t *win, Seqs &S, const uint8_t *beg, uint32_t ilen, uint32_t olen,
-                                              uint32_t n, uint32_t wcap, const uint4 *__restrict__ dsc) {
+                                              uint32_t n, uint32_t lmax, uint32_t wcap, const uint4 *__restrict__ dsc) {
   const uint32_t tid = threadIdx.x;
   const int lane = tid & 31;
   // a. stage
@@ -494,16 +543,19 @@ __device__ __forceinline__ bool resolve_block(uint8_t *win, Seqs &S, const uint8
   // for all k: op[k] <= md[k] <= op[k + 1] <= olen, the literal run lies in
   // the block, and a match's offset reaches no further back than byte 0
   bool bad = false;
+  if (lmax > kLevelCap) bad = true;
   for (uint32_t j = tid; j < n; j += kThreads) {
     const uint4 e = dsc[j];
-    const uint32_t d = e.w & 0xFFFFu;
+    const uint32_t d = e.w & 0xFFFFu, ls = e.x & 0x1FFFFu, lv = e.x >> 17;
     const uint32_t md = e.y + e.z;
-    if (e.y > olen || e.z > olen - e.y || e.x > ilen || e.z > ilen - e.x || d > md) bad = true;
+    if (e.y > olen || e.z > olen - e.y || ls > ilen || e.z > ilen - ls || d > md || (d != 0) != (lv != 0) ||
+        lv > lmax)
+      bad = true;
     S.op[j] = e.y;
     S.md[j] = md;
-    S.le[j] = e.x + e.z;
+    S.le[j] = ls + e.z;
     S.dist[j] = (uint16_t)d;
-    S.rnd[j] = d ? (uint16_t)0xFFFF : (uint16_t)0;
+    S.lvl[j] = (uint16_t)lv;
   }
   if (tid == 0) S.op[n] = olen;
   __syncthreads();
@@ -558,79 +610,75 @@ __device__ __forceinline__ bool resolve_block(uint8_t *win, Seqs &S, const uint8
     }
   }
 
-  // c. matches: the initial list holds every sequence with a match
-  for (uint32_t j0 = 0; j0 < n; j0 += kThreads) {
-    const uint32_t j = j0 + tid;
-    bool take = false;
-    if (j < n && S.dist[j]) {
-      const uint32_t md = S.md[j], d = S.dist[j], M = S.op[j + 1] - md;
-      const uint32_t lo = md - d, hi = lo + (d < M ? d : M);
-      const uint32_t uf = upper_bound(S.op, n, lo), ul = upper_bound(S.op, n, hi - 1);
-      S.le[j] = (uf ? uf - 1 : 0u) | ((ul ? ul - 1 : 0u) << 16);  // sequences holding the source's ends
-      take = true;
+  // c. matches, one level at a time
+  if (lmax >= kLevelCap) {  // levels saturated: warp 0 replays every match in order
+    __syncthreads();
+    if (tid < 32) {
+      for (uint32_t j0 = 0; j0 < n; j0 += 32) {
+        const uint32_t jl = j0 + (uint32_t)lane;
+        unsigned pm = __ballot_sync(0xFFFFFFFFu, jl < n && S.dist[jl] != 0);
+        while (pm) {
+          const uint32_t j = j0 + (uint32_t)(__ffs(pm) - 1);
+          pm &= pm - 1;
+          const uint32_t md = S.md[j];
+          copy_match<32>(win, md, S.dist[j], S.op[j + 1] - md, lane, 0xFFFFFFFFu);
+          __syncwarp();
+        }
+      }
     }
-    append_pending(S.u.list[0], &S.cnt[0], &S.first[0], take, j, lane);
+    return true;
+  }
+  // counting sort of the matches by level into S.u.m.order
+  for (uint32_t i = tid; i <= kLevelCap; i += kThreads) S.u.m.start[i] = 0;
+  __syncthreads();
+  uint32_t rank[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const uint32_t j = tid + (uint32_t)q * kThreads;
+    rank[q] = (j < n && S.lvl[j]) ? atomicAdd(&S.u.m.start[S.lvl[j]], 1u) : 0u;
   }
   __syncthreads();
-  for (int r = 0;; ++r) {
-    const uint32_t P = S.cnt[r % 3];
-    if (P == 0) break;
-    const uint32_t F = S.first[r % 3];
-    if (r >= kMatchRounds || P <= kSerialTail) {  // few left or long chains: finish in order
-      if (tid < 32) {
-        for (uint32_t j0 = F; j0 < n; j0 += 32) {
-          const uint32_t jl = j0 + (uint32_t)lane;
-          unsigned pm = __ballot_sync(0xFFFFFFFFu, jl < n && S.rnd[jl] == 0xFFFF);
-          while (pm) {
-            const uint32_t j = j0 + (uint32_t)(__ffs(pm) - 1);
-            pm &= pm - 1;
-            const uint32_t md = S.md[j], d = S.dist[j], M = S.op[j + 1] - md;
-            copy_match<32>(win, md, d, M, lane, 0xFFFFFFFFu);
-            __syncwarp();
-          }
-        }
-      }
-      break;
+  if (tid < 32) {  // exclusive scan of the level counts (levels 1..lmax; 8 per lane)
+    uint32_t c[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t lv = 8 * (uint32_t)lane + (uint32_t)i;
+      c[i] = lv <= kLevelCap ? S.u.m.start[lv] : 0u;
+      sum += c[i];
     }
-    if (tid == 0) {
-      S.first[(r + 2) % 3] = 0xFFFFFFFFu;
-      S.cnt[(r + 2) % 3] = 0;
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += v;
     }
-    const uint16_t *cur = S.u.list[r & 1];
-    uint16_t *nxt = S.u.list[(r + 1) & 1];
-    for (uint32_t i0 = 32 * (tid >> 5); i0 < P; i0 += kThreads) {  // warp-uniform
-      const uint32_t i = i0 + (uint32_t)lane;
-      uint32_t j = 0, md = 0, d = 0, M = 0;
-      bool ready = false, live = i < P;
-      if (live) {
-        j = cur[i];
-        md = S.md[j];
-        d = S.dist[j];
-        M = S.op[j + 1] - md;
-        const uint32_t lo = md - d, hi = lo + (d < M ? d : M);
-        const uint32_t kf = S.le[j] & 0xFFFFu, kl = S.le[j] >> 16;
-        ready = kl < F;
-        if (!ready) {
-          const uint32_t k0 = kf > F ? kf : F;
-          ready = kl - k0 < kScanMax;
-          for (uint32_t k = k0; ready && k <= kl; ++k)
-            if (S.rnd[k] > (uint32_t)r && S.md[k] < hi && S.op[k + 1] > lo) ready = false;
-        }
+    uint32_t run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t lv = 8 * (uint32_t)lane + (uint32_t)i;
+      if (lv <= kLevelCap) S.u.m.start[lv] = run;
+      run += c[i];
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const uint32_t j = tid + (uint32_t)q * kThreads;
+    if (j < n && S.lvl[j]) S.u.m.order[S.u.m.start[S.lvl[j]] + rank[q]] = (uint16_t)j;
+  }
+  __syncthreads();
+  // level by level: 8 lanes per match, four matches per warp at a time
+  const int warp = (int)(tid >> 5), sub = lane >> 3;
+  for (uint32_t lv = 1; lv <= lmax; ++lv) {
+    const uint32_t a = S.u.m.start[lv], end = S.u.m.start[lv + 1];  // lmax < kLevelCap: start[lmax + 1] = all matches
+    for (uint32_t base = a + 4 * (uint32_t)warp; base < end; base += 4 * kWarps) {
+      const uint32_t i = base + (uint32_t)sub;
+      if (i < end) {
+        const uint32_t j = S.u.m.order[i];
+        const uint32_t md = S.md[j];
+        copy_match<8>(win, md, S.dist[j], S.op[j + 1] - md, lane & 7, 0xFFu << (8 * sub));
       }
-      // the ready matches, four at a time: 8 lanes copy each
-      const unsigned rm = __ballot_sync(0xFFFFFFFFu, ready);
-      const int nr = __popc(rm);
-      const int sub = lane >> 3;
-      for (int g = 0; g < nr; g += 4) {
-        const int which = g + sub;
-        const int src = which < nr ? (int)__fns(rm, 0, which + 1) : 0;
-        const uint32_t bd = __shfl_sync(0xFFFFFFFFu, md, src), bo = __shfl_sync(0xFFFFFFFFu, d, src);
-        const uint32_t bm = __shfl_sync(0xFFFFFFFFu, M, src);
-        if (which < nr) copy_match<8>(win, bd, bo, bm, lane & 7, 0xFFu << (8 * sub));
-        __syncwarp();
-      }
-      if (ready) S.rnd[j] = (uint16_t)(r + 1);
-      append_pending(nxt, &S.cnt[(r + 1) % 3], &S.first[(r + 1) % 3], live && !ready, j, lane);
+      __syncwarp();
     }
     __syncthreads();
   }
@@ -644,7 +692,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
   extern __shared__ uint4 smem_u4[];
   uint8_t *win = reinterpret_cast<uint8_t *>(smem_u4) + kPad;
   __shared__ Seqs S;
-  __shared__ uint32_t s_n, s_st;
+  __shared__ uint32_t s_n, s_st, s_lmax;
   const uint32_t wcap = win_cap(batch.max_block_bytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -668,11 +716,10 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
       const uint4 h = hdr ? hdr[blk] : make_uint4(0u, kNoIndex, 0u, 0u);
       s_n = h.x;
       s_st = h.y;
-      S.first[0] = S.first[1] = S.first[2] = 0xFFFFFFFFu;
-      S.cnt[0] = S.cnt[1] = S.cnt[2] = 0;
+      s_lmax = h.z;
     }
     __syncthreads();
-    const uint32_t n = s_n;
+    const uint32_t n = s_n, lmax = s_lmax;
     uint32_t st = s_st;
     if (st != 0 && st != kOverflow && st != kNoIndex && st != kNoInPlace) {
       // the parse found a malformed block: report it; its output stays unwritten
@@ -684,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
     const uint32_t lead = (uint32_t)(reinterpret_cast<uintptr_t>(jb.comp + s0) & 15);
     if (st == 0 && (n > kCap || s1 < s0 || s1 > jb.comp_bytes || s1 - s0 + lead > wcap))
       st = kNoIndex;  // never from the parse
-    if (st == 0 && !resolve_block(win, S, jb.comp + s0, (uint32_t)(s1 - s0), olen, n, wcap, desc + blk * kCap))
+    if (st == 0 && !resolve_block(win, S, jb.comp + s0, (uint32_t)(s1 - s0), olen, n, lmax, wcap, desc + blk * kCap))
       st = kNoIndex;
     if (st != 0 && warp == 0) {
       int err = LT_ERR_CORRUPT_STREAM;
