@@ -43,6 +43,7 @@ constexpr uint32_t kNoIndex = 0x101;     // no workspace: every block takes the 
 constexpr uint32_t kNoInPlace = 0x102;   // parse status: the block cannot be staged in its window
 constexpr uint32_t kWinSlack = 512;      // window bytes past the largest block, for in-place staging
 constexpr uint32_t kLevelCap = 255;      // match levels saturate here (the block is then replayed in order)
+constexpr uint32_t kTailMatches = 32;    // matches left when warp 0 finishes the levels alone
 
 // Window bytes a CTA holds for blocks of up to max_block_bytes: the block
 // plus room to stage its compressed bytes at the end.
@@ -496,16 +497,17 @@ struct Seqs {
       uint16_t order[kCap];           // sequences with a match, by level
     } m;
   } u;
+  uint32_t tail_level;  // levels from here on hold at most kTailMatches matches in all
 };
 
 // Rebuild one block whose sequence index is in the workspace (n <= kCap
 // sequences, staged in place by the parse's rule). All threads of the CTA.
 //  a. stage: the compressed bytes go to the end of the window (16-byte
 //     cp.async copies), the index into Seqs;
-//  b. literals: in rounds of 16 output bytes per thread, in output order.
-//     Each thread reads the staged literal bytes of its four output words
+//  b. literals: in rounds of 32 output bytes per thread, in output order.
+//     Each thread reads the staged literal bytes of its eight output words
 //     (one 4-byte gather per word), the CTA syncs, and the thread stores
-//     them as one aligned 16-byte word (bytes of a match are written too,
+//     them as two aligned 16-byte words (bytes of a match are written too,
 //     with junk: the matches overwrite them).
 //     The parse checked that a literal's output position never lies past
 //     its staged position, so a round's stores only hit staged bytes whose
@@ -572,16 +574,16 @@ __device__ __forceinline__ bool resolve_block(uint8_t *win, Seqs &S, const uint8
   // b. literals. A 4-byte output word holds literals of at most one run
   // (two runs are separated by a match of at least 4 bytes), so each word
   // is one 4-byte gather from the staged bytes at that run's offset.
-  for (uint32_t r0 = 0; r0 < olen; r0 += 16 * kThreads) {
-    const uint32_t p0 = r0 + 16 * tid;
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
+  for (uint32_t r0 = 0; r0 < olen; r0 += 32 * kThreads) {
+    const uint32_t p0 = r0 + 32 * tid;
+    uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
     bool any = false;
     if (p0 < olen) {
       uint32_t k = S.u.seg[p0 >> 8];
       uint32_t o = S.op[k], m = S.md[k], nx = S.op[k + 1];
       int32_t delta = (int32_t)(S0 + S.le[k] - m);  // staged index of output byte p is p + delta (within k's literals)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 8; ++q) {
         const uint32_t p = p0 + 4 * q;
         if (p < olen) {
           while (nx <= p + 3 && k + 1 < n) {  // k: the last sequence starting at or before the word's last byte
@@ -600,11 +602,12 @@ __device__ __forceinline__ bool resolve_block(uint8_t *win, Seqs &S, const uint8
     }
     __syncthreads();
     if (any) {
-      if (p0 + 16 <= olen) {
+      if (p0 + 32 <= olen) {
         *reinterpret_cast<uint4 *>(win + p0) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4 *>(win + p0 + 16) = make_uint4(w[4], w[5], w[6], w[7]);
       } else {
 #pragma unroll
-        for (uint32_t i = 0; i < 16; ++i)
+        for (uint32_t i = 0; i < 32; ++i)
           if (p0 + i < olen) win[p0 + i] = (uint8_t)(w[i >> 2] >> (8 * (i & 3)));
       }
     }
@@ -653,12 +656,17 @@ __device__ __forceinline__ bool resolve_block(uint8_t *win, Seqs &S, const uint8
       if (lane >= o) incl += v;
     }
     uint32_t run = incl - sum;
+    const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    uint32_t tail = lmax + 1;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const uint32_t lv = 8 * (uint32_t)lane + (uint32_t)i;
       if (lv <= kLevelCap) S.u.m.start[lv] = run;
+      if (lv >= 1 && lv <= lmax && total - run <= kTailMatches && lv < tail) tail = lv;
       run += c[i];
     }
+    tail = __reduce_min_sync(0xFFFFFFFFu, tail);
+    if (lane == 0) S.tail_level = tail;
   }
   __syncthreads();
 #pragma unroll
@@ -667,9 +675,11 @@ __device__ __forceinline__ bool resolve_block(uint8_t *win, Seqs &S, const uint8
     if (j < n && S.lvl[j]) S.u.m.order[S.u.m.start[S.lvl[j]] + rank[q]] = (uint16_t)j;
   }
   __syncthreads();
-  // level by level: 8 lanes per match, four matches per warp at a time
+  // level by level: 8 lanes per match, four matches per warp at a time;
+  // the last few matches by warp 0 alone (no CTA barriers)
   const int warp = (int)(tid >> 5), sub = lane >> 3;
-  for (uint32_t lv = 1; lv <= lmax; ++lv) {
+  const uint32_t tail = S.tail_level;
+  for (uint32_t lv = 1; lv < tail; ++lv) {
     const uint32_t a = S.u.m.start[lv], end = S.u.m.start[lv + 1];  // lmax < kLevelCap: start[lmax + 1] = all matches
     for (uint32_t base = a + 4 * (uint32_t)warp; base < end; base += 4 * kWarps) {
       const uint32_t i = base + (uint32_t)sub;
@@ -681,6 +691,20 @@ __device__ __forceinline__ bool resolve_block(uint8_t *win, Seqs &S, const uint8
       __syncwarp();
     }
     __syncthreads();
+  }
+  if (tid < 32) {
+    for (uint32_t lv = tail; lv <= lmax; ++lv) {
+      const uint32_t a = S.u.m.start[lv], end = S.u.m.start[lv + 1];
+      for (uint32_t base = a; base < end; base += 4) {
+        const uint32_t i = base + (uint32_t)sub;
+        if (i < end) {
+          const uint32_t j = S.u.m.order[i];
+          const uint32_t md = S.md[j];
+          copy_match<8>(win, md, S.dist[j], S.op[j + 1] - md, lane & 7, 0xFFu << (8 * sub));
+        }
+        __syncwarp();
+      }
+    }
   }
   return true;
 }
@@ -750,21 +774,46 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
       const int64_t g0 = gs >= 0 ? (k0 >> gs) : 0;
       const uint32_t koff = gs >= 0 ? (uint32_t)(k0 - (g0 << gs)) : 0u;
       const uint32_t nw = (nk + 7) / 8;  // window words (8 codes each)
-      for (uint32_t q = threadIdx.x; 4 * q < nw; q += kThreads) {  // 4 words = 32 codes per thread
-        const uint32_t kr = 32 * q;                                // first code
-        if (vec && G % 32 == 0 && kr + 32 <= nk) {
-          const int64_t g = gs >= 0 ? g0 + (int64_t)((koff + kr) >> gs) : (k0 + kr) / G;
-          const uint32_t s2 = bcast_half(__ldg(jb.scales + g));
-          const uint32_t zm = jb.zeros ? int4_zero_magic(__ldg(jb.zeros + g)) : 0x54006400u;
-          const uint4 v = reinterpret_cast<const uint4 *>(win)[q];
-          uint16_t *o = out + k0 + kr;
-          st_u128(o, int4x8_dequant(v.x, zm, s2));
-          st_u128(o + 8, int4x8_dequant(v.y, zm, s2));
-          st_u128(o + 16, int4x8_dequant(v.z, zm, s2));
-          st_u128(o + 24, int4x8_dequant(v.w, zm, s2));
-          continue;
+      const uint32_t nq = (nw + 3) / 4;  // units of 4 words = 32 codes
+      if (vec && G % 32 == 0 && gs >= 0) {
+        // a unit lies in one group (units start at multiples of 32 codes);
+        // the scales and zero points of 8 units are loaded before any is used
+        for (uint32_t q0 = threadIdx.x; q0 < nq; q0 += 8 * kThreads) {
+          uint32_t sc[8], zr[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t q = q0 + (uint32_t)i * kThreads;
+            const int64_t g = g0 + (int64_t)((koff + 32 * (q < nq ? q : 0u)) >> gs);
+            sc[i] = q < nq ? __ldg(jb.scales + g) : 0u;
+            zr[i] = q < nq && jb.zeros ? __ldg(jb.zeros + g) : 0u;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t q = q0 + (uint32_t)i * kThreads;
+            if (q >= nq) break;
+            const uint32_t kr = 32 * q;
+            const uint32_t s2 = bcast_half((uint16_t)sc[i]);
+            const uint32_t zm = jb.zeros ? int4_zero_magic((uint8_t)zr[i]) : 0x54006400u;
+            if (kr + 32 <= nk) {
+              const uint4 v = reinterpret_cast<const uint4 *>(win)[q];
+              uint16_t *o = out + k0 + kr;
+              st_u128(o, int4x8_dequant(v.x, zm, s2));
+              st_u128(o + 8, int4x8_dequant(v.y, zm, s2));
+              st_u128(o + 16, int4x8_dequant(v.z, zm, s2));
+              st_u128(o + 24, int4x8_dequant(v.w, zm, s2));
+            } else {  // the block's last, partial unit
+              for (uint32_t kk = kr; kk < nk; ++kk) {
+                const uint8_t byte = win[kk >> 1];
+                const int32_t qv = (kk & 1) ? (byte >> 4) : (byte & 0x0F);
+                const int64_t g = (k0 + kk) / G;
+                const int32_t z = jb.zeros ? jb.zeros[g] : 0;
+                out[k0 + kk] = dequant_scalar(qv - z, jb.scales[g]);
+              }
+            }
+          }
         }
-        for (uint32_t wi = 4 * q; wi < 4 * q + 4 && wi < nw; ++wi) {
+      } else {
+        for (uint32_t wi = threadIdx.x; wi < nw; wi += kThreads) {
           const uint32_t kw = 8 * wi;
           if (vec && kw + 8 <= nk) {
             const int64_t g = gs >= 0 ? g0 + (int64_t)((koff + kw) >> gs) : (k0 + kw) / G;
