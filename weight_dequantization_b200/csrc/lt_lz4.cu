@@ -4,27 +4,25 @@
 // Phase 6.1), plus the same decoder writing raw bytes.
 //
 // The one serial part of LZ4 is the walk over sequence headers: where a
-// sequence's literals and match are depends on every length before it. A
-// warp that walks one block needs ~230 cycles per sequence (two dependent
-// shared-memory reads), i.e. ~40 us for a 64 KB block of this data, while
-// only three 64 KB windows fit in an SM's shared memory. So the walk is kept
-// off the window-holding CTAs:
-//  1. k_lz4_parse: one thread per block walks its token stream (read through
-//     L1, prefetched ahead), validates every field against the block bounds
-//     and writes a sequence index -- literal source, output position,
-//     literal length, match offset and length, 16 bytes per sequence -- to a
-//     caller-provided workspace. Thousands of blocks walk in parallel.
+// sequence's literals and match are depends on every length before it.
+// Everything else is parallel once that walk has produced an index, so a
+// call is two kernels:
+//  1. k_lz4_parse: one warp per block walks its token stream (through a
+//     small cp.async ring in shared memory), validates every field against
+//     the block bounds in the oracle's order, gives each match a dependency
+//     level, and writes a sequence index -- literal source and level,
+//     output position, literal length, match offset and length, 16 bytes per
+//     sequence -- to a caller-provided workspace. Thousands of blocks walk
+//     side by side.
 //  2. k_lz4_expand: one CTA per block (persistent, three per SM) rebuilds the
 //     block in a 64 KB shared-memory window -- decompressed bytes never reach
-//     HBM. All eight warps copy the literal runs (no dependencies) from HBM
-//     (prefetched into L2 one block ahead); then warp 0 replays the matches
-//     in order -- a match of offset d that overlaps itself repeats its last d
-//     bytes: copied in rounds of d bytes (d >= 16), as a byte fill (d == 1)
-//     or byte by byte with win[p + i] = win[p - d + (i mod d)] -- publishing
-//     how many window bytes are final, while warps 1..7 turn final window
-//     bytes into binary16 (8 codes per 4-byte word, one 16-byte store each).
-// Blocks with more than kCap sequences, and calls without a workspace, are
-// decoded by warp 0 walking the block itself (slower, same result).
+//     HBM: it stages the compressed block at the end of the window, copies
+//     all literal runs in parallel rounds, copies the matches one dependency
+//     level at a time, then turns the window into binary16 (8 codes per
+//     4-byte word, 16-byte stores).
+// Blocks with more than kCap sequences, calls without a workspace, and blocks
+// that cannot be staged in place are decoded by warp 0 walking the block
+// itself (slower, same result).
 
 #include <mutex>
 
