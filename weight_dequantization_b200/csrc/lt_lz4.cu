@@ -282,11 +282,16 @@ struct Leveler {
 // Walk LZ4 block [beg, end) that must decode to exactly olen bytes; write
 // descriptors {literal source | level << 17, output position, literal
 // length, match offset | (match length - 4) << 16} (offset 0: no match).
-// Returns 0, a stream status, kOverflow or kNoInPlace. Every step checks
-// the bounds the oracle checks, in the same order, so statuses agree.
-// Warp-uniform: every lane reads the same header bytes (broadcast). A
-// match's level is worked out one sequence later, right after the next
-// token is read, so it overlaps that read.
+// Returns 0, a stream status, kOverflow or kNoInPlace. Warp-uniform: every
+// lane reads the same header bytes (broadcast).
+//
+// Most sequences take the fast path: all header bytes readable, at most one
+// extra length byte each for the literal and the match length, and every
+// bound satisfied -- tested with flags, no branch per check. Any other
+// sequence (the last one, long lengths, anything out of bounds) is walked
+// by the slow path, which checks the bounds the oracle checks in the same
+// order, so statuses agree. A match's level is worked out one sequence
+// later, right after the next token is read, so it overlaps that read.
 __device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint32_t wcap, uint8_t *lmap,
                                                 uint4 *__restrict__ out, uint32_t &n_out, uint32_t &lmax_out) {
   n_out = 0;
@@ -314,22 +319,51 @@ __device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint
   uint4 pe = make_uint4(0u, 0u, 0u, 0u);
   uint32_t ip = lead, op = 0, n = 0, st = 0;
   for (;;) {
-    if (ip >= iend) { st = LT_ERR_CORRUPT_STREAM; break; }
-    r.need(ip, ip + 2 < iend ? ip + 2 : iend);
-    const uint32_t token = r.at(ip);
-    uint32_t b = ip + 1 < iend ? r.at(ip + 1) : 0u;
+    // --- fast path ---
+    const uint32_t ic = ip < iend ? ip : iend - 1;  // clamped: reads stay inside the block
+    r.need(ic, ic + 3 < iend ? ic + 3 : iend);
+    const uint32_t token = r.at(ic), t1 = r.at(ic + 1), t2 = r.at(ic + 2);
     if (pend) {  // the previous match
       pe.x |= lv.level(pe.y + pe.z, pe.w & 0xFFFFu, (pe.w >> 16) + 4) << 17;
       dout.push(pe);
       pend = false;
     }
+    const uint32_t lx = (token >> 4) == 15 ? 1u : 0u;  // one extra literal-length byte
+    const uint32_t lit = (token >> 4) + (lx ? t1 : 0u);
+    const uint32_t ls = ip + 1 + lx;  // first literal
+    const uint32_t mp = ls + lit;     // match offset bytes
+    // The literal side is settled before the offset bytes are fetched: that
+    // fetch may move the ring past the token, and the slow path below then
+    // uses the token and its first length byte from registers.
+    if (ip + 3 <= iend && !(lx && t1 == 255u) && mp + 3 <= iend && op + lit <= olen && n < kCap) {
+      r.need(mp, mp + 3);
+      const uint32_t o0 = r.at(mp), o1 = r.at(mp + 1), o2 = r.at(mp + 2);
+      const uint32_t d = o0 | (o1 << 8);
+      const uint32_t mx = (token & 15u) == 15u ? 1u : 0u;  // one extra match-length byte
+      const uint32_t mlen = (token & 15u) + 4 + (mx ? o2 : 0u);
+      if (!(mx && o2 == 255u) && d != 0 && d <= op + lit && op + lit + mlen <= olen) {
+        if (lit && op > so16 + ls) inplace = false;
+        pe = make_uint4(ls - lead, op, lit, d | ((mlen - 4) << 16));
+        pend = true;
+        ++n;
+        op += lit + mlen;
+        ip = mp + 2 + mx;
+        r.top_up(ip);
+        continue;
+      }
+    }
+    // --- slow path: one sequence, every check in the oracle's order; the
+    // bytes after the first length byte are read from the ring, which
+    // still holds them (see above) ---
+    if (ip >= iend) { st = LT_ERR_CORRUPT_STREAM; break; }
+    uint32_t b = ip + 1 < iend ? t1 : 0u;
     ip += 1;
-    uint32_t lit = token >> 4;
-    if (lit == 15) {
+    uint32_t slit = token >> 4;
+    if (slit == 15) {
       for (;;) {
-        if (ip >= iend || lit > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
+        if (ip >= iend || slit > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
         ip += 1;
-        lit += b;
+        slit += b;
         if (b != 255) break;
         if (ip < iend) {
           r.need(ip, ip + 1);
@@ -338,30 +372,30 @@ __device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint
       }
       if (st) break;
     }
-    if ((uint64_t)ip + lit > iend || (uint64_t)op + lit > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
-    if (lit && op > so16 + ip) inplace = false;
-    const uint32_t ls = ip - lead;
-    ip += lit;
+    if ((uint64_t)ip + slit > iend || (uint64_t)op + slit > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
+    if (slit && op > so16 + ip) inplace = false;
+    const uint32_t sls = ip - lead;
+    ip += slit;
     if (ip == iend) {  // the last sequence has literals only
       if (n >= kCap) { st = kOverflow; break; }
-      dout.push(make_uint4(ls, op, lit, 0u));
+      dout.push(make_uint4(sls, op, slit, 0u));
       ++n;
-      op += lit;
+      op += slit;
       if (op != olen) st = LT_ERR_SIZE_MISMATCH;
       break;
     }
     if (ip + 2 > iend) { st = LT_ERR_CORRUPT_STREAM; break; }
     r.need(ip, ip + 3 < iend ? ip + 3 : iend);
-    const uint32_t d = r.at(ip) | (r.at(ip + 1) << 8);
+    const uint32_t sd = r.at(ip) | (r.at(ip + 1) << 8);
     b = ip + 2 < iend ? r.at(ip + 2) : 0u;
     ip += 2;
-    if (d == 0 || d > op + lit) { st = LT_ERR_CORRUPT_STREAM; break; }
-    uint32_t mlen = (token & 15u) + 4;
+    if (sd == 0 || sd > op + slit) { st = LT_ERR_CORRUPT_STREAM; break; }
+    uint32_t smlen = (token & 15u) + 4;
     if ((token & 15u) == 15u) {
       for (;;) {
-        if (ip >= iend || mlen > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
+        if (ip >= iend || smlen > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
         ip += 1;
-        mlen += b;
+        smlen += b;
         if (b != 255) break;
         if (ip < iend) {
           r.need(ip, ip + 1);
@@ -370,12 +404,12 @@ __device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint
       }
       if (st) break;
     }
-    if ((uint64_t)op + lit + mlen > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
+    if ((uint64_t)op + slit + smlen > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
     if (n >= kCap) { st = kOverflow; break; }
-    pe = make_uint4(ls, op, lit, d | ((mlen - 4) << 16));
+    pe = make_uint4(sls, op, slit, sd | ((smlen - 4) << 16));
     pend = true;
     ++n;
-    op += lit + mlen;
+    op += slit + smlen;
     r.top_up(ip);
   }
   if (st == 0) dout.flush();  // (a valid block ends with a literal-only sequence: nothing is pending)
@@ -505,8 +539,8 @@ struct Seqs {
 //  b. literals: in rounds of 32 output bytes per thread, in output order.
 //     Each thread reads the staged literal bytes of its eight output words
 //     (one 4-byte gather per word), the CTA syncs, and the thread stores
-//     them as two aligned 16-byte words (bytes of a match are written too,
-//     with junk: the matches overwrite them).
+//     them (bytes of a match are written too, with junk: the matches
+//     overwrite them).
 //     The parse checked that a literal's output position never lies past
 //     its staged position, so a round's stores only hit staged bytes whose
 //     output lies in this round or earlier ones -- bytes already read;
