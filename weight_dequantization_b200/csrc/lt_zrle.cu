@@ -5,13 +5,16 @@
 // One warp per chunk, no shared memory (so up to 64 warps per SM keep the
 // HBM streams busy):
 //  1. the chunk's output is zero-filled with 16-byte stores;
-//  2. the encoded bytes are read 128 at a time into registers (4 bytes per
-//     lane = two 16-bit fields per lane), realigned to the chunk's 16-bit
-//     grid with funnel shifts;
-//  3. the records are walked in the registers -- each step reads a
-//     record's (zero run, literal count) pair with two warp shuffles -- and
-//     the lanes holding a record's literals store them to their output
-//     positions (L2 merges these with the zero fill before HBM sees them).
+//  2. the encoded bytes are read 128 at a time into registers (two 16-bit
+//     fields per lane), realigned to the chunk's 16-bit grid with funnel
+//     shifts;
+//  3. in each window the warp walks the record chain -- one shuffle per
+//     record reads its (zero run, literal count) -- and parks record k's
+//     position and header in lane k; then all records of the window are
+//     finished in parallel: a warp scan gives each record's output offset,
+//     a vote finds the first bad record (the oracle's checks, in its order),
+//     and every lane stores the literals it holds (L2 merges them with the
+//     zero fill before HBM sees them).
 // A record whose literals run past the 128-byte window carries over into
 // the next window. Every loop is bounded by the chunk's byte range.
 #include "lt_common.cuh"
@@ -51,11 +54,11 @@ __device__ __forceinline__ void zero_fill(uint16_t *out, uint32_t len, int lane)
   for (uint32_t i = i0 + 8 * n16 + lane; i < len; i += 32) out[i] = 0;
 }
 
-__global__ void __launch_bounds__(kThreads) k_zrle(const uint8_t *__restrict__ enc, uint64_t enc_bytes,
+__global__ void __launch_bounds__(kThreads, 6) k_zrle(const uint8_t *__restrict__ enc, uint64_t enc_bytes,
                                                    const uint64_t *__restrict__ offsets, int64_t n, int32_t chunk,
                                                    int64_t n_chunks, uint16_t *__restrict__ out,
                                                    int32_t *d_status) {
-  const int lane = threadIdx.x & 31;
+  const uint32_t lane = threadIdx.x & 31;
   const int64_t warp_global = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int64_t warps_total = (int64_t)gridDim.x * kWarps;
 
@@ -63,7 +66,7 @@ __global__ void __launch_bounds__(kThreads) k_zrle(const uint8_t *__restrict__ e
     const int64_t e0 = c * (int64_t)chunk;
     const uint32_t len = (uint32_t)((n - e0) < chunk ? (n - e0) : chunk);
     uint16_t *o = out + e0;
-    zero_fill(o, len, lane);
+    zero_fill(o, len, (int)lane);
     __syncwarp();  // the literal stores below land after the zero fill
 
     const uint64_t b0 = offsets[c], b1 = offsets[c + 1];
@@ -72,7 +75,7 @@ __global__ void __launch_bounds__(kThreads) k_zrle(const uint8_t *__restrict__ e
       continue;
     }
     const uint64_t nbytes = b1 - b0;  // the chunk's bytes
-    uint32_t done = 0;                // elements produced
+    uint32_t done = 0;                // elements accounted for (zero runs and literals)
     uint64_t q = 0;                   // byte offset of the window in the chunk (even)
     uint32_t p = 0;                   // next record start, in 16-bit slots from q
     uint32_t lit_rem = 0, lit_out = 0;  // literals carried over from the previous window
@@ -84,16 +87,19 @@ __global__ void __launch_bounds__(kThreads) k_zrle(const uint8_t *__restrict__ e
         break;
       }
       // window: chunk bytes [q, q + 128) as 64 u16 slots; lane l holds slots
-      // 2l (low half) and 2l + 1 (high half)
+      // 2l, 2l + 1 in `pair` and slots 2l + 1, 2l + 2 in `podd`
       const uint64_t A = b0 + q;  // absolute byte index of slot 0
       const uint64_t al = A & ~uint64_t(3);
       const uint32_t sh = (uint32_t)(A & 3) * 8;
       const uint32_t w0 = load_word(enc, al + 4 * (uint64_t)lane, enc_bytes);
       const uint32_t w33 = (lane == 31) ? load_word(enc, al + 128, enc_bytes) : 0u;
+      const uint32_t w34 = (lane == 31) ? load_word(enc, al + 132, enc_bytes) : 0u;
       uint32_t w1 = __shfl_down_sync(0xFFFFFFFFu, w0, 1);
       if (lane == 31) w1 = w33;
       const uint32_t pair = __funnelshift_r(w0, w1, sh);  // slots 2*lane, 2*lane + 1
-      // slots that exist in the chunk's bytes
+      uint32_t pnext = __shfl_down_sync(0xFFFFFFFFu, pair, 1);
+      if (lane == 31) pnext = __funnelshift_r(w33, w34, sh);  // slots 64, 65
+      const uint32_t podd = __funnelshift_r(pair, pnext, 16);  // slots 2*lane + 1, 2*lane + 2
       const uint64_t win_bytes = (nbytes - q) < kWin ? (nbytes - q) : kWin;
       const uint32_t win_slots = (uint32_t)(win_bytes / 2);
 
@@ -101,7 +107,7 @@ __global__ void __launch_bounds__(kThreads) k_zrle(const uint8_t *__restrict__ e
       if (lit_rem) {
         const uint32_t take = lit_rem < win_slots ? lit_rem : win_slots;
         for (int h = 0; h < 2; ++h) {
-          const uint32_t s = 2 * (uint32_t)lane + h;
+          const uint32_t s = 2 * lane + h;
           if (s < take) o[lit_out + s] = (uint16_t)(h ? (pair >> 16) : (pair & 0xFFFFu));
         }
         lit_rem -= take;
@@ -116,43 +122,79 @@ __global__ void __launch_bounds__(kThreads) k_zrle(const uint8_t *__restrict__ e
           continue;
         }
       }
-      // 2. records starting in this window (header fully inside it)
-      while (done < len && p + 1 < 64) {
-        if (p + 1 >= win_slots) {  // the chunk's bytes end before the next header: too few records
-          err = LT_ERR_SIZE_MISMATCH;
-          break;
+      // 2. walk the records whose header lies in this window and in the
+      //    chunk's bytes, until the chunk is accounted for; record k's slot
+      //    and header go to lane k
+      const int32_t lim = nbytes >= q + 4 ? (int32_t)((nbytes - q - 4) / 2 < 62 ? (nbytes - q - 4) / 2 : 62) : -1;
+      const uint32_t rem = len - done;
+      uint32_t pp = p, k = 0, dsum = 0, myP = 0, myV = 0;
+      while ((int32_t)pp <= lim && dsum < rem) {  // at most 32 records: each takes >= 2 slots
+        const uint32_t v = __shfl_sync(0xFFFFFFFFu, (pp & 1) ? podd : pair, (int)(pp >> 1));
+        if (lane == k) {
+          myP = pp;
+          myV = v;
         }
-        const uint32_t zp = __shfl_sync(0xFFFFFFFFu, pair, p >> 1);
-        const uint32_t np = __shfl_sync(0xFFFFFFFFu, pair, (p + 1) >> 1);
-        const uint32_t zrun = (p & 1) ? (zp >> 16) : (zp & 0xFFFFu);
-        const uint32_t nlit = ((p + 1) & 1) ? (np >> 16) : (np & 0xFFFFu);
-        if ((uint64_t)done + zrun + nlit > len || q + 2 * ((uint64_t)p + 2 + nlit) > nbytes) {
-          err = LT_ERR_CORRUPT_STREAM;
-          break;
-        }
-        done += zrun;
-        const uint32_t ls = p + 2;  // first literal slot
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t s = 2 * (uint32_t)lane + h;
-          if (s >= ls && s < ls + nlit && s < 64) o[done + (s - ls)] = (uint16_t)(h ? (pair >> 16) : (pair & 0xFFFFu));
-        }
-        if (ls + nlit > 64) {  // literals continue in the next window(s)
-          const uint32_t in_win = ls < 64 ? 64 - ls : 0u;
-          lit_rem = nlit - in_win;
-          lit_out = done + in_win;
-        }
-        done += nlit;
-        p = ls + nlit;
+        ++k;
+        dsum += (v & 0xFFFFu) + (v >> 16);
+        pp += 2 + (v >> 16);
       }
-      if (err) break;
+      // 3. the walked records, in parallel
+      const bool rec = lane < k;
+      const uint32_t zr = myV & 0xFFFFu, nl = myV >> 16;
+      const uint32_t lk = rec ? zr + nl : 0u;
+      uint32_t incl = lk;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if ((int)lane >= off) incl += t;
+      }
+      const uint32_t before = incl - lk;  // elements of the window's earlier records
+      const bool bad = rec && ((uint64_t)done + before + lk > len || q + 2 * ((uint64_t)myP + 2 + nl) > nbytes);
+      const unsigned badm = __ballot_sync(0xFFFFFFFFu, bad);
+      const uint32_t ok = badm ? (uint32_t)(__ffs(badm) - 1) : k;  // records before the first bad one
+      const bool live = lane < ok;
+      const uint32_t mlo = __reduce_or_sync(0xFFFFFFFFu, live && myP < 32 ? 1u << myP : 0u);
+      const uint32_t mhi = __reduce_or_sync(0xFFFFFFFFu, live && myP >= 32 ? 1u << (myP - 32) : 0u);
+      const uint32_t lend = myP + 2 + nl < 64 ? myP + 2 + nl : 64u;
+      const uint32_t span = (myP + 2) | (lend << 16);     // the record's literal slots in this window
+      const uint32_t obase = done + before + zr - (myP + 2);  // output index of literal slot s: obase + s
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t s = 2 * lane + h;  // the slot this lane holds
+        const uint32_t cnt = __popc(mlo & (s >= 31 ? 0xFFFFFFFFu : (2u << s) - 1u)) +
+                             (s >= 32 ? __popc(mhi & (s == 63 ? 0xFFFFFFFFu : (2u << (s - 32)) - 1u)) : 0);
+        const int r = cnt ? (int)cnt - 1 : 0;  // the last record starting at or before s
+        const uint32_t sp = __shfl_sync(0xFFFFFFFFu, span, r);
+        const uint32_t ob = __shfl_sync(0xFFFFFFFFu, obase, r);
+        if (cnt && s >= (sp & 0xFFFFu) && s < (sp >> 16)) o[ob + s] = (uint16_t)(h ? (pair >> 16) : (pair & 0xFFFFu));
+      }
+      if (badm) {
+        err = LT_ERR_CORRUPT_STREAM;
+        break;
+      }
+      // 4. carry-over from the window's last record, and the next window
+      if (k) {
+        const uint32_t lastP = __shfl_sync(0xFFFFFFFFu, myP, (int)k - 1);
+        const uint32_t lastV = __shfl_sync(0xFFFFFFFFu, myV, (int)k - 1);
+        const uint32_t lastB = __shfl_sync(0xFFFFFFFFu, before, (int)k - 1);
+        const uint32_t lend_all = lastP + 2 + (lastV >> 16);
+        if (lend_all > 64) {
+          lit_rem = lend_all - 64;
+          lit_out = done + lastB + (lastV & 0xFFFFu) + (64 - lastP - 2);
+        }
+      }
+      done += dsum;
       if (done >= len && !lit_rem) break;
-      // next window: at the next record's header (or past the carried literals)
-      if (p < 64) {
-        q += 2 * (uint64_t)p;
-        p = 0;
-      } else {
+      if (done < len && (int32_t)pp <= 62 && (int32_t)pp > lim) {  // the next header does not fit in the chunk's bytes
+        err = LT_ERR_SIZE_MISMATCH;
+        break;
+      }
+      if (lit_rem) {
         q += kWin;
-        p -= 64;
+        p = pp - 64;
+      } else {
+        q += 2 * (uint64_t)pp;
+        p = 0;
       }
     }
     if (err && lane == 0) report(d_status, err);
