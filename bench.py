@@ -227,6 +227,8 @@ class DeviceWorkload:
         self.torch = torch
         self.hw = hw
         self.h2d = []  # (pinned host tensor, device tensor)
+        self.unit_h2d = {}  # unit ("C1", ..., ("C5", layer)) -> its (pinned host, device) pairs
+        unit = [None]
 
         def put(a):
             if a is None:
@@ -242,22 +244,27 @@ class DeviceWorkload:
                 ph = torch.empty_like(host).pin_memory()
                 ph.copy_(host)
                 self.h2d.append((ph, d))
+                self.unit_h2d.setdefault(unit[0], []).append((ph, d))
             return d
 
         if "C1" in hw:
             c1 = hw["C1"]
+            unit[0] = "C1"
             self.c1 = dict(packed=put(c1["packed"]), scales=put(c1["scales"]), zeros=put(c1["zeros"]))
             self.c1_out = torch.empty(c1["rows"] * c1["cols"], dtype=torch.float16, device="cuda")
         if "C2" in hw:
             c2 = hw["C2"]
+            unit[0] = "C2"
             self.c2 = dict(q=put(c2["q"]), scales=put(c2["scales"]))
             self.c2_out = torch.empty(c2["rows"] * c2["cols"], dtype=torch.float16, device="cuda")
         if "C3" in hw:
             c3 = hw["C3"]
+            unit[0] = "C3"
             self.c3 = dict(enc=put(c3["enc"]), offsets=put(c3["offsets"]))
             self.c3_out = torch.empty(c3["n"], dtype=torch.float16, device="cuda")
         if "C4" in hw:
             c4 = hw["C4"]
+            unit[0] = "C4"
             self.c4 = dict(comp=put(c4["comp"]), offsets=put(c4["offsets"]), scales=put(c4["scales"]),
                            zeros=put(c4["zeros"]))
             self.c4_out = torch.empty(c4["rows"] * c4["cols"], dtype=torch.float16, device="cuda")
@@ -265,7 +272,8 @@ class DeviceWorkload:
         if "C5" in hw:
             layer_elems = max(sum(m["rows"] * m["cols"] for m in mats) for mats in hw["C5"])
             self.c5_out = torch.empty(layer_elems, dtype=torch.float16, device="cuda")  # one reused layer buffer
-            for mats in hw["C5"]:
+            for li, mats in enumerate(hw["C5"]):
+                unit[0] = ("C5", li)
                 descs, base = [], 0
                 for m in mats:
                     n = m["rows"] * m["cols"]
@@ -286,12 +294,39 @@ class DeviceWorkload:
         self.status_host = torch.zeros(1, dtype=torch.int32).pin_memory() if pinned else None
         self.h2d_bytes = sum(int(p.numel() * p.element_size()) for p, _ in self.h2d)
 
-    # one pass of the whole hot path; `ev` (optional) receives per-codec events
-    def step(self, ev=None):
+    def units(self):
+        """The decode calls of one step, in order."""
+        hw = self.hw
+        return [u for u in ("C1", "C2", "C3", "C4") if u in hw] + [("C5", i) for i in range(len(self.c5))]
+
+    def run_unit(self, u, s):
+        """Issue unit u's decode call on stream s."""
         from weight_dequantization_b200 import lt_decode as L
 
-        torch = self.torch
         hw = self.hw
+        if u == "C1":
+            c1 = hw["C1"]
+            L.lt_dequant_int4(self.c1["packed"], self.c1["scales"], self.c1["zeros"], c1["rows"], c1["cols"],
+                              c1["group_size"], self.c1_out, s)
+        elif u == "C2":
+            c2 = hw["C2"]
+            L.lt_dequant_int8(self.c2["q"], self.c2["scales"], None, L.LT_SCALE_PER_ROW, c2["rows"], c2["cols"],
+                              self.c2_out, s)
+        elif u == "C3":
+            c3 = hw["C3"]
+            L.lt_zrle_decode(self.c3["enc"], int(c3["enc"].size), self.c3["offsets"], c3["n"], c3["chunk_elems"],
+                             self.c3_out, self.status, s)
+        elif u == "C4":
+            c4 = hw["C4"]
+            L.lt_lz4_int4_decode(self.c4["comp"], int(c4["comp"].size), self.c4["offsets"], c4["block_bytes"],
+                                 self.c4["scales"], self.c4["zeros"], c4["rows"], c4["cols"], c4["group_size"],
+                                 self.c4_out, self.ws, self.status, s)
+        else:
+            L.lt_lz4_int4_decode_batch(self.c5[u[1]], self.ws, self.status, s)
+
+    # one pass of the whole hot path; `ev` (optional) receives per-codec events
+    def step(self, ev=None):
+        torch = self.torch
         s = torch.cuda.current_stream()
 
         def mark(key):
@@ -302,36 +337,30 @@ class DeviceWorkload:
 
         mark("start")
         n = 0
-        if "C1" in hw:
-            c1 = hw["C1"]
-            L.lt_dequant_int4(self.c1["packed"], self.c1["scales"], self.c1["zeros"], c1["rows"], c1["cols"],
-                              c1["group_size"], self.c1_out, s)
-            mark("C1")
-            n += 1
-        if "C2" in hw:
-            c2 = hw["C2"]
-            L.lt_dequant_int8(self.c2["q"], self.c2["scales"], None, L.LT_SCALE_PER_ROW, c2["rows"], c2["cols"],
-                              self.c2_out, s)
-            mark("C2")
-            n += 1
-        if "C3" in hw:
-            c3 = hw["C3"]
-            L.lt_zrle_decode(self.c3["enc"], int(c3["enc"].size), self.c3["offsets"], c3["n"], c3["chunk_elems"],
-                             self.c3_out, self.status, s)
-            mark("C3")
-            n += 1
-        if "C4" in hw:
-            c4 = hw["C4"]
-            L.lt_lz4_int4_decode(self.c4["comp"], int(c4["comp"].size), self.c4["offsets"], c4["block_bytes"],
-                                 self.c4["scales"], self.c4["zeros"], c4["rows"], c4["cols"], c4["group_size"],
-                                 self.c4_out, self.ws, self.status, s)
-            mark("C4")
-            n += 1
-        for descs in self.c5:
-            L.lt_lz4_int4_decode_batch(descs, self.ws, self.status, s)
-            mark("C5")
+        for u in self.units():
+            self.run_unit(u, s)
+            mark(u if isinstance(u, str) else "C5")
             n += 1
         return n  # kernel launches of this step
+
+    def e2e_step(self, cs, freed):
+        """One step end to end: each unit's inputs are copied from pinned host
+        memory on stream cs while the previous unit decodes on the current
+        stream; a unit's copy waits until its buffers' last decode is done
+        (`freed`: one event per unit, recorded after each decode)."""
+        torch = self.torch
+        s = torch.cuda.current_stream()
+        for i, u in enumerate(self.units()):
+            cs.wait_event(freed[i])
+            with torch.cuda.stream(cs):
+                for ph, d in self.unit_h2d.get(u, []):
+                    d.copy_(ph, non_blocking=True)
+            copied = torch.cuda.Event()
+            copied.record(cs)
+            s.wait_event(copied)
+            self.run_unit(u, s)
+            freed[i].record(s)
+        self.download_status()
 
     def upload_inputs(self):
         for ph, d in self.h2d:
@@ -551,7 +580,8 @@ def run_lt(args, rank, world, local):
                 "peak_kind": peak_kind, "algorithmic_bytes_per_launch": launch_bytes,
                 "frac_of_8TBps": achieved / NOMINAL_HBM_GBS}
 
-    # end-to-end: inputs copied from pinned host memory every step, status read back
+    # end-to-end: every step copies all its inputs from pinned host memory and
+    # reads the status back; unit i + 1's copy overlaps unit i's decode
     torch.cuda.synchronize()
     dw.upload_inputs()
     torch.cuda.synchronize()
@@ -560,11 +590,15 @@ def run_lt(args, rank, world, local):
     f0 = torch.cuda.Event(enable_timing=True)
     f1 = torch.cuda.Event(enable_timing=True)
     KE = max(1, args.e2e_steps)
+    cs = torch.cuda.Stream()
     f0.record(s)
+    freed = []
+    for _ in dw.units():  # every unit's buffers are free at the start of the timed region
+        e = torch.cuda.Event()
+        e.record(s)
+        freed.append(e)
     for _ in range(KE):
-        dw.upload_inputs()
-        dw.step()
-        dw.download_status()
+        dw.e2e_step(cs, freed)
     f1.record(s)
     torch.cuda.synchronize()
     e2e_t = max_over_ranks(f0.elapsed_time(f1) / 1e3, dist)
