@@ -367,3 +367,52 @@ def test_lz4_compressed_stream_not_16_byte_aligned(shift):
     assert int(stat.item()) == 0
     o = out.cpu().numpy()
     assert np.array_equal(o[:raw.size], raw) and np.all(o[raw.size:] == 0xEE)
+
+
+# --------------------------------------------------------------------------- dependency depth
+
+def _chain_block(n_matches: int, out_len: int, seed: int):
+    """One LZ4 block whose matches form a single dependency chain: after 8
+    literal bytes, every sequence is one literal byte and a 4-byte match of
+    offset 5, which copies exactly the previous match's output; a literal
+    run fills the block to `out_len` bytes (the format's end rules)."""
+    from tests._lz4gen import _sequence
+
+    rng = np.random.default_rng(seed)
+    lits = rng.integers(0, 256, 8, dtype=np.uint8).tobytes()
+    comp = bytearray()
+    out = bytearray(lits)
+    first = True
+    for _ in range(n_matches):
+        lit = rng.integers(0, 256, 1, dtype=np.uint8).tobytes()
+        seq_lits = (lits + lit) if first else lit
+        first = False
+        out += lit
+        for _ in range(4):
+            out.append(out[-5])
+        comp += _sequence(seq_lits, 5, 4)
+    tail = rng.integers(0, 256, out_len - len(out), dtype=np.uint8).tobytes()
+    assert len(tail) >= 12
+    comp += _sequence(tail, 0, 0)
+    out += tail
+    return np.frombuffer(bytes(comp), np.uint8).copy(), np.frombuffer(bytes(out), np.uint8).copy()
+
+
+@pytest.mark.parametrize("ws", ["ws", "none"])
+@pytest.mark.parametrize("n_matches", [100, 400])
+def test_lz4_long_match_dependency_chains(n_matches, ws):
+    # 100 chained matches: 100 match levels, copied level by level (CTA-wide,
+    # then the last ones by one warp); 400: the levels saturate and the block
+    # is replayed in stream order. Both must give the oracle's bytes.
+    comp, want = _chain_block(n_matches, 2048, seed=n_matches)
+    got_o, st_o = oracle.lz4_block_decode(comp, want.size)
+    assert st_o == 0 and np.array_equal(got_o, want)
+    got, st = run_raw(comp, np.array([0, comp.size], np.uint64), 2048, want.size, ws)
+    assert st == 0 and np.array_equal(got, want)
+    # the same block through the fused decode: 2 x 2048 codes, G 128
+    d = dict(rows=2, cols=2048, group_size=128, block_bytes=2048, comp=comp, offsets=np.array([0, comp.size], np.uint64),
+             scales=fp16_uniform(n_matches, 32, 0.001, 0.1, stream=1), zeros=u8_uniform(n_matches, 32, 0, 15, stream=2))
+    got_f, st_f = run_fused(d, ws=ws)
+    want_f, st_of = oracle_fused(d)
+    assert st_f == st_of == 0
+    assert_f16_parity(got_f, want_f, what="fused decode of a dependency chain")
