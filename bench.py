@@ -490,6 +490,17 @@ def oracle_sample_tasks(hw, frac: float, pieces: int):
     return tasks
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline_threads(hw, frac: float):
     """The same oracle sample as cpu_baseline, spread over all host cores:
     independent pieces on a thread pool (the oracle's C code runs without
@@ -505,7 +516,7 @@ def cpu_baseline_threads(hw, frac: float):
     if any(st != 0 for _, st in results):
         raise RuntimeError("the oracle reported an error in the threaded sample")
     dec = sum(b for _, b in tasks)
-    return {"value": dec / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+    return {"value": dec / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle", "cpu": cpu_model(),
             "sample": f"the cpu_baseline sample ({dec / 1e6:.1f} MB decoded) in {len(tasks)} independent pieces "
                       f"on {threads} threads, {dt:.2f} s"}
 
@@ -519,7 +530,7 @@ def cpu_baseline(hw, budget_s: float = 15.0):
         frac = frac2
         dec, dt = oracle_sample_step(hw, frac)
     return {
-        "value": dec / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+        "value": dec / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle", "cpu": cpu_model(),
         "sample": f"first {frac:.4%} of the units (rows, chunks, 64 KB blocks) of every workload of one step "
                   f"({dec / 1e6:.1f} MB decoded in {dt:.1f} s, single-threaded plain C oracle)",
         "frac": frac,
@@ -679,24 +690,32 @@ def run_lt(args, rank, world, local):
     K = args.steps
     order = [c for c in ("C1", "C2", "C3", "C4") if c in hw] + ["C5"] * len(dw.c5)
     t_c = {c: 0.0 for c in alg}
+    per_step = {c: [] for c in alg}  # device ms of the codec's launches in each step
     layer_t = []
     idx = {c: 0 for c in set(order)}
     for k in range(K):
         prev = ev["start"][k]
+        step_c = {c: 0.0 for c in alg}
         for c in order:
             cur = ev[c][idx[c]]
             idx[c] += 1
             dt = prev.elapsed_time(cur)
             t_c[c] += dt
+            step_c[c] += dt
             if c == "C5":
                 layer_t.append(dt)
             prev = cur
+        for c in alg:
+            per_step[c].append(step_c[c])
     L5 = max(1, len(dw.c5))
     peak, peak_kind = read_peaks()
     per_codec = {}
     for c, (rd, wr) in alg.items():
         t = t_c[c] / 1e3 / K
-        per_codec[c] = {"decoded_GBps": wr / t / 1e9, "us_per_call": t * 1e6 / (L5 if c == "C5" else 1),
+        calls = L5 if c == "C5" else 1
+        per_codec[c] = {"decoded_GBps": wr / t / 1e9, "us_per_call": t * 1e6 / calls,
+                        "us_per_call_median": statistics.median(per_step[c]) * 1e3 / calls,
+                        "us_per_call_min": min(per_step[c]) * 1e3 / calls,
                         "bytes_read": rd, "bytes_written": wr,
                         "hbm_frac_of_measured": (rd + wr) / t / 1e9 / peak,
                         "hbm_frac_of_8TBps": (rd + wr) / t / 1e9 / NOMINAL_HBM_GBS}
