@@ -7,7 +7,8 @@ One step = one pass of every decode workload over its synthetic input:
   C3  zero-run decode, 8 x 2048 x 11008 fp16 ReLU-like activations
   C4  fused LZ4 -> INT4 -> fp16, 4096 x 14336, group 128, 64 KB blocks
   C5  8 Llama-2-70B-shaped layers (q, o, k, v, gate, up, down), fused LZ4 ->
-      INT4 -> fp16, each layer decoded (one launch) into one reused buffer
+      INT4 -> fp16: one index launch over the blocks of all layers, then each
+      layer expanded (one launch) into one reused buffer
 The headline value is the step's total decoded fp16 bytes / step time
 (GB/s, 1e9). Inputs are resident in HBM when the timed region starts; the
 step touches ~16 GB, far more than L2, so no L2 flush is needed between
@@ -283,21 +284,33 @@ class DeviceWorkload:
                                       cols=m["cols"], group_size=m["group_size"], block_bytes=m["block_bytes"]))
                     base += n
                 self.c5.append(descs)
-        # LZ4 workspace (sequence index), sized for the largest single call
+        # LZ4 workspace (sequence index), sized for the largest call: the
+        # C5 index covers every layer (the layers are then expanded one by one)
         from weight_dequantization_b200 import lt_decode as L
 
+        self.c5_first, tot = [], 0
+        for descs in self.c5:
+            self.c5_first.append(tot)
+            tot += sum(L.desc_blocks(d) for d in descs)
+        self.c5_blocks = tot
+        self.c5_all = [d for descs in self.c5 for d in descs]
         nblk = [len(hw["C4"]["offsets"]) - 1] if "C4" in hw else []
-        nblk += [sum(len(m["offsets"]) - 1 for m in mats) for mats in hw.get("C5", [])]
+        nblk += [sum(len(m["offsets"]) - 1 for m in mats) for mats in hw.get("C5", [])] + [tot]
         self.ws = torch.empty(max([L.lt_lz4_workspace_bytes(n) for n in nblk] + [16]), dtype=torch.uint8,
                               device="cuda")
         self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
         self.status_host = torch.zeros(1, dtype=torch.int32).pin_memory() if pinned else None
         self.h2d_bytes = sum(int(p.numel() * p.element_size()) for p, _ in self.h2d)
 
-    def units(self):
-        """The decode calls of one step, in order."""
+    def units(self, two_step: bool = True):
+        """The decode calls of one step, in order. two_step: C5 as one index
+        call over all layers, then one expand call per layer; otherwise one
+        decode call per layer."""
         hw = self.hw
-        return [u for u in ("C1", "C2", "C3", "C4") if u in hw] + [("C5", i) for i in range(len(self.c5))]
+        c5 = [("C5", i) for i in range(len(self.c5))]
+        if two_step and c5:
+            c5 = ["C5index"] + [("C5x", i) for i in range(len(self.c5))]
+        return [u for u in ("C1", "C2", "C3", "C4") if u in hw] + c5
 
     def run_unit(self, u, s):
         """Issue unit u's decode call on stream s."""
@@ -321,6 +334,10 @@ class DeviceWorkload:
             L.lt_lz4_int4_decode(self.c4["comp"], int(c4["comp"].size), self.c4["offsets"], c4["block_bytes"],
                                  self.c4["scales"], self.c4["zeros"], c4["rows"], c4["cols"], c4["group_size"],
                                  self.c4_out, self.ws, self.status, s)
+        elif u == "C5index":
+            L.lt_lz4_index_batch(self.c5_all, self.ws, s)
+        elif u[0] == "C5x":
+            L.lt_lz4_int4_expand_batch(self.c5[u[1]], self.ws, self.c5_blocks, self.c5_first[u[1]], self.status, s)
         else:
             L.lt_lz4_int4_decode_batch(self.c5[u[1]], self.ws, self.status, s)
 
@@ -339,7 +356,7 @@ class DeviceWorkload:
         n = 0
         for u in self.units():
             self.run_unit(u, s)
-            mark(u if isinstance(u, str) else "C5")
+            mark(u if u in ("C1", "C2", "C3", "C4") else "C5")
             n += 1
         return n  # kernel launches of this step
 
@@ -350,7 +367,7 @@ class DeviceWorkload:
         (`freed`: one event per unit, recorded after each decode)."""
         torch = self.torch
         s = torch.cuda.current_stream()
-        for i, u in enumerate(self.units()):
+        for i, u in enumerate(self.units(two_step=False)):
             cs.wait_event(freed[i])
             with torch.cuda.stream(cs):
                 for ph, d in self.unit_h2d.get(u, []):
@@ -382,7 +399,9 @@ def launches_per_step(hw) -> int:
         c2 = hw["C2"]
         assert (c2["rows"] * c2["cols"]) % 8 == 0 and c2["cols"] % 8 == 0
         n += 1
-    n += ("C3" in hw) + ("C4" in hw) + len(hw.get("C5", []))
+    # C3: one kernel; C4: parse + expand; C5: one index launch over all
+    # layers, then one expand launch per layer
+    n += ("C3" in hw) + 2 * ("C4" in hw) + ((1 + len(hw["C5"])) if hw.get("C5") else 0)
     return n
 
 
@@ -688,7 +707,7 @@ def run_lt(args, rank, world, local):
     # per codec (device time of the launches, summed over steps): events are
     # recorded at the step start and after every launch, in launch order
     K = args.steps
-    order = [c for c in ("C1", "C2", "C3", "C4") if c in hw] + ["C5"] * len(dw.c5)
+    order = [c for c in ("C1", "C2", "C3", "C4") if c in hw] + ["C5"] * ((1 + len(dw.c5)) if dw.c5 else 0)
     t_c = {c: 0.0 for c in alg}
     per_step = {c: [] for c in alg}  # device ms of the codec's launches in each step
     layer_t = []
@@ -726,9 +745,10 @@ def run_lt(args, rank, world, local):
     # roofline of the dominant kernel: the fused LZ4 decode, one launch per
     # C5 layer (the C4 launch when C5 is not run)
     if layer_t:
-        avg_s = statistics.mean(layer_t) / 1e3
+        avg_s = t_c["C5"] / 1e3 / K / L5  # a layer's expand launch + its share of the all-layer index launch
         launch_bytes = statistics.mean([rd + wr for rd, wr in layer_alg])
-        kname = "k_lz4<fused> (C5 layer, 7 matrices per launch)"
+        kname = ("k_lz4_parse (one launch over all C5 layers) + k_lz4_expand (one launch per layer, 7 matrices): "
+                 "per layer")
     elif "C4" in alg:
         avg_s = t_c["C4"] / 1e3 / K
         launch_bytes = sum(alg["C4"])
@@ -760,7 +780,7 @@ def run_lt(args, rank, world, local):
     cs = torch.cuda.Stream()
     f0.record(s)
     freed = []
-    for _ in dw.units():  # every unit's buffers are free at the start of the timed region
+    for _ in dw.units(two_step=False):  # every unit's buffers are free at the start of the timed region
         e = torch.cuda.Event()
         e.record(s)
         freed.append(e)

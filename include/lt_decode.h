@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define LT_ABI_VERSION 2
+#define LT_ABI_VERSION 3
 
 /* Same type as cudaStream_t. */
 typedef struct CUstream_st *lt_stream_t;
@@ -174,7 +174,7 @@ lt_status lt_lz4_int4_decode(const uint8_t *comp, uint64_t comp_bytes, const uin
  * workspace covers the blocks of all descriptors together.
  * 1 <= n_desc <= LT_LZ4_BATCH_MAX, else LT_ERR_INVALID_ARG / UNSUPPORTED.
  */
-#define LT_LZ4_BATCH_MAX 16
+#define LT_LZ4_BATCH_MAX 64
 typedef struct {
   const uint8_t *comp;
   uint64_t comp_bytes;
@@ -190,6 +190,40 @@ typedef struct {
 
 lt_status lt_lz4_int4_decode_batch(const lt_lz4_int4_desc *descs, int32_t n_desc, void *workspace,
                                    uint64_t workspace_bytes, int32_t *d_status, lt_stream_t stream);
+
+/*
+ * The same decode in two steps, so that the serial part -- the walk over
+ * each block's sequence headers -- can run over many more blocks in one
+ * launch than one decode call covers (e.g. every layer of a model, while
+ * the layers are still decoded one at a time into one reused buffer).
+ *
+ * lt_lz4_index_batch walks every block of descs[0 .. n_desc) and writes its
+ * sequence index (and any stream error it finds) to `index`, a device
+ * buffer of at least lt_lz4_workspace_bytes(total blocks) bytes laid out
+ * like the workspace of the one-step calls. Blocks are numbered across the
+ * descriptors in order: descriptor i's block b is block
+ * (blocks of descriptors 0 .. i-1) + b, where a descriptor has
+ * ceil(ceil(rows*cols/2) / block_bytes) blocks. It writes no output and
+ * reports nothing to a status word.
+ *
+ * lt_lz4_int4_expand_batch decodes descs[0 .. n_desc) -- which must be
+ * consecutive descriptors of an earlier lt_lz4_index_batch call, with the
+ * same compressed streams, starting at its block `first_block` -- from that
+ * index: `index` and `index_bytes` are the buffer given to the index call,
+ * `index_blocks` the total block count of that call. Stream errors found by
+ * the index call, and errors found now, go to *d_status as in
+ * lt_lz4_int4_decode. The index must be complete (the same stream, or an
+ * event) and unchanged since. first_block + the descriptors' blocks >
+ * index_blocks, or an index buffer too small for index_blocks, returns
+ * LT_ERR_INVALID_ARG.
+ * 1 <= n_desc <= LT_LZ4_BATCH_MAX for both, else LT_ERR_INVALID_ARG /
+ * UNSUPPORTED.
+ */
+lt_status lt_lz4_index_batch(const lt_lz4_int4_desc *descs, int32_t n_desc, void *index, uint64_t index_bytes,
+                             lt_stream_t stream);
+lt_status lt_lz4_int4_expand_batch(const lt_lz4_int4_desc *descs, int32_t n_desc, const void *index,
+                                   uint64_t index_bytes, int64_t index_blocks, int64_t first_block,
+                                   int32_t *d_status, lt_stream_t stream);
 
 /*
  * Plain LZ4 block decompression to bytes (the same decoder as the fused

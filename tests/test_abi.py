@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert L.abi_version() == 2
+    assert L.abi_version() == 3
     for code in range(8):
         s = L.status_string(code)
         assert s and s != "unknown status"
@@ -70,9 +70,26 @@ def test_host_argument_errors_return_synchronously(lib):
     assert lib.lt_lz4_int4_decode(P, 16, P, 65536, P, None, 1, 8, 8, P, P + 4, 1 << 20, None, None) == \
         L.LT_ERR_MISALIGNED
     assert lib.lt_lz4_decode(P, 16, P, 8, P, 100, None, 0, None, None) == L.LT_ERR_UNSUPPORTED
-    arr = (L.LtLz4Int4Desc * 17)()
-    assert lib.lt_lz4_int4_decode_batch(arr, 17, None, 0, None, None) == L.LT_ERR_UNSUPPORTED
+    arr = (L.LtLz4Int4Desc * (L.LT_LZ4_BATCH_MAX + 1))()
+    assert lib.lt_lz4_int4_decode_batch(arr, L.LT_LZ4_BATCH_MAX + 1, None, 0, None, None) == L.LT_ERR_UNSUPPORTED
     assert lib.lt_lz4_int4_decode_batch(arr, 0, None, 0, None, None) == L.LT_ERR_INVALID_ARG
+    # the two-step decode: index and expand
+    assert lib.lt_lz4_index_batch(arr, 0, P, 1 << 20, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_lz4_index_batch(arr, L.LT_LZ4_BATCH_MAX + 1, P, 1 << 20, None) == L.LT_ERR_UNSUPPORTED
+    one = (L.LtLz4Int4Desc * 2)()
+    for i in range(2):  # 16 x 8192 codes = 64 KB packed = one 64 KB block each
+        one[i] = L.LtLz4Int4Desc(P, 16, P, P, None, P, 16, 8192, 128, 65536)
+    need = lib.lt_lz4_workspace_bytes(2)
+    assert lib.lt_lz4_index_batch(one, 2, P, need - 1, None) == L.LT_ERR_INVALID_ARG  # index too small
+    assert lib.lt_lz4_index_batch(one, 2, None, need, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_lz4_index_batch(one, 2, P + 8, need, None) == L.LT_ERR_MISALIGNED
+    # expanding descriptor 1 of a 2-block index starts at block 1; block 2 is past its end
+    assert lib.lt_lz4_int4_expand_batch(one, 1, P, need, 2, 2, None, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_lz4_int4_expand_batch(one, 2, P, need, 2, 1, None, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_lz4_int4_expand_batch(one, 1, P, need, 2, -1, None, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_lz4_int4_expand_batch(one, 1, P, need - 1, 2, 1, None, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_lz4_int4_expand_batch(one, 1, None, need, 2, 1, None, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_lz4_int4_expand_batch(one, 1, P, need, 2, 1, P + 2, None) == L.LT_ERR_MISALIGNED
     # workspace sizing: a 16-byte index header plus 512 descriptors per block
     assert lib.lt_lz4_workspace_bytes(0) == 0
     assert lib.lt_lz4_workspace_bytes(448) >= 448 * (16 + 16 * 512)

@@ -416,3 +416,49 @@ def test_lz4_long_match_dependency_chains(n_matches, ws):
     want_f, st_of = oracle_fused(d)
     assert st_f == st_of == 0
     assert_f16_parity(got_f, want_f, what="fused decode of a dependency chain")
+
+
+# --------------------------------------------------------------------------- two-step decode
+
+def test_index_then_expand_in_slices_matches_oracle():
+    # one index call over three matrices, then the matrices decoded in two
+    # slices of that index (as the C5 sweep does with its layers)
+    mats = [make_matrix(64, 8192, 128, 65536, seed=71), make_matrix(48, 4096, 128, 65536, seed=72),
+            make_matrix(32, 8192, 128, 32768, seed=73)]
+    descs, outs = [], []
+    for m in mats:
+        out = f16_out(m["rows"] * m["cols"], 0)
+        outs.append(out)
+        descs.append(dict(comp=dev(m["comp"]), comp_bytes=int(m["comp"].size), block_offsets=dev(m["offsets"]),
+                          scales=dev(m["scales"]), zeros=dev(m["zeros"]), out=out, rows=m["rows"], cols=m["cols"],
+                          group_size=m["group_size"], block_bytes=m["block_bytes"]))
+    blocks = [L.desc_blocks(d) for d in descs]
+    total = sum(blocks)
+    index = torch.empty(L.lt_lz4_workspace_bytes(total), dtype=torch.uint8, device="cuda")
+    L.lt_lz4_index_batch(descs, index)
+    stat = status_buf()
+    L.lt_lz4_int4_expand_batch(descs[:1], index, total, 0, stat)
+    L.lt_lz4_int4_expand_batch(descs[1:2], index, total, blocks[0], stat)
+    # the last slice has only 32 KB blocks, so its window is smaller than the
+    # one the index was built for: its blocks are walked by the expanding CTA
+    L.lt_lz4_int4_expand_batch(descs[2:], index, total, blocks[0] + blocks[1], stat)
+    torch.cuda.synchronize()
+    assert int(stat.item()) == 0
+    for m, out in zip(mats, outs):
+        want, st = oracle_fused(m)
+        assert st == 0
+        assert_f16_parity(host_bits(out), want, what="index + expand")
+    # a stream error the index finds is reported by the expand covering its block
+    bad = dict(mats[2])
+    comp = bad["comp"].copy()
+    comp[int(bad["offsets"][1]):int(bad["offsets"][2])] = 0xFF  # block 1: every token claims a long literal run
+    bad["comp"] = comp
+    descs[2] = dict(descs[2], comp=dev(comp))
+    L.lt_lz4_index_batch(descs, index)
+    stat0, stat1 = status_buf(), status_buf()
+    L.lt_lz4_int4_expand_batch(descs[:2], index, total, 0, stat0)
+    L.lt_lz4_int4_expand_batch(descs[2:], index, total, blocks[0] + blocks[1], stat1)
+    torch.cuda.synchronize()
+    _, st_o = oracle_fused(bad)
+    assert int(stat0.item()) == 0
+    assert int(stat1.item()) == st_o != 0

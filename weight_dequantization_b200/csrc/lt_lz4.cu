@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(kParseWarps * 32) k_lz4_parse(const __grid_con
       r.top_up(0);
       st = parse_block(r, olen, win_cap(batch.max_block_bytes), lmaps[warp], desc + blk * kCap, n, lmax);
     }
-    if (lane == 0) hdr[blk] = make_uint4(n, st, lmax, 0u);
+    if (lane == 0) hdr[blk] = make_uint4(n, st, lmax, win_cap(batch.max_block_bytes));  // the window checked against
   }
 }
 
@@ -773,6 +773,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
       s_n = h.x;
       s_st = h.y;
       s_lmax = h.z;
+      if (h.y == 0 && h.w != wcap) s_st = kNoIndex;  // indexed for another window size: walk the block instead
     }
     __syncthreads();
     const uint32_t n = s_n, lmax = s_lmax;
@@ -881,18 +882,37 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
 
 uint64_t workspace_need(int64_t total_blocks) { return (uint64_t)total_blocks * (16ull + 16ull * kCap) + 256; }
 
+// The sequence index of `total` blocks in a workspace: a header per block,
+// then kCap descriptors per block, from the first 256-byte boundary.
+void index_arrays(const void *ws, int64_t total, uint4 *&hdr, uint4 *&desc) {
+  uintptr_t p = (reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255);
+  hdr = reinterpret_cast<uint4 *>(p);
+  desc = hdr + total;
+}
+
+void launch_parse(const Batch &batch, uint4 *hdr, uint4 *desc, cudaStream_t st) {
+  const int64_t need = (batch.total_blocks + kParseWarps - 1) / kParseWarps;
+  const int64_t cap = (int64_t)num_sms() * blocks_per_sm((const void *)k_lz4_parse, kParseWarps * 32, 0);
+  k_lz4_parse<<<(int)(need < cap ? need : cap), kParseWarps * 32, 0, st>>>(batch, hdr, desc);
+}
+
+lt_status launch_expand(const Batch &batch, bool fused, const uint4 *hdr, const uint4 *desc, int32_t *d_status,
+                        cudaStream_t st);
+
 lt_status launch(const Batch &batch, bool fused, void *workspace, uint64_t workspace_bytes, int32_t *d_status,
                  cudaStream_t st) {
   if (batch.total_blocks == 0) return LT_OK;
   uint4 *hdr = nullptr, *desc = nullptr;
   if (workspace && workspace_bytes >= workspace_need(batch.total_blocks)) {
-    uintptr_t p = (reinterpret_cast<uintptr_t>(workspace) + 255) & ~uintptr_t(255);
-    hdr = reinterpret_cast<uint4 *>(p);
-    desc = hdr + batch.total_blocks;
-    const int64_t need = (batch.total_blocks + kParseWarps - 1) / kParseWarps;
-    const int64_t cap = (int64_t)num_sms() * blocks_per_sm((const void *)k_lz4_parse, kParseWarps * 32, 0);
-    k_lz4_parse<<<(int)(need < cap ? need : cap), kParseWarps * 32, 0, st>>>(batch, hdr, desc);
+    index_arrays(workspace, batch.total_blocks, hdr, desc);
+    launch_parse(batch, hdr, desc, st);
   }
+  return launch_expand(batch, fused, hdr, desc, d_status, st);
+}
+
+lt_status launch_expand(const Batch &batch, bool fused, const uint4 *hdr, const uint4 *desc, int32_t *d_status,
+                        cudaStream_t st) {
+  if (batch.total_blocks == 0) return LT_OK;
   const size_t smem = (size_t)win_cap(batch.max_block_bytes) + 2 * kPad;
   const void *k = fused ? (const void *)k_lz4_expand<true> : (const void *)k_lz4_expand<false>;
   static int attr_set[2][64] = {{0}};
@@ -984,6 +1004,53 @@ LT_API lt_status lt_lz4_int4_decode_batch(const lt_lz4_int4_desc *descs, int32_t
     if (s != LT_OK) return s;
   }
   return launch(batch, true, workspace, workspace_bytes, d_status, (cudaStream_t)stream);
+}
+
+namespace lt {
+namespace {
+lt_status batch_from(const lt_lz4_int4_desc *descs, int32_t n_desc, Batch &batch) {
+  if (n_desc < 1 || !descs) return LT_ERR_INVALID_ARG;
+  if (n_desc > LT_LZ4_BATCH_MAX) return LT_ERR_UNSUPPORTED;
+  for (int32_t i = 0; i < n_desc; ++i) {
+    const lt_lz4_int4_desc &d = descs[i];
+    lt_status s = add_fused_job(batch, d.comp, d.comp_bytes, d.block_offsets, d.block_bytes, d.scales, d.zeros,
+                                d.rows, d.cols, d.group_size, d.out);
+    if (s != LT_OK) return s;
+  }
+  return LT_OK;
+}
+}  // namespace
+}  // namespace lt
+
+LT_API lt_status lt_lz4_index_batch(const lt_lz4_int4_desc *descs, int32_t n_desc, void *index, uint64_t index_bytes,
+                                    lt_stream_t stream) {
+  Batch batch = empty_batch();
+  lt_status s = batch_from(descs, n_desc, batch);
+  if (s != LT_OK) return s;
+  if (batch.total_blocks == 0) return LT_OK;
+  if (!index || index_bytes < workspace_need(batch.total_blocks)) return LT_ERR_INVALID_ARG;
+  if (!aligned(index, 16)) return LT_ERR_MISALIGNED;
+  uint4 *hdr, *desc;
+  index_arrays(index, batch.total_blocks, hdr, desc);
+  launch_parse(batch, hdr, desc, (cudaStream_t)stream);
+  return launch_status();
+}
+
+LT_API lt_status lt_lz4_int4_expand_batch(const lt_lz4_int4_desc *descs, int32_t n_desc, const void *index,
+                                          uint64_t index_bytes, int64_t index_blocks, int64_t first_block,
+                                          int32_t *d_status, lt_stream_t stream) {
+  if (!aligned(d_status, 4)) return LT_ERR_MISALIGNED;
+  Batch batch = empty_batch();
+  lt_status s = batch_from(descs, n_desc, batch);
+  if (s != LT_OK) return s;
+  if (batch.total_blocks == 0) return LT_OK;
+  if (!index || index_blocks < 1 || index_blocks > ((int64_t)1 << 40) || first_block < 0 ||
+      first_block > index_blocks - batch.total_blocks || index_bytes < workspace_need(index_blocks))
+    return LT_ERR_INVALID_ARG;
+  if (!aligned(index, 16)) return LT_ERR_MISALIGNED;
+  uint4 *hdr, *desc;
+  index_arrays(index, index_blocks, hdr, desc);
+  return launch_expand(batch, true, hdr + first_block, desc + first_block * kCap, d_status, (cudaStream_t)stream);
 }
 
 LT_API lt_status lt_lz4_decode(const uint8_t *comp, uint64_t comp_bytes, const uint64_t *block_offsets,

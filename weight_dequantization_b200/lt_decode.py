@@ -27,11 +27,12 @@ LT_ERR_CUDA = 6
 LT_ERR_TIMEOUT = 7
 LT_SCALE_PER_TENSOR = 0
 LT_SCALE_PER_ROW = 1
-LT_LZ4_BATCH_MAX = 16
+LT_LZ4_BATCH_MAX = 64
 
 EXPORTED = (
     "lt_dequant_int4", "lt_dequant_int8", "lt_zrle_decode", "lt_lz4_int4_decode",
-    "lt_lz4_int4_decode_batch", "lt_lz4_decode", "lt_lz4_workspace_bytes", "lt_lz4_int4_decode_noalloc",
+    "lt_lz4_int4_decode_batch", "lt_lz4_index_batch", "lt_lz4_int4_expand_batch", "lt_lz4_decode",
+    "lt_lz4_workspace_bytes", "lt_lz4_int4_decode_noalloc",
     "lt_status_string", "lt_abi_version",
 )
 LT_NOALLOC_MAX_BLOCKS = 512
@@ -70,13 +71,15 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.lt_zrle_decode.argtypes = [P, U64, P, I64, I32, P, P, P]
     lib.lt_lz4_int4_decode.argtypes = [P, U64, P, I32, P, P, I64, I64, I32, P, P, U64, P, P]
     lib.lt_lz4_int4_decode_batch.argtypes = [ctypes.POINTER(LtLz4Int4Desc), I32, P, U64, P, P]
+    lib.lt_lz4_index_batch.argtypes = [ctypes.POINTER(LtLz4Int4Desc), I32, P, U64, P]
+    lib.lt_lz4_int4_expand_batch.argtypes = [ctypes.POINTER(LtLz4Int4Desc), I32, P, U64, I64, I64, P, P]
     lib.lt_lz4_decode.argtypes = [P, U64, P, I32, P, U64, P, U64, P, P]
     lib.lt_lz4_int4_decode_noalloc.argtypes = [P, U64, P, I32, P, P, I64, I64, I32, P, P, P]
     lib.lt_lz4_int4_decode_noalloc.restype = ctypes.c_int
     lib.lt_lz4_workspace_bytes.argtypes = [I64]
     lib.lt_lz4_workspace_bytes.restype = U64
     for f in ("lt_dequant_int4", "lt_dequant_int8", "lt_zrle_decode", "lt_lz4_int4_decode",
-              "lt_lz4_int4_decode_batch", "lt_lz4_decode"):
+              "lt_lz4_int4_decode_batch", "lt_lz4_index_batch", "lt_lz4_int4_expand_batch", "lt_lz4_decode"):
         getattr(lib, f).restype = ctypes.c_int
     lib.lt_status_string.argtypes = [ctypes.c_int]
     lib.lt_status_string.restype = ctypes.c_char_p
@@ -175,6 +178,43 @@ def lt_lz4_int4_decode_batch(descs: Sequence[dict], workspace=None, d_status=Non
     wp, wb = _ws(workspace)
     _check(load_library().lt_lz4_int4_decode_batch(arr, n, wp, wb, _ptr(d_status), _stream(stream, like)),
            "lt_lz4_int4_decode_batch")
+
+
+def _desc_array(descs: Sequence[dict]):
+    arr = (LtLz4Int4Desc * max(len(descs), 1))()
+    for i, d in enumerate(descs):
+        arr[i] = LtLz4Int4Desc(_ptr(d["comp"]), d["comp_bytes"], _ptr(d["block_offsets"]), _ptr(d["scales"]),
+                               _ptr(d.get("zeros")), _ptr(d["out"]), d["rows"], d["cols"], d["group_size"],
+                               d["block_bytes"])
+    return arr
+
+
+def desc_blocks(d: dict) -> int:
+    """LZ4 blocks of one lt_lz4_int4_desc (as a dict): its numbering width in an index."""
+    packed = (d["rows"] * d["cols"] + 1) // 2
+    return (packed + d["block_bytes"] - 1) // d["block_bytes"]
+
+
+def lt_lz4_index_batch(descs: Sequence[dict], index, stream=None) -> None:
+    """Sequence index of every block of ``descs`` into ``index`` (a device
+    tensor of at least lt_lz4_workspace_bytes(total blocks) bytes)."""
+    arr = _desc_array(descs)
+    ip, ib = _ws(index)
+    like = descs[0]["out"] if descs else None
+    _check(load_library().lt_lz4_index_batch(arr, len(descs), ip, ib, _stream(stream, like)), "lt_lz4_index_batch")
+
+
+def lt_lz4_int4_expand_batch(descs: Sequence[dict], index, index_blocks: int, first_block: int, d_status=None,
+                             stream=None) -> None:
+    """Decode ``descs`` from an index built by lt_lz4_index_batch over a
+    descriptor list of ``index_blocks`` blocks in which these start at block
+    ``first_block``."""
+    arr = _desc_array(descs)
+    ip, ib = _ws(index)
+    like = descs[0]["out"] if descs else None
+    _check(load_library().lt_lz4_int4_expand_batch(arr, len(descs), ip, ib, index_blocks, first_block,
+                                                    _ptr(d_status), _stream(stream, like)),
+           "lt_lz4_int4_expand_batch")
 
 
 def lt_lz4_decode(comp, comp_bytes: int, block_offsets, block_bytes: int, out, out_bytes: int, workspace=None,
