@@ -39,10 +39,12 @@ METRIC = "decoded FP16 GB/s per codec; % of B200 HBM roofline (bytes read+writte
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
 
-# dram__bytes_read.sum + dram__bytes_write.sum per launch of the fused LZ4
-# kernel on one C5 layer, from the ncu capture summarised under profiles/;
-# valid only while the kernel sources hash to `sources_sha256`.
-NCU_TRAFFIC = {"sources_sha256": None, "bytes_per_launch": None, "profile": None}
+# dram__bytes_read.sum + dram__bytes_write.sum of one C5 layer's decode (its
+# expand launch + 1/8 of the all-layer index launch), from the ncu capture
+# summarised under profiles/; valid only while the kernel sources hash to
+# `sources_sha256`.
+NCU_TRAFFIC = {"sources_sha256": "63a5cd457f225dd203cbb9031ff944683b2ee41c9b3537e97a5b568a8cd039ea", "bytes_per_launch": 2631657536,
+               "profile": "profiles/k_lz4_c5_layer_traffic.md"}
 
 
 def kernel_sources_sha() -> str:
