@@ -65,7 +65,7 @@ typedef enum {
   LT_ERR_CORRUPT_STREAM = 4, /* (device status) malformed LZ4 / zero-run data */
   LT_ERR_SIZE_MISMATCH = 5,  /* (device status) stream decodes to a different length */
   LT_ERR_CUDA = 6,           /* a CUDA launch failed */
-  LT_ERR_TIMEOUT = 7         /* (device status) an internal on-chip wait ran out; never expected */
+  LT_ERR_TIMEOUT = 7         /* (device status) an internal on-chip wait ran out; reserved: no current kernel waits */
 } lt_status;
 
 typedef enum { LT_SCALE_PER_TENSOR = 0, LT_SCALE_PER_ROW = 1 } lt_scale_mode;
@@ -126,10 +126,11 @@ lt_status lt_zrle_decode(const uint8_t *enc, uint64_t enc_bytes, const uint64_t 
 
 /*
  * Workspace of the LZ4 decoders. The serial part of LZ4 -- walking the
- * sequence headers of a block -- runs as a separate pass, one thread per
- * block, that writes a small sequence index (16 bytes per sequence, at most
- * 512 sequences per block) into a caller-provided device workspace; the
- * expansion then runs with the index in hand. lt_lz4_workspace_bytes(n)
+ * sequence headers of a block -- runs as a separate pass, one warp per
+ * block, that writes a small sequence index (a 16-byte header per block,
+ * then 16 bytes per sequence, at most 512 sequences per block) into a
+ * caller-provided device workspace; the expansion then runs with the index
+ * in hand. lt_lz4_workspace_bytes(n)
  * is the size needed for n blocks in one call (the sum over a batch). A
  * call given NULL or a smaller workspace still decodes correctly, each
  * block walked by the expanding CTA itself (much slower), and so is a block
