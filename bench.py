@@ -43,7 +43,7 @@ NOMINAL_HBM_GBS = 8000.0
 # expand launch + 1/8 of the all-layer index launch), from the ncu capture
 # summarised under profiles/; valid only while the kernel sources hash to
 # `sources_sha256`.
-NCU_TRAFFIC = {"sources_sha256": "63a5cd457f225dd203cbb9031ff944683b2ee41c9b3537e97a5b568a8cd039ea", "bytes_per_launch": 2631657536,
+NCU_TRAFFIC = {"sources_sha256": "274eeac86d1dce72ce68943d10b4df4e3a22917c101e6abf970074008054fc2a", "bytes_per_launch": 2364607616,
                "profile": "profiles/k_lz4_c5_layer_traffic.md"}
 
 

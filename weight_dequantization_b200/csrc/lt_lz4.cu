@@ -83,7 +83,6 @@ __device__ __forceinline__ uint32_t block_len(const Job &jb, int64_t b) {
   return (uint32_t)((jb.packed_bytes - d0) < jb.block_bytes ? (jb.packed_bytes - d0) : jb.block_bytes);
 }
 
-__device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
 // 4 bytes at window byte index s (may be slightly negative or past the end:
 // the window has kPad guard bytes on both sides)
@@ -757,17 +756,6 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
     const Job &jb = find_job(batch, blk, b);
     const int64_t d0 = b * (int64_t)jb.block_bytes;
     const uint32_t olen = block_len(jb, b);
-    {  // bring the next block's compressed bytes into L2 while this one is built
-      const int64_t nblk = blk + gridDim.x;
-      if (nblk < batch.total_blocks) {
-        int64_t nb;
-        const Job &nj = find_job(batch, nblk, nb);
-        const uint64_t a0 = nj.offsets[nb], a1 = nj.offsets[nb + 1];
-        if (a0 <= a1 && a1 <= nj.comp_bytes)
-          for (uint64_t o = a0 + 128 * (uint64_t)threadIdx.x; o < a1; o += 128 * (uint64_t)kThreads)
-            prefetch_l2(nj.comp + o);
-      }
-    }
     if (threadIdx.x == 0) {
       const uint4 h = hdr ? hdr[blk] : make_uint4(0u, kNoIndex, 0u, 0u);
       s_n = h.x;
