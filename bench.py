@@ -43,7 +43,7 @@ NOMINAL_HBM_GBS = 8000.0
 # expand launch + 1/8 of the all-layer index launch), from the ncu capture
 # summarised under profiles/; valid only while the kernel sources hash to
 # `sources_sha256`.
-NCU_TRAFFIC = {"sources_sha256": "274eeac86d1dce72ce68943d10b4df4e3a22917c101e6abf970074008054fc2a", "bytes_per_launch": 2364607616,
+NCU_TRAFFIC = {"sources_sha256": "01fb0eca59039f20b66eee0d5f59d4ff11d4e14c708273a52667e50ffc8d0dca", "bytes_per_launch": 2364607616,
                "profile": "profiles/k_lz4_c5_layer_traffic.md"}
 
 

@@ -20,9 +20,12 @@
 //     all literal runs in parallel rounds, copies the matches one dependency
 //     level at a time, then turns the window into binary16 (8 codes per
 //     4-byte word, 16-byte stores).
-// Blocks with more than kCap sequences, calls without a workspace, and blocks
-// that cannot be staged in place are decoded by warp 0 walking the block
-// itself (slower, same result).
+// The two kernels can also be launched separately: lt_lz4_index_batch runs
+// the parse over many matrices at once, lt_lz4_int4_expand_batch expands a
+// slice of its index. Blocks with more than kCap sequences, calls without a
+// workspace, blocks that cannot be staged in place, and blocks indexed for a
+// different window size are decoded by warp 0 walking the block itself
+// (slower, same result).
 
 #include <mutex>
 
