@@ -53,7 +53,8 @@ def _load():
         lib.oracle_lz4_block_decode.argtypes = [P, U64, P, U64]
         lib.oracle_lz4_decode_blocks.argtypes = [P, U64, P, I64, P, U64]
         lib.oracle_lz4_int4_decode.argtypes = [P, U64, P, I64, P, P, I64, I64, I64, P]
-        for f in ("oracle_dequant_int4", "oracle_dequant_int8", "oracle_zrle_decode",
+        lib.oracle_value_dict_decode.argtypes = [P, I32, P, I64, P]
+        for f in ("oracle_dequant_int4", "oracle_dequant_int8", "oracle_zrle_decode", "oracle_value_dict_decode",
                   "oracle_lz4_block_decode", "oracle_lz4_decode_blocks", "oracle_lz4_int4_decode"):
             getattr(lib, f).restype = I32
         _lib = lib
@@ -133,4 +134,19 @@ def lz4_int4_decode(comp, offsets, block_bytes: int, scales, zeros, rows: int, c
     out = np.zeros(rows * cols, dtype=np.uint16)
     st = _load().oracle_lz4_int4_decode(_p(comp), comp.size, _p(offsets), block_bytes, _p(scales), _p(zeros),
                                         rows, cols, group_size, _p(out))
+    return out, st
+
+
+def value_dict_decode(packed, bits: int, dictionary, n: int):
+    """Returns (fp16 bits as uint16 [n], status): out[k] = dictionary[index k],
+    index k the ``bits``-wide field at bit k * bits, least-significant first."""
+    packed = _c(packed, np.uint8)
+    dictionary = _c(dictionary, np.uint16)
+    if bits in (1, 2, 4, 8):
+        if dictionary.size != 1 << bits:
+            raise ValueError("the dictionary holds 2**bits entries")
+        if n > 0 and packed.size * 8 < n * bits:
+            raise ValueError("packed holds fewer than n indices")
+    out = np.zeros(max(n, 0), dtype=np.uint16)
+    st = _load().oracle_value_dict_decode(_p(packed), bits, _p(dictionary), n, _p(out))
     return out, st

@@ -19,7 +19,12 @@
  *        65536).
  *   [L]  "LoreToken-powered GPU memory layer" (freemwiki ChatGPT export):
  *        compression strategies, "Zero-run encoding - extremely effective on
- *        ReLU activations that are mostly zero".
+ *        ReLU activations that are mostly zero"; "Value dictionary
+ *        compression" for tensors that hold few distinct values (a
+ *        dictionary plus small indices).
+ *   [S]  "GPU sidecar brain" explanation (freemwiki ChatGPT export), its
+ *        list of strategies: value dictionaries store small integer codes
+ *        plus a tiny lookup table.
  *   LZ4 block format: the public description of the LZ4 block layout
  *        (token, literal run, 2-byte little-endian offset, match length
  *        with minimum 4, 255-continuation length bytes, literal-only last
@@ -32,7 +37,9 @@
  * groups run along the contiguous row of a row-major [rows, cols] tensor;
  * per-channel means per row; the zero-run chunk format is the
  * (u16 zero run, u16 literal count, fp16 literals)* record list with
- * little-endian fields.
+ * little-endian fields; a value dictionary is one table of 2^bits fp16
+ * entries per tensor, indexed by bits-wide fields packed least-significant
+ * bits first (the INT4 nibble order).
  *
  * Status values returned: 0 ok, 4 corrupt stream, 5 decoded size differs
  * from the declared size, 1 invalid argument.
@@ -161,6 +168,30 @@ ORACLE_EXPORT int oracle_dequant_int8(const int8_t *q, const uint16_t *scales, c
       out[k] = oracle_f16_from_f64((double)((int)q[k] - z) * s);
     }
   }
+  return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Value-dictionary decoding   [L] compression strategies, [S]         */
+/* ------------------------------------------------------------------ */
+
+/* Index k: the bits-wide field that starts at bit k * bits of the packed
+ * byte stream, bit 0 being the least significant bit of byte 0 (for
+ * bits == 4 this is the INT4 order above: even k in the low nibble). A
+ * field never straddles two bytes because bits divides 8. */
+static unsigned dict_index(const uint8_t *packed, int64_t k, int bits) {
+  uint64_t bit = (uint64_t)k * (uint64_t)bits;
+  unsigned byte = packed[bit / 8];
+  return (byte >> (bit % 8)) & ((1u << bits) - 1u);
+}
+
+/* out[k] = dict[index k] for k in [0, n): the entry's fp16 bit pattern is
+ * copied as it is (no arithmetic, so NaN payloads and -0 survive). dict
+ * holds 2^bits entries; bits is 1, 2, 4 or 8. */
+ORACLE_EXPORT int oracle_value_dict_decode(const uint8_t *packed, int bits, const uint16_t *dict, int64_t n,
+                                           uint16_t *out) {
+  if (n < 0 || !(bits == 1 || bits == 2 || bits == 4 || bits == 8)) return ORACLE_INVALID;
+  for (int64_t k = 0; k < n; ++k) out[k] = dict[dict_index(packed, k, bits)];
   return ORACLE_OK;
 }
 

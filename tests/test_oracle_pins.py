@@ -2,7 +2,7 @@
 
 Nothing here is checked against the oracle itself: expected values come from
 the pages' worked examples (tests/golden), from numpy's own binary16
-conversion, from an exact-rational brute-force search of the binary16 grid,
+conversion and bit unpacking, from an exact-rational brute-force search of the binary16 grid,
 from closed forms and invariants, and from the system LZ4 library.
 """
 from __future__ import annotations
@@ -222,6 +222,80 @@ def test_int8_symmetric_quantizer_round_trip_within_half_step():
     xhat = out.view(np.float16).astype(np.float64)
     bound = scale / 2 + np.abs(q) * abs(float(s16) - scale) + np.abs(xhat) * 2.0 ** -11
     assert np.all(np.abs(xhat - x) <= bound * (1 + 1e-12))
+
+
+# ---------------------------------------------------------------------------
+# value-dictionary decoding (LoreToken page and sidecar page, strategy lists)
+# ---------------------------------------------------------------------------
+
+def _unpack_indices(packed: np.ndarray, bits: int, n: int) -> np.ndarray:
+    # numpy's little-endian bit unpacking: bit j of byte b is stream bit 8b + j
+    stream = np.unpackbits(np.asarray(packed, np.uint8), bitorder="little")[: n * bits]
+    fields = stream.reshape(n, bits).astype(np.int64)
+    return (fields << np.arange(bits)).sum(axis=1)
+
+
+def test_value_dict_int4_worked_example_order(golden_dir):
+    # the INT4 worked example's bytes hold codes 0..7, low nibble first; a
+    # dictionary whose entry i is the page's expected value for code i must
+    # reproduce the page's output (entries 8..15 are never used)
+    g = json.load(open(os.path.join(golden_dir, "int4_worked_example.json")))
+    d = np.array(g["expected_f16_bits"] + [0x7E00] * 8, np.uint16)
+    out, st = oracle.value_dict_decode(np.array(g["packed"], np.uint8), 4, d, 8)
+    assert st == 0
+    assert list(out) == g["expected_f16_bits"]
+
+
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
+def test_value_dict_every_byte_value(bits):
+    packed = np.arange(256, dtype=np.uint8)
+    n = 256 * 8 // bits
+    d = RNG.permutation(np.arange(1 << 16, dtype=np.uint32))[: 1 << bits].astype(np.uint16)
+    out, st = oracle.value_dict_decode(packed, bits, d, n)
+    assert st == 0
+    assert np.array_equal(out, d[_unpack_indices(packed, bits, n)])
+
+
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
+def test_value_dict_ragged_tail_ignores_unused_bits(bits):
+    per_byte = 8 // bits
+    for n in range(0, 3 * per_byte + 1):
+        packed = RNG.integers(0, 256, 3, dtype=np.uint8)
+        packed[-1] = 0xFF  # unused high fields of the last byte point at the last entry
+        d = np.arange(1 << bits, dtype=np.uint16) + 0x1000
+        out, st = oracle.value_dict_decode(packed, bits, d, n)
+        assert st == 0 and out.size == n
+        assert np.array_equal(out, d[_unpack_indices(packed, bits, n)])
+
+
+def test_value_dict_copies_bit_patterns():
+    specials = [0x8000, 0x0000, 0x7C00, 0xFC00, 0x7E01, 0xFD55, 0x0001, 0x83FF,
+                0x7BFF, 0xFBFF, 0x3C00, 0xBC00, 0x7FFF, 0x0400, 0x8400, 0x3555]
+    d = np.array(specials, np.uint16)
+    codes = np.arange(32) % 16
+    packed = (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)
+    out, st = oracle.value_dict_decode(packed, 4, d, 32)
+    assert st == 0 and list(out) == specials * 2
+
+
+def test_value_dict_affine_dictionary_equals_int4_dequant():
+    # with dictionary entry q = fp16_rn((q - z) * s) (numpy's rounding of the
+    # exact product), decoding 4-bit indices is INT4 dequant with one group
+    for s_bits, z in ((0x3800, 0), (0x2E66, 7), (0xB1EC, 15), (0x0003, 3)):
+        s = float(np.array([s_bits], np.uint16).view(np.float16)[0])
+        d = _np_f16_bits((np.arange(16, dtype=np.float64) - z) * s)
+        packed = RNG.integers(0, 256, 512, dtype=np.uint8)
+        got, st = oracle.value_dict_decode(packed, 4, d, 1024)
+        ref, st2 = oracle.dequant_int4(packed, np.array([s_bits], np.uint16), np.array([z], np.uint8),
+                                       1, 1024, 1024)
+        assert st == 0 and st2 == 0
+        assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("bits", [0, 3, 5, 16, -1])
+def test_value_dict_rejects_other_widths(bits):
+    _, st = oracle.value_dict_decode(np.zeros(4, np.uint8), bits, np.zeros(2, np.uint16), 4)
+    assert st == oracle.INVALID
 
 
 # ---------------------------------------------------------------------------
