@@ -64,8 +64,9 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=8, help="C5 layers (8 is the workload)")
-    ap.add_argument("--only", default="C1,C2,C3,C4,C5",
-                    help="comma-separated subset of the workloads to run (profiling); the bench line uses all")
+    ap.add_argument("--only", default="C1,C2,C3,C4,C5,V",
+                    help="comma-separated subset of the workloads to run (profiling); the bench line uses all. "
+                         "C1-C5 form the timed step; V (value-dictionary decode) is timed on its own afterwards")
     return ap.parse_args()
 
 
@@ -662,6 +663,47 @@ def c1_graph_steady_state(hw, peak: float, n_sets: int = 64, chains: int = 8, re
             "hbm_frac_of_measured": (rd + 2 * n) / per / 1e9 / peak, "outputs_identical": bool(same)}
 
 
+def value_dict_timing(peak: float, reps: int = 30, warmup: int = 3):
+    """The value-dictionary decode on its workload (4096 x 14336 4-bit
+    indices with C4's code law, one 16-entry fp16 dictionary), timed per
+    call with CUDA events on the launching stream; before every call a
+    256 MB scratch write (not timed) flushes L2."""
+    import numpy as np
+    import torch
+
+    from weight_dequantization_b200 import lt_decode as L
+    from weight_dequantization_b200.synth import workloads as W
+
+    d = W.v_value_dict()
+    n, bits = d["n"], d["bits"]
+    packed = torch.from_numpy(d["packed"]).cuda()
+    dictionary = torch.from_numpy(d["dictionary"].view(np.int16)).cuda()
+    out = torch.empty(n, dtype=torch.float16, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.current_stream()
+    times = []
+    for r in range(warmup + reps):
+        flush.fill_(r & 0xFF)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        L.lt_value_dict_decode(packed, bits, dictionary, n, out, s)
+        e1.record(s)
+        torch.cuda.synchronize()
+        if r >= warmup:
+            times.append(e0.elapsed_time(e1) / 1e3)
+    rd = int(d["packed"].nbytes + d["dictionary"].nbytes)
+    wr = 2 * n
+    med = statistics.median(times)
+    del flush
+    return {"label": f"value-dictionary decode: {d['rows']}x{d['cols']} {bits}-bit indices (C4's code law), "
+                     f"one {1 << bits}-entry fp16 dictionary; L2 flushed before each of {reps} calls",
+            "kernel": f"k_dict_vec<{bits}>", "us_per_call_median": med * 1e6, "us_per_call_min": min(times) * 1e6,
+            "decoded_GBps": wr / med / 1e9, "bytes_read": rd, "bytes_written": wr,
+            "hbm_frac_of_measured": (rd + wr) / med / 1e9 / peak,
+            "hbm_frac_of_8TBps": (rd + wr) / med / 1e9 / NOMINAL_HBM_GBS}
+
+
 def run_lt(args, rank, world, local):
     import torch
 
@@ -805,6 +847,7 @@ def run_lt(args, rank, world, local):
             cpu = cpu_baseline(hw)
             cpu_thr = cpu_baseline_threads(hw, cpu["frac"])
         c1g = c1_graph_steady_state(hw, peak) if "C1" in hw else None
+        vd = value_dict_timing(peak) if "V" in only else None
         result = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": elapsed / K * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -812,7 +855,8 @@ def run_lt(args, rank, world, local):
             "config": workload_config(hw, args.layers, only), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": nlaunch * K, "clocks": {"sm_mhz": ck["sm_mhz"], "sm_max_mhz": ck["sm_max_mhz"],
                                                      "reasons": ck["reasons"], "samples": ck["samples"]},
-            "per_codec": per_codec, "c1_graph": c1g, "cpu_baseline_threads": cpu_thr, "impl": "lt",
+            "per_codec": per_codec, "c1_graph": c1g, "value_dict": vd, "cpu_baseline_threads": cpu_thr,
+            "impl": "lt",
         }
     if dist is not None:
         dist.barrier()

@@ -12,6 +12,11 @@
  *   fused LZ4 -> INT4 -> fp16   "GPU Compression Pipeline - TDD Roadmap",
  *                               Phase 2.1 LZ4 + INT4 Fused Kernel, with the
  *                               64 KB blocks of Phase 3.1 / Phase 6.1
+ *   value-dictionary decoding   "LoreToken-powered GPU memory layer",
+ *                               compression strategies (value dictionary
+ *                               compression), and the "GPU sidecar brain"
+ *                               explanation's strategy list (small integer
+ *                               codes plus a tiny lookup table)
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -49,7 +54,7 @@
 extern "C" {
 #endif
 
-#define LT_ABI_VERSION 3
+#define LT_ABI_VERSION 4
 
 /* Same type as cudaStream_t. */
 typedef struct CUstream_st *lt_stream_t;
@@ -123,6 +128,26 @@ lt_status lt_dequant_int8(const int8_t *q, const lt_half *scales, const int8_t *
  */
 lt_status lt_zrle_decode(const uint8_t *enc, uint64_t enc_bytes, const uint64_t *chunk_offsets, int64_t n_elements,
                          int32_t chunk_elems, lt_half *out, int32_t *d_status, lt_stream_t stream);
+
+/*
+ * Value-dictionary decoding ("LoreToken-powered GPU memory layer",
+ * compression strategies: a tensor that holds few distinct values stored as
+ * a dictionary plus small indices).
+ *
+ *   packed  ceil(n*bits/8) bytes of indices: index k is the bits-wide field
+ *           that starts at bit k*bits of the byte stream, bit 0 being the
+ *           least significant bit of byte 0 (for bits == 4, the nibble
+ *           order of lt_dequant_int4: even k in the low nibble). Unused high
+ *           bits of the last byte are ignored.
+ *   bits    1, 2, 4 or 8, else LT_ERR_INVALID_ARG.
+ *   dict    2^bits binary16 entries (one dictionary for the tensor).
+ *   out     n binary16 values, out[k] = dict[index k], copied bit for bit
+ *           (no arithmetic: -0 and NaN payloads are kept).
+ *   A 4-byte-aligned `packed` with a 16-byte-aligned `out` (8-byte for
+ *   bits == 8) takes the vectorized kernel.
+ */
+lt_status lt_value_dict_decode(const uint8_t *packed, int32_t bits, const lt_half *dict, int64_t n, lt_half *out,
+                               lt_stream_t stream);
 
 /*
  * Workspace of the LZ4 decoders. The serial part of LZ4 -- walking the

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert L.abi_version() == 3
+    assert L.abi_version() == 4
     for code in range(8):
         s = L.status_string(code)
         assert s and s != "unknown status"
@@ -59,6 +59,15 @@ def test_host_argument_errors_return_synchronously(lib):
     assert lib.lt_dequant_int4(P, P, None, 0, 8, 8, P, None) == L.LT_OK  # empty: nothing enqueued
     assert lib.lt_dequant_int8(P, P, None, 2, 4, 4, P, None) == L.LT_ERR_INVALID_ARG  # bad scale mode
     assert lib.lt_dequant_int8(P, P, None, 1, 4, 4, P + 1, None) == L.LT_ERR_MISALIGNED
+    for bits in (0, 3, 5, 16, -4):
+        assert lib.lt_value_dict_decode(P, bits, P, 64, P, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_value_dict_decode(P, 4, P, -1, P, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_value_dict_decode(P, 4, None, 64, P, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_value_dict_decode(None, 4, P, 64, P, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_value_dict_decode(P, 4, P + 1, 64, P, None) == L.LT_ERR_MISALIGNED
+    assert lib.lt_value_dict_decode(P, 4, P, 64, P + 1, None) == L.LT_ERR_MISALIGNED
+    assert lib.lt_value_dict_decode(P, 4, P, (1 << 62), P, None) == L.LT_ERR_INVALID_ARG  # n * bits overflows
+    assert lib.lt_value_dict_decode(None, 4, None, 0, None, None) == L.LT_OK  # empty: nothing enqueued
     assert lib.lt_zrle_decode(P, 16, P, 100, 0, P, None, None) == L.LT_ERR_UNSUPPORTED
     assert lib.lt_zrle_decode(P, 16, P, 100, 65536, P, None, None) == L.LT_ERR_UNSUPPORTED
     assert lib.lt_zrle_decode(P, 16, P + 4, 100, 4096, P, None, None) == L.LT_ERR_MISALIGNED

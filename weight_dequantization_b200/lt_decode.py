@@ -30,7 +30,7 @@ LT_SCALE_PER_ROW = 1
 LT_LZ4_BATCH_MAX = 64
 
 EXPORTED = (
-    "lt_dequant_int4", "lt_dequant_int8", "lt_zrle_decode", "lt_lz4_int4_decode",
+    "lt_dequant_int4", "lt_dequant_int8", "lt_value_dict_decode", "lt_zrle_decode", "lt_lz4_int4_decode",
     "lt_lz4_int4_decode_batch", "lt_lz4_index_batch", "lt_lz4_int4_expand_batch", "lt_lz4_decode",
     "lt_lz4_workspace_bytes", "lt_lz4_int4_decode_noalloc",
     "lt_status_string", "lt_abi_version",
@@ -68,6 +68,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     P, U64, I64, I32 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int64, ctypes.c_int32
     lib.lt_dequant_int4.argtypes = [P, P, P, I64, I64, I32, P, P]
     lib.lt_dequant_int8.argtypes = [P, P, P, I32, I64, I64, P, P]
+    lib.lt_value_dict_decode.argtypes = [P, I32, P, I64, P, P]
     lib.lt_zrle_decode.argtypes = [P, U64, P, I64, I32, P, P, P]
     lib.lt_lz4_int4_decode.argtypes = [P, U64, P, I32, P, P, I64, I64, I32, P, P, U64, P, P]
     lib.lt_lz4_int4_decode_batch.argtypes = [ctypes.POINTER(LtLz4Int4Desc), I32, P, U64, P, P]
@@ -78,7 +79,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.lt_lz4_int4_decode_noalloc.restype = ctypes.c_int
     lib.lt_lz4_workspace_bytes.argtypes = [I64]
     lib.lt_lz4_workspace_bytes.restype = U64
-    for f in ("lt_dequant_int4", "lt_dequant_int8", "lt_zrle_decode", "lt_lz4_int4_decode",
+    for f in ("lt_dequant_int4", "lt_dequant_int8", "lt_value_dict_decode", "lt_zrle_decode", "lt_lz4_int4_decode",
               "lt_lz4_int4_decode_batch", "lt_lz4_index_batch", "lt_lz4_int4_expand_batch", "lt_lz4_decode"):
         getattr(lib, f).restype = ctypes.c_int
     lib.lt_status_string.argtypes = [ctypes.c_int]
@@ -136,6 +137,11 @@ def lt_dequant_int4(packed, scales, zeros, rows: int, cols: int, group_size: int
 def lt_dequant_int8(q, scales, zeros, scale_mode: int, rows: int, cols: int, out, stream=None) -> None:
     _check(load_library().lt_dequant_int8(_ptr(q), _ptr(scales), _ptr(zeros), scale_mode, rows, cols, _ptr(out),
                                           _stream(stream, out)), "lt_dequant_int8")
+
+
+def lt_value_dict_decode(packed, bits: int, dictionary, n: int, out, stream=None) -> None:
+    _check(load_library().lt_value_dict_decode(_ptr(packed), bits, _ptr(dictionary), n, _ptr(out),
+                                               _stream(stream, out)), "lt_value_dict_decode")
 
 
 def lt_zrle_decode(enc, enc_bytes: int, chunk_offsets, n_elements: int, chunk_elems: int, out, d_status=None,

@@ -19,6 +19,11 @@ laws and the layout stay the same; only the element count changes).
   C5  Llama-2-70B-shaped sweep: 8 layers x {q, o: 8192 x 8192; k, v:
       8192 x 1024; gate, up: 8192 x 28672; down: 28672 x 8192}, C4's law and
       layout; one stream id per (layer, matrix).                   seed 5
+  V   Value-dictionary decode: [4096, 14336] (C4's shape), 4-bit indices
+      with C4's code law (clip(round(N(8, 2)), 0, 15), 30 % of the
+      128-index runs constant), one dictionary of 16 fp16 entries
+      fp16_rn(U[-0.1, 0.1]). Other widths (1, 2, 8 bits) take uniform
+      random index bytes.                                          seed 6
 """
 from __future__ import annotations
 
@@ -116,3 +121,17 @@ def c5_layers(layers: int = LLAMA70B_LAYERS, scale: float = 1.0, seed: int = 5, 
             mats.append(d)
         out.append(mats)
     return out
+
+
+def v_value_dict(scale: float = 1.0, seed: int = 6, bits: int = 4):
+    if bits not in (1, 2, 4, 8):
+        raise ValueError("bits is 1, 2, 4 or 8")
+    rows = max(1, int(round(4096 * scale)))
+    cols = 14336
+    n = rows * cols
+    if bits == 4:
+        packed = int4_gauss_groups_packed(seed, n, group=128, p_const=0.3, mu=8.0, sigma=2.0, stream=0)
+    else:
+        packed = u8_uniform(seed, (n * bits + 7) // 8, 0, 255, stream=0)
+    return dict(kind="value_dict", rows=rows, cols=cols, n=n, bits=bits, packed=packed,
+                dictionary=fp16_uniform(seed, 1 << bits, -0.1, 0.1, stream=1))
