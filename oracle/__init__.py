@@ -54,6 +54,12 @@ def _load():
         lib.oracle_lz4_decode_blocks.argtypes = [P, U64, P, I64, P, U64]
         lib.oracle_lz4_int4_decode.argtypes = [P, U64, P, I64, P, P, I64, I64, I64, P]
         lib.oracle_value_dict_decode.argtypes = [P, I32, P, I64, P]
+        lib.oracle_xxh3_64_secret.argtypes = [P, U64, P, U64]
+        lib.oracle_xxh3_64_secret.restype = U64
+        lib.oracle_hct2_validate.argtypes = [P, U64, P]
+        lib.oracle_hct2_validate.restype = I32
+        lib.oracle_hct2_meta.argtypes = [P, U64, P, P]
+        lib.oracle_hct2_meta.restype = I32
         for f in ("oracle_dequant_int4", "oracle_dequant_int8", "oracle_zrle_decode", "oracle_value_dict_decode",
                   "oracle_lz4_block_decode", "oracle_lz4_decode_blocks", "oracle_lz4_int4_decode"):
             getattr(lib, f).restype = I32
@@ -150,3 +156,46 @@ def value_dict_decode(packed, bits: int, dictionary, n: int):
     out = np.zeros(max(n, 0), dtype=np.uint16)
     st = _load().oracle_value_dict_decode(_p(packed), bits, _p(dictionary), n, _p(out))
     return out, st
+
+
+XXH3_SECRET_MIN = 136
+
+
+def xxh3_64(data, secret) -> int:
+    """XXH3 64-bit hash of ``data`` with ``secret`` (>= 136 bytes), seed 0."""
+    d = _c(np.frombuffer(bytes(data), np.uint8) if not isinstance(data, np.ndarray) else data, np.uint8)
+    sec = _c(np.frombuffer(bytes(secret), np.uint8) if not isinstance(secret, np.ndarray) else secret, np.uint8)
+    if sec.size < XXH3_SECRET_MIN:
+        raise ValueError("the XXH3 secret holds at least 136 bytes")
+    buf = d if d.size else np.zeros(1, np.uint8)
+    return int(_load().oracle_xxh3_64_secret(_p(buf), d.size, _p(sec), sec.size))
+
+
+HCT_OK, HCT_BAD_HEADER, HCT_TRUNCATED, HCT_META_MISMATCH, HCT_BLOCK_MISMATCH = 0, 1, 2, 3, 4
+HCT_META_FIELDS = ("version", "compression", "quantization", "checksum", "block_size", "rows", "cols",
+                   "group_size", "secret_len", "n_blocks", "payload_bytes", "n_groups")
+HCT_SECTIONS = ("offsets", "hashes", "scales", "zeros", "payload", "end")
+
+
+def _buf(container) -> np.ndarray:
+    b = container if isinstance(container, np.ndarray) else np.frombuffer(bytes(container), np.uint8)
+    b = _c(b, np.uint8)
+    return b if b.size else np.zeros(1, np.uint8)
+
+
+def hct2_validate(container):
+    """(status, first mismatching block or None) of an HCT v2 container."""
+    b = _buf(container)
+    n = len(container)
+    bad = np.zeros(1, np.uint64)
+    st = _load().oracle_hct2_validate(_p(b), n, _p(bad))
+    return st, (int(bad[0]) if st == HCT_BLOCK_MISMATCH else None)
+
+
+def hct2_meta(container):
+    """(status, header fields as a dict, section byte offsets as a dict)."""
+    b = _buf(container)
+    meta = np.zeros(12, np.uint64)
+    sec = np.zeros(6, np.uint64)
+    st = _load().oracle_hct2_meta(_p(b), len(container), _p(meta), _p(sec))
+    return st, dict(zip(HCT_META_FIELDS, map(int, meta))), dict(zip(HCT_SECTIONS, map(int, sec)))

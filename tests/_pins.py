@@ -5,6 +5,9 @@
   encoding with an even last bit, magnitudes at or past 65520 to infinity.
 * ``liblz4``: the system LZ4 library (ctypes), used as an outside decoder and
   encoder of the raw LZ4 block format.
+* ``libxxhash``: the system xxHash library (ctypes), an outside XXH3-64.
+* ``hct2_build``: an HCT v2 container laid out byte by byte with ``struct``,
+  its hashes from the system xxHash library.
 """
 from __future__ import annotations
 
@@ -83,3 +86,50 @@ def lz4_lib_compress(data: bytes) -> bytes:
 
 def hexbytes(s: str) -> bytes:
     return bytes.fromhex(s.replace(" ", ""))
+
+
+@lru_cache(maxsize=1)
+def libxxhash():
+    name = ctypes.util.find_library("xxhash") or "libxxhash.so.0"
+    try:
+        lib = ctypes.CDLL(name)
+    except OSError:
+        return None
+    lib.XXH3_64bits_withSecret.argtypes = [ctypes.c_char_p, ctypes.c_size_t, ctypes.c_char_p, ctypes.c_size_t]
+    lib.XXH3_64bits_withSecret.restype = ctypes.c_uint64
+    return lib
+
+
+def xxh3_lib(data: bytes, secret: bytes) -> int:
+    return int(libxxhash().XXH3_64bits_withSecret(bytes(data), len(data), bytes(secret), len(secret)))
+
+
+def _pad16(b: bytearray) -> None:
+    b.extend(b"\0" * (-len(b) % 16))
+
+
+def hct2_build(blocks, block_size: int, rows: int, cols: int, group_size: int, quantization: int,
+               scales: bytes = b"", zeros: bytes = b"", secret: bytes = b"", compression: int = 1) -> bytes:
+    """An HCT v2 container: 64-byte header, secret, offsets, block hashes,
+    scales, zero points and payload, each section from a 16-byte boundary."""
+    import struct
+
+    payload = b"".join(bytes(x) for x in blocks)
+    offs = [0]
+    for x in blocks:
+        offs.append(offs[-1] + len(x))
+    head = bytearray(struct.pack("<4sHHBBBBIQQIIQQQ", b"HCT2", 2, 0, compression, quantization, 1, 0, block_size,
+                                 rows, cols, group_size, len(secret), len(blocks), len(payload), 0))
+    assert len(head) == 64
+    head += secret
+    _pad16(head)
+    head += struct.pack(f"<{len(offs)}Q", *offs)
+    _pad16(head)
+    head += struct.pack(f"<{len(blocks)}Q", *[xxh3_lib(bytes(x), secret) for x in blocks])
+    _pad16(head)
+    head += scales
+    _pad16(head)
+    head += zeros
+    _pad16(head)
+    head[56:64] = struct.pack("<Q", xxh3_lib(bytes(head), secret))
+    return bytes(head) + payload

@@ -3,7 +3,8 @@
 Nothing here is checked against the oracle itself: expected values come from
 the pages' worked examples (tests/golden), from numpy's own binary16
 conversion and bit unpacking, from an exact-rational brute-force search of the binary16 grid,
-from closed forms and invariants, and from the system LZ4 library.
+from closed forms and invariants, and from the system LZ4 and xxHash
+libraries.
 """
 from __future__ import annotations
 
@@ -15,7 +16,8 @@ import numpy as np
 import pytest
 
 import oracle
-from tests._pins import hexbytes, liblz4, lz4_lib_compress, lz4_lib_decompress, nearest_f16_bits
+from tests._pins import (hct2_build, hexbytes, liblz4, libxxhash, lz4_lib_compress, lz4_lib_decompress,
+                         nearest_f16_bits, xxh3_lib)
 
 RNG = np.random.default_rng(20261202)
 
@@ -498,3 +500,102 @@ def test_lz4_random_sequence_blocks_match_direct_simulation():
             c = comp[int(offs[b]):int(offs[b + 1])].tobytes()
             want = raw[b * 65536:(b + 1) * 65536].tobytes()
             assert lz4_lib_decompress(c, len(want)) == want
+
+
+# ---------------------------------------------------------------------------
+# XXH3-64 and the HCT v2 container (roadmap Phase 6.1)
+# ---------------------------------------------------------------------------
+
+needs_xxhash = pytest.mark.skipif(libxxhash() is None, reason="system libxxhash not present")
+
+
+@needs_xxhash
+@pytest.mark.parametrize("secret_len", [136, 192, 193, 256])
+def test_xxh3_matches_libxxhash_in_every_length_class(secret_len):
+    # 0, 1-3, 4-8, 9-16, 17-128, 129-240 and the striped path, across the
+    # boundaries of the secret's scramble blocks ((secret_len - 64) / 8
+    # stripes of 64 bytes)
+    secret = RNG.integers(0, 256, secret_len, dtype=np.uint8).tobytes()
+    block = 64 * ((secret_len - 64) // 8)
+    lengths = list(range(0, 260)) + [block - 1, block, block + 1, 2 * block, 2 * block + 63, 2 * block + 64,
+                                     4096, 47_000, 65_536, 100_003]
+    for n in lengths:
+        data = RNG.integers(0, 256, n, dtype=np.uint8).tobytes()
+        assert oracle.xxh3_64(data, secret) == xxh3_lib(data, secret), n
+
+
+@needs_xxhash
+def test_xxh3_structured_inputs():
+    secret = bytes((7 * i + 3) & 0xFF for i in range(192))
+    for data in (b"", b"\0", b"\0" * 17, b"\xff" * 241, b"\0" * 65536, bytes(range(256)) * 300):
+        assert oracle.xxh3_64(data, secret) == xxh3_lib(data, secret), len(data)
+
+
+def _lz4_int4_container(secret_len=192):
+    # a small LZ4+INT4 matrix: 8 x 8192 codes = 32 KB packed in 4 blocks of 8 KB
+    from weight_dequantization_b200.synth import (fp16_uniform, int4_gauss_groups_packed, lz4_compress_blocks,
+                                                  u8_uniform)
+    rows, cols, G, bs = 8, 8192, 128, 8192
+    packed = int4_gauss_groups_packed(9, rows * cols)
+    comp, offs = lz4_compress_blocks(packed, bs)
+    blocks = [comp[offs[b]:offs[b + 1]].tobytes() for b in range(len(offs) - 1)]
+    n_groups = rows * cols // G
+    scales = fp16_uniform(9, n_groups, 0.001, 0.1, stream=1).tobytes()
+    zeros = u8_uniform(9, n_groups, 0, 15, stream=2).tobytes()
+    secret = RNG.integers(0, 256, secret_len, dtype=np.uint8).tobytes()
+    return hct2_build(blocks, bs, rows, cols, G, 1, scales, zeros, secret), blocks
+
+
+@needs_xxhash
+def test_hct2_checksum_valid():
+    c, _ = _lz4_int4_container()
+    assert oracle.hct2_validate(c) == (oracle.HCT_OK, None)
+
+
+@needs_xxhash
+def test_hct2_checksum_detects_corruption():
+    c, _ = _lz4_int4_container()
+    bad = bytearray(c)
+    bad[100] ^= 0xFF  # the page's flipped byte
+    assert oracle.hct2_validate(bytes(bad))[0] != oracle.HCT_OK
+
+
+@needs_xxhash
+def test_hct2_every_flipped_byte_is_reported():
+    c, blocks = _lz4_int4_container(secret_len=136)
+    _, _, sec = oracle.hct2_meta(c)
+    for i in range(len(c)):
+        bad = bytearray(c)
+        bad[i] ^= 0x5A
+        st, blk = oracle.hct2_validate(bytes(bad))
+        assert st != oracle.HCT_OK, i
+        if i >= sec["payload"]:  # a payload byte: the block holding it, found by its hash
+            rel = i - sec["payload"]
+            ends = np.cumsum([len(b) for b in blocks])
+            assert (st, blk) == (oracle.HCT_BLOCK_MISMATCH, int(np.searchsorted(ends, rel, side="right"))), i
+
+
+@needs_xxhash
+def test_hct2_metadata():
+    c, blocks = _lz4_int4_container()
+    st, meta, sec = oracle.hct2_meta(c)
+    assert st == oracle.HCT_OK
+    assert meta["compression"] == 1 and meta["quantization"] == 1  # LZ4, INT4
+    assert meta["block_size"] == 8192 and meta["rows"] == 8 and meta["cols"] == 8192 and meta["group_size"] == 128
+    assert meta["n_blocks"] == len(blocks) and meta["payload_bytes"] == sum(len(b) for b in blocks)
+    assert meta["n_groups"] == 512 and sec["end"] == len(c)
+    assert all(v % 16 == 0 for k, v in sec.items() if k != "end")
+    # the page's block size through the same header
+    c2 = hct2_build([b"\x10"], 65536, 1, 2, 2, 1, b"\x00\x3c", b"\x00", bytes(136))
+    assert oracle.hct2_meta(c2)[1]["block_size"] == 65536
+
+
+@needs_xxhash
+def test_hct2_header_and_size_errors():
+    c, _ = _lz4_int4_container()
+    assert oracle.hct2_validate(c[:-1])[0] == oracle.HCT_TRUNCATED
+    assert oracle.hct2_validate(c + b"\0")[0] == oracle.HCT_TRUNCATED
+    assert oracle.hct2_validate(b"HCT1" + c[4:])[0] == oracle.HCT_BAD_HEADER
+    assert oracle.hct2_validate(c[:40])[0] == oracle.HCT_BAD_HEADER
+    short_secret = hct2_build([b"ab"], 64, 1, 2, 2, 1, b"\0\0", b"\0", bytes(135))
+    assert oracle.hct2_validate(short_secret)[0] == oracle.HCT_BAD_HEADER
