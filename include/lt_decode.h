@@ -12,6 +12,8 @@
  *   fused LZ4 -> INT4 -> fp16   "GPU Compression Pipeline - TDD Roadmap",
  *                               Phase 2.1 LZ4 + INT4 Fused Kernel, with the
  *                               64 KB blocks of Phase 3.1 / Phase 6.1
+ *   block checksums             "GPU Compression Pipeline - TDD Roadmap",
+ *                               Phase 6.1 HCT Format V2 (XXH3 checksums)
  *   value-dictionary decoding   "LoreToken-powered GPU memory layer",
  *                               compression strategies (value dictionary
  *                               compression), and the "GPU sidecar brain"
@@ -54,7 +56,7 @@
 extern "C" {
 #endif
 
-#define LT_ABI_VERSION 4
+#define LT_ABI_VERSION 5
 
 /* Same type as cudaStream_t. */
 typedef struct CUstream_st *lt_stream_t;
@@ -70,7 +72,8 @@ typedef enum {
   LT_ERR_CORRUPT_STREAM = 4, /* (device status) malformed LZ4 / zero-run data */
   LT_ERR_SIZE_MISMATCH = 5,  /* (device status) stream decodes to a different length */
   LT_ERR_CUDA = 6,           /* a CUDA launch failed */
-  LT_ERR_TIMEOUT = 7         /* (device status) an internal on-chip wait ran out; reserved: no current kernel waits */
+  LT_ERR_TIMEOUT = 7,        /* (device status) an internal on-chip wait ran out; reserved: no current kernel waits */
+  LT_ERR_CHECKSUM = 8        /* (device status) a block's checksum differs from the stored one */
 } lt_status;
 
 typedef enum { LT_SCALE_PER_TENSOR = 0, LT_SCALE_PER_ROW = 1 } lt_scale_mode;
@@ -148,6 +151,29 @@ lt_status lt_zrle_decode(const uint8_t *enc, uint64_t enc_bytes, const uint64_t 
  */
 lt_status lt_value_dict_decode(const uint8_t *packed, int32_t bits, const lt_half *dict, int64_t n, lt_half *out,
                                lt_stream_t stream);
+
+/*
+ * Per-block XXH3-64 checksums ("GPU Compression Pipeline - TDD Roadmap",
+ * Phase 6.1 HCT Format V2: XXH3 checksums; a flipped byte must be reported
+ * as a checksum mismatch).
+ *
+ *   data, data_bytes  the byte stream (e.g. the LZ4 payload of a container).
+ *   offsets           n_blocks + 1 byte offsets into data (uint64, device);
+ *                     block b is data[offsets[b], offsets[b+1]).
+ *   secret            the XXH3 secret (device), secret_len >= 136 bytes; the
+ *                     hash is XXH3-64 (xxHash 0.8) with this secret, seed 0.
+ *   hashes            n_blocks uint64 outputs, or NULL.
+ *   expected          n_blocks uint64 stored checksums, or NULL. A block
+ *                     whose hash differs sets LT_ERR_CHECKSUM in *d_status
+ *                     and lowers *d_first_bad (caller-initialised, e.g. to
+ *                     UINT64_MAX) to its index.
+ *   At least one of hashes / expected, else LT_ERR_INVALID_ARG.
+ *   Device status: LT_ERR_CORRUPT_STREAM for an offset pair out of order or
+ *   past data_bytes (that block is not hashed).
+ */
+lt_status lt_xxh3_blocks(const uint8_t *data, uint64_t data_bytes, const uint64_t *offsets, int64_t n_blocks,
+                         const uint8_t *secret, int32_t secret_len, uint64_t *hashes, const uint64_t *expected,
+                         int32_t *d_status, uint64_t *d_first_bad, lt_stream_t stream);
 
 /*
  * Workspace of the LZ4 decoders. The serial part of LZ4 -- walking the

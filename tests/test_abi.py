@@ -41,8 +41,8 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert L.abi_version() == 4
-    for code in range(8):
+    assert L.abi_version() == 5
+    for code in range(9):
         s = L.status_string(code)
         assert s and s != "unknown status"
     assert L.status_string(99) == "unknown status"
@@ -59,6 +59,13 @@ def test_host_argument_errors_return_synchronously(lib):
     assert lib.lt_dequant_int4(P, P, None, 0, 8, 8, P, None) == L.LT_OK  # empty: nothing enqueued
     assert lib.lt_dequant_int8(P, P, None, 2, 4, 4, P, None) == L.LT_ERR_INVALID_ARG  # bad scale mode
     assert lib.lt_dequant_int8(P, P, None, 1, 4, 4, P + 1, None) == L.LT_ERR_MISALIGNED
+    assert lib.lt_xxh3_blocks(P, 64, P, 1, P, 135, P, None, None, None, None) == L.LT_ERR_INVALID_ARG  # short secret
+    assert lib.lt_xxh3_blocks(P, 64, P, -1, P, 192, P, None, None, None, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_xxh3_blocks(P, 64, P, 1, P, 192, None, None, None, None, None) == L.LT_ERR_INVALID_ARG  # no output
+    assert lib.lt_xxh3_blocks(None, 64, P, 1, P, 192, P, None, None, None, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_xxh3_blocks(P, 64, P + 4, 1, P, 192, P, None, None, None, None) == L.LT_ERR_MISALIGNED
+    assert lib.lt_xxh3_blocks(P, 64, P, 1, P, 192, None, P + 4, None, None, None) == L.LT_ERR_MISALIGNED
+    assert lib.lt_xxh3_blocks(P, 64, P, 0, P, 192, P, None, None, None, None) == L.LT_OK  # empty
     for bits in (0, 3, 5, 16, -4):
         assert lib.lt_value_dict_decode(P, bits, P, 64, P, None) == L.LT_ERR_INVALID_ARG
     assert lib.lt_value_dict_decode(P, 4, P, -1, P, None) == L.LT_ERR_INVALID_ARG

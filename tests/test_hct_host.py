@@ -1,0 +1,42 @@
+"""HCT v2 container header on the host (no GPU): the library's layout and
+parser agree with the oracle's reading of containers built byte by byte."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle
+from tests._pins import hct2_build, libxxhash
+from weight_dequantization_b200 import hct
+
+pytestmark = pytest.mark.skipif(libxxhash() is None, reason="system libxxhash not present")
+RNG = np.random.default_rng(23)
+
+
+def _containers():
+    sec = RNG.integers(0, 256, 192, dtype=np.uint8).tobytes()
+    blocks = [RNG.integers(0, 256, n, dtype=np.uint8).tobytes() for n in (100, 0, 4097, 31)]
+    yield hct2_build(blocks, 8192, 4, 8192, 128, 1, bytes(2 * 256), bytes(256), sec)          # INT4
+    yield hct2_build(blocks[:1], 65536, 3, 10, 0, 2, bytes(2 * 3), b"", sec[:136])            # INT8
+    yield hct2_build([], 65536, 0, 0, 0, 0, b"", b"", sec, compression=0)                     # empty
+
+
+@pytest.mark.parametrize("idx", range(3))
+def test_header_and_sections_match_the_oracle(idx):
+    c = list(_containers())[idx]
+    st, meta, sec = oracle.hct2_meta(c)
+    assert st == oracle.HCT_OK
+    h = hct.read_header(c)
+    for k in ("compression", "quantization", "block_size", "rows", "cols", "group_size", "secret_len", "n_blocks",
+              "payload_bytes", "n_groups", "version", "checksum"):
+        assert getattr(h, k) == meta[k], k
+    assert h.sections() == sec
+    assert h.pack()[:56] == c[:56]
+
+
+def test_parser_rejects_what_the_oracle_rejects():
+    c = next(_containers())
+    for bad in (c[:-1], c + b"\0", b"HCT1" + c[4:], c[:40]):
+        assert oracle.hct2_validate(bad)[0] in (oracle.HCT_TRUNCATED, oracle.HCT_BAD_HEADER)
+        with pytest.raises(hct.HctError):
+            hct.read_header(bad)

@@ -65,6 +65,8 @@ LT_API const char *lt_status_string(lt_status s) {
       return "CUDA launch failed";
     case LT_ERR_TIMEOUT:
       return "an on-chip wait ran out (internal error)";
+    case LT_ERR_CHECKSUM:
+      return "block checksum mismatch";
   }
   return "unknown status";
 }

@@ -25,6 +25,7 @@ LT_ERR_CORRUPT_STREAM = 4
 LT_ERR_SIZE_MISMATCH = 5
 LT_ERR_CUDA = 6
 LT_ERR_TIMEOUT = 7
+LT_ERR_CHECKSUM = 8
 LT_SCALE_PER_TENSOR = 0
 LT_SCALE_PER_ROW = 1
 LT_LZ4_BATCH_MAX = 64
@@ -32,7 +33,7 @@ LT_LZ4_BATCH_MAX = 64
 EXPORTED = (
     "lt_dequant_int4", "lt_dequant_int8", "lt_value_dict_decode", "lt_zrle_decode", "lt_lz4_int4_decode",
     "lt_lz4_int4_decode_batch", "lt_lz4_index_batch", "lt_lz4_int4_expand_batch", "lt_lz4_decode",
-    "lt_lz4_workspace_bytes", "lt_lz4_int4_decode_noalloc",
+    "lt_lz4_workspace_bytes", "lt_lz4_int4_decode_noalloc", "lt_xxh3_blocks",
     "lt_status_string", "lt_abi_version",
 )
 LT_NOALLOC_MAX_BLOCKS = 512
@@ -77,6 +78,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.lt_lz4_decode.argtypes = [P, U64, P, I32, P, U64, P, U64, P, P]
     lib.lt_lz4_int4_decode_noalloc.argtypes = [P, U64, P, I32, P, P, I64, I64, I32, P, P, P]
     lib.lt_lz4_int4_decode_noalloc.restype = ctypes.c_int
+    lib.lt_xxh3_blocks.argtypes = [P, U64, P, I64, P, I32, P, P, P, P, P]
+    lib.lt_xxh3_blocks.restype = ctypes.c_int
     lib.lt_lz4_workspace_bytes.argtypes = [I64]
     lib.lt_lz4_workspace_bytes.restype = U64
     for f in ("lt_dequant_int4", "lt_dequant_int8", "lt_value_dict_decode", "lt_zrle_decode", "lt_lz4_int4_decode",
@@ -148,6 +151,14 @@ def lt_zrle_decode(enc, enc_bytes: int, chunk_offsets, n_elements: int, chunk_el
                    stream=None) -> None:
     _check(load_library().lt_zrle_decode(_ptr(enc), enc_bytes, _ptr(chunk_offsets), n_elements, chunk_elems,
                                          _ptr(out), _ptr(d_status), _stream(stream, out)), "lt_zrle_decode")
+
+
+def lt_xxh3_blocks(data, data_bytes: int, offsets, n_blocks: int, secret, secret_len: int, hashes=None,
+                   expected=None, d_status=None, d_first_bad=None, stream=None) -> None:
+    like = hashes if hashes is not None else expected
+    _check(load_library().lt_xxh3_blocks(_ptr(data), data_bytes, _ptr(offsets), n_blocks, _ptr(secret), secret_len,
+                                         _ptr(hashes), _ptr(expected), _ptr(d_status), _ptr(d_first_bad),
+                                         _stream(stream, like)), "lt_xxh3_blocks")
 
 
 def lt_lz4_workspace_bytes(n_blocks: int) -> int:
