@@ -60,6 +60,8 @@ def _load():
         lib.oracle_hct2_validate.restype = I32
         lib.oracle_hct2_meta.argtypes = [P, U64, P, P]
         lib.oracle_hct2_meta.restype = I32
+        lib.oracle_int4_matmul.argtypes = [P, I64, P, P, P, I64, I64, I64, P, P]
+        lib.oracle_int4_matmul.restype = I32
         for f in ("oracle_dequant_int4", "oracle_dequant_int8", "oracle_zrle_decode", "oracle_value_dict_decode",
                   "oracle_lz4_block_decode", "oracle_lz4_decode_blocks", "oracle_lz4_int4_decode"):
             getattr(lib, f).restype = I32
@@ -199,3 +201,18 @@ def hct2_meta(container):
     sec = np.zeros(6, np.uint64)
     st = _load().oracle_hct2_meta(_p(b), len(container), _p(meta), _p(sec))
     return st, dict(zip(HCT_META_FIELDS, map(int, meta))), dict(zip(HCT_SECTIONS, map(int, sec)))
+
+
+def int4_matmul(x, M: int, packed, scales, zeros, K: int, N: int, group_size: int):
+    """(out, absum, status): out = x @ W in double, W the INT4 dequant of a
+    [K, N] matrix (groups along each row), x binary16 bits [M, K]; absum is
+    the sum of |x[m, k] * W[k, n]|."""
+    x = _c(x, np.uint16)
+    packed = _c(packed, np.uint8)
+    scales = _c(scales, np.uint16)
+    zeros = None if zeros is None else _c(zeros, np.uint8)
+    out = np.zeros((M, N), np.float64)
+    absum = np.zeros((M, N), np.float64)
+    st = _load().oracle_int4_matmul(_p(x), M, _p(packed), _p(scales), _p(zeros), K, N, group_size, _p(out),
+                                    _p(absum))
+    return out, absum, st

@@ -612,3 +612,51 @@ ORACLE_EXPORT int oracle_hct2_meta(const uint8_t *buf, uint64_t len, uint64_t me
   memcpy(sections, s, sizeof s);
   return HCT_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* Decode -> matrix multiply   [R] Phase 4.1, [L] decode + GEMM        */
+/* ------------------------------------------------------------------ */
+/* [R] Phase 4.1 (test_tensor_usable_in_matmul) multiplies an input by a
+ * decoded weight tensor, input.matmul(weights); [L] lists "decode + GEMM"
+ * benchmarks (decompress, then multiply). Two plain steps: W = the INT4
+ * dequant of oracle_dequant_int4 as a [K, N] matrix (rows = K, cols = N,
+ * groups along each row), then out[m, n] = sum over k of x[m, k] * W[k, n]
+ * with x a row-major [M, K] binary16 matrix. Products of two binary16
+ * values are exact in double, and the sum is taken in double in order of
+ * k; absum[m, n] = sum of |x[m, k] * W[k, n]| bounds the rounding error
+ * of any other summation order. */
+ORACLE_EXPORT int oracle_int4_matmul(const uint16_t *x, int64_t M, const uint8_t *packed, const uint16_t *scales,
+                                     const uint8_t *zeros, int64_t K, int64_t N, int64_t group_size, double *out,
+                                     double *absum) {
+  if (M < 0 || K < 0 || N < 0) return ORACLE_INVALID;
+  uint16_t *w = (uint16_t *)malloc((size_t)(K * N > 0 ? K * N : 1) * sizeof(uint16_t));
+  double *wd = (double *)malloc((size_t)(K * N > 0 ? K * N : 1) * sizeof(double));
+  double *xd = (double *)malloc((size_t)(M * K > 0 ? M * K : 1) * sizeof(double));
+  if (!w || !wd || !xd) {
+    free(w);
+    free(wd);
+    free(xd);
+    return ORACLE_INVALID;
+  }
+  int st = oracle_dequant_int4(packed, scales, zeros, K, N, group_size, w);
+  if (st == ORACLE_OK) {
+    for (int64_t i = 0; i < K * N; ++i) wd[i] = oracle_f16_to_f64(w[i]);
+    for (int64_t i = 0; i < M * K; ++i) xd[i] = oracle_f16_to_f64(x[i]);
+    for (int64_t m = 0; m < M; ++m) {
+      for (int64_t n = 0; n < N; ++n) {
+        double s = 0.0, a = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+          double p = xd[m * K + k] * wd[k * N + n];
+          s += p;
+          a += fabs(p);
+        }
+        out[m * N + n] = s;
+        if (absum) absum[m * N + n] = a;
+      }
+    }
+  }
+  free(w);
+  free(wd);
+  free(xd);
+  return st;
+}

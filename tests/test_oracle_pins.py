@@ -599,3 +599,69 @@ def test_hct2_header_and_size_errors():
     assert oracle.hct2_validate(c[:40])[0] == oracle.HCT_BAD_HEADER
     short_secret = hct2_build([b"ab"], 64, 1, 2, 2, 1, b"\0\0", b"\0", bytes(135))
     assert oracle.hct2_validate(short_secret)[0] == oracle.HCT_BAD_HEADER
+
+
+# ---------------------------------------------------------------------------
+# decode -> matrix multiply (roadmap Phase 4.1: input.matmul(weights))
+# ---------------------------------------------------------------------------
+
+def _np_int4_dequant(packed, scales, zeros, K, N, G):
+    # numpy's own path: nibbles low first, (q - z) * s exact in double,
+    # rounded by numpy's binary16 conversion
+    codes = np.stack([packed & 0xF, packed >> 4], axis=1).ravel()[: K * N].astype(np.float64)
+    z = np.repeat(zeros.astype(np.float64), G)
+    s = np.repeat(scales.view(np.float16).astype(np.float64), G)
+    return ((codes - z) * s).astype(np.float16).astype(np.float64).reshape(K, N)
+
+
+def _int4_operands(seed, M, K, N, G):
+    rng = np.random.default_rng(seed)
+    packed = rng.integers(0, 256, K * N // 2, dtype=np.uint8)
+    scales = rng.uniform(0.001, 0.1, K * N // G).astype(np.float16).view(np.uint16)
+    zeros = rng.integers(0, 16, K * N // G, dtype=np.uint8)
+    x = rng.standard_normal((M, K)).astype(np.float16)
+    return x, packed, scales, zeros
+
+
+def test_int4_matmul_identity_input_returns_the_decoded_matrix():
+    K, N, G = 48, 40, 8
+    _, packed, scales, zeros = _int4_operands(1, K, K, N, G)
+    eye = np.eye(K, dtype=np.float16)
+    out, absum, st = oracle.int4_matmul(eye.view(np.uint16), K, packed, scales, zeros, K, N, G)
+    assert st == 0
+    w = _np_int4_dequant(packed, scales, zeros, K, N, G)
+    assert np.array_equal(out, w) and np.array_equal(absum, np.abs(w))
+
+
+def test_int4_matmul_matches_numpy_matmul():
+    M, K, N, G = 24, 256, 96, 32  # M, K, N distinct: a transposed operand cannot pass
+    x, packed, scales, zeros = _int4_operands(2, M, K, N, G)
+    out, absum, st = oracle.int4_matmul(x.view(np.uint16), M, packed, scales, zeros, K, N, G)
+    assert st == 0
+    w = _np_int4_dequant(packed, scales, zeros, K, N, G)
+    xd = x.astype(np.float64)
+    assert np.all(np.abs(out - xd @ w) <= 1e-13 * absum + 1e-300)
+    assert np.allclose(absum, np.abs(xd) @ np.abs(w), rtol=1e-13, atol=0)
+
+
+def test_int4_matmul_small_integers_are_exact():
+    M, K, N, G = 5, 64, 32, 16
+    rng = np.random.default_rng(3)
+    codes = rng.integers(0, 16, K * N)
+    packed = (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)
+    zeros = rng.integers(0, 16, K * N // G, dtype=np.uint8)
+    scales = np.full(K * N // G, 0x3C00, np.uint16)  # 1.0
+    xi = rng.integers(-8, 9, (M, K))
+    out, _, st = oracle.int4_matmul(xi.astype(np.float16).view(np.uint16), M, packed, scales, zeros, K, N, G)
+    assert st == 0
+    wi = codes.reshape(K, N) - np.repeat(zeros.astype(np.int64), G).reshape(K, N)
+    assert np.array_equal(out, (xi @ wi).astype(np.float64))
+
+
+def test_int4_matmul_worked_example_row(golden_dir):
+    # the INT4 worked example as a 1 x 8 weight; an input of [[2.0]] doubles it
+    g = json.load(open(os.path.join(golden_dir, "int4_worked_example.json")))
+    out, _, st = oracle.int4_matmul(np.array([[0x4000]], np.uint16), 1, np.array(g["packed"], np.uint8),
+                                    np.array([g["scale_f16_bits"]], np.uint16), np.array([g["zero_point"]], np.uint8),
+                                    1, 8, 8)
+    assert st == 0 and list(out[0]) == [2 * v for v in g["expected_values"]]
