@@ -185,15 +185,10 @@ def lt_lz4_int4_decode(comp, comp_bytes: int, block_offsets, block_bytes: int, s
 
 def lt_lz4_int4_decode_batch(descs: Sequence[dict], workspace=None, d_status=None, stream=None) -> None:
     """``descs``: dicts with the keys of lt_lz4_int4_desc (tensors or addresses)."""
-    n = len(descs)
-    arr = (LtLz4Int4Desc * max(n, 1))()
-    for i, d in enumerate(descs):
-        arr[i] = LtLz4Int4Desc(_ptr(d["comp"]), d["comp_bytes"], _ptr(d["block_offsets"]), _ptr(d["scales"]),
-                               _ptr(d.get("zeros")), _ptr(d["out"]), d["rows"], d["cols"], d["group_size"],
-                               d["block_bytes"])
-    like = descs[0]["out"] if n else None
+    arr = _desc_array(descs)
+    like = descs[0]["out"] if descs else None
     wp, wb = _ws(workspace)
-    _check(load_library().lt_lz4_int4_decode_batch(arr, n, wp, wb, _ptr(d_status), _stream(stream, like)),
+    _check(load_library().lt_lz4_int4_decode_batch(arr, len(descs), wp, wb, _ptr(d_status), _stream(stream, like)),
            "lt_lz4_int4_decode_batch")
 
 
