@@ -246,8 +246,3 @@ def lt_lz4_int4_decode_noalloc(comp, comp_bytes: int, block_offsets, block_bytes
                                                      _ptr(scales), _ptr(zeros), rows, cols, group_size, _ptr(out),
                                                      _ptr(d_status), _stream(stream, out)),
            "lt_lz4_int4_decode_noalloc")
-
-
-def lz4_blocks(n_bytes: int, block_bytes: int) -> int:
-    """Number of LZ4 blocks of ``block_bytes`` covering ``n_bytes``."""
-    return (int(n_bytes) + block_bytes - 1) // block_bytes
