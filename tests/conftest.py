@@ -12,6 +12,17 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
 
 
+# The checksum tests are collected after every other module, so that under
+# -x a failure in them leaves the decoders' parity tests already run.
+RUN_LAST = ("test_gpu_xxh3.py",)
+
+
+def pytest_collection_modifyitems(config, items):
+    last = [it for it in items if os.path.basename(str(it.fspath)) in RUN_LAST]
+    if last:
+        items[:] = [it for it in items if it not in last] + last
+
+
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")

@@ -4,8 +4,8 @@ lt_lz4_int4_decode_noalloc keeps the sequence index the decode needs in a
 scratch array built into the library instead of a caller-provided workspace,
 so a caller whose device memory is budgeted up front (an engine plugin, a
 component that does not own the allocator) can still use the fast path. This
-file is collected last on purpose: a failure here leaves every other test
-already run.
+file is collected after the decoders' parity tests on purpose: a failure here
+leaves them already run.
 """
 from __future__ import annotations
 
