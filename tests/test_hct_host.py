@@ -40,3 +40,25 @@ def test_parser_rejects_what_the_oracle_rejects():
         assert oracle.hct2_validate(bad)[0] in (oracle.HCT_TRUNCATED, oracle.HCT_BAD_HEADER)
         with pytest.raises(hct.HctError):
             hct.read_header(bad)
+
+
+def test_writer_rejects_bad_arguments_before_any_device_work():
+    with pytest.raises(hct.HctError):
+        hct.write([b"ab"], 65536, 1, 2, hct.QUANT_INT4, 2, np.zeros(1, np.uint16), np.zeros(1, np.uint8),
+                  secret=bytes(135))  # secret too short
+    with pytest.raises(hct.HctError):
+        hct.write([b"ab"], 65536, 1, 4, hct.QUANT_INT4, 2, np.zeros(1, np.uint16), np.zeros(2, np.uint8),
+                  secret=bytes(136))  # 2 groups need 2 scales
+
+
+@pytest.mark.parametrize("field,offset,value", [
+    ("version", 4, b"\x03\x00"), ("compression", 8, b"\x02"), ("quantization", 9, b"\x03"),
+    ("checksum", 10, b"\x00"), ("secret_len", 36, (135).to_bytes(4, "little")),
+    ("block_size", 12, bytes(4)), ("group_size", 32, (3).to_bytes(4, "little")),
+])
+def test_parser_rejects_each_bad_field(field, offset, value):
+    c = bytearray(next(_containers()))
+    c[offset:offset + len(value)] = value
+    with pytest.raises(hct.HctError):
+        hct.read_header(bytes(c))
+    assert oracle.hct2_validate(bytes(c))[0] == oracle.HCT_BAD_HEADER, field
