@@ -176,6 +176,69 @@ lt_status lt_xxh3_blocks(const uint8_t *data, uint64_t data_bytes, const uint64_
                          int32_t *d_status, uint64_t *d_first_bad, lt_stream_t stream);
 
 /*
+ * HCT v2 container header ("GPU Compression Pipeline - TDD Roadmap",
+ * Phase 6.1 HCT Format V2: compression / quantization metadata, block size
+ * and XXH3 checksums; the page leaves the header's design open, so this
+ * layout is this library's). HOST functions: buf / out / h are host memory,
+ * nothing touches a device.
+ *
+ * Bytes 0..63, little-endian: "HCT2", version u16 (= 2), reserved u16,
+ * compression u8 (0 none, 1 raw LZ4 blocks), quantization u8 (0 none = fp16,
+ * 1 INT4, 2 INT8), checksum u8 (1 = XXH3-64), reserved u8, block_size u32,
+ * rows u64, cols u64, group_size u32, secret_len u32, n_blocks u64,
+ * payload_bytes u64, meta_hash u64. Then the XXH3 secret (secret_len >= 136
+ * bytes) and, each from a 16-byte boundary: block offsets u64[n_blocks + 1]
+ * (relative to the payload), block hashes u64[n_blocks] (lt_xxh3_blocks of
+ * the payload), scales fp16[n_groups], zero points u8[n_groups] (INT4 only),
+ * and the payload, which ends the container. n_groups is rows*cols /
+ * group_size for INT4, rows for INT8, 0 otherwise. meta_hash is XXH3-64 of
+ * every byte before the payload with the meta_hash field read as zero.
+ */
+#define LT_HCT2_VERSION 2
+#define LT_HCT2_HEADER_BYTES 64
+#define LT_HCT2_SECRET_MIN 136
+typedef struct {
+  /* the stored fields */
+  uint16_t version;
+  uint8_t compression;
+  uint8_t quantization;
+  uint8_t checksum;
+  uint32_t block_size;
+  uint64_t rows;
+  uint64_t cols;
+  uint32_t group_size;
+  uint32_t secret_len;
+  uint64_t n_blocks;
+  uint64_t payload_bytes;
+  uint64_t meta_hash;
+  /* derived by lt_hct2_layout: group count and byte offsets of the sections */
+  uint64_t n_groups;
+  uint64_t offsets_at;
+  uint64_t hashes_at;
+  uint64_t scales_at;
+  uint64_t zeros_at;
+  uint64_t payload_at;
+  uint64_t total_bytes;
+} lt_hct2_header;
+
+/* Check the stored fields of *h and fill in the derived ones.
+ * LT_ERR_INVALID_ARG for an unknown version, compression, quantization or
+ * checksum kind, a secret shorter than 136 bytes, block_size 0, more than
+ * 2^40 blocks or 2^50 elements, or an INT4 group size that does not divide
+ * cols. */
+lt_status lt_hct2_layout(lt_hct2_header *h);
+
+/* Parse the header of a container of buf_bytes bytes (host memory) into *h
+ * (stored and derived fields). LT_ERR_INVALID_ARG for a bad magic or fields
+ * as in lt_hct2_layout, LT_ERR_SIZE_MISMATCH if the sections do not end at
+ * buf_bytes. No checksum is checked here (lt_xxh3_blocks does that). */
+lt_status lt_hct2_read_header(const uint8_t *buf, uint64_t buf_bytes, lt_hct2_header *h);
+
+/* Write the 64 header bytes of *h's stored fields to out (host memory),
+ * after the checks of lt_hct2_layout. */
+lt_status lt_hct2_write_header(const lt_hct2_header *h, uint8_t *out);
+
+/*
  * Workspace of the LZ4 decoders. The serial part of LZ4 -- walking the
  * sequence headers of a block -- runs as a separate pass, one warp per
  * block, that writes a small sequence index (a 16-byte header per block,

@@ -66,6 +66,10 @@ def test_host_argument_errors_return_synchronously(lib):
     assert lib.lt_xxh3_blocks(P, 64, P + 4, 1, P, 192, P, None, None, None, None) == L.LT_ERR_MISALIGNED
     assert lib.lt_xxh3_blocks(P, 64, P, 1, P, 192, None, P + 4, None, None, None) == L.LT_ERR_MISALIGNED
     assert lib.lt_xxh3_blocks(P, 64, P, 0, P, 192, P, None, None, None, None) == L.LT_OK  # empty
+    assert lib.lt_hct2_layout(None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_hct2_read_header(None, 64, None) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_hct2_read_header(b"HCT2" + bytes(60), 64, ctypes.byref(L.LtHct2Header())) == L.LT_ERR_INVALID_ARG
+    assert lib.lt_hct2_write_header(ctypes.byref(L.LtHct2Header()), None) == L.LT_ERR_INVALID_ARG
     for bits in (0, 3, 5, 16, -4):
         assert lib.lt_value_dict_decode(P, bits, P, 64, P, None) == L.LT_ERR_INVALID_ARG
     assert lib.lt_value_dict_decode(P, 4, P, -1, P, None) == L.LT_ERR_INVALID_ARG

@@ -117,7 +117,7 @@ def test_container_verified_on_the_device():
     blocks, bs, rows, cols, G, scales, zeros, secret = _container_parts()
     c = hct.write(blocks, bs, rows, cols, hct.QUANT_INT4, G, scales, zeros, secret)
     assert hct.verify(c) == (True, None, True)
-    sec = hct.read_header(c).sections()
+    sec = hct.sections(hct.read_header(c))
     ends = np.cumsum([len(b) for b in blocks])
     for rel in (0, int(ends[2]) + 7, int(ends[-1]) - 1):
         bad = bytearray(c)

@@ -1,5 +1,6 @@
-"""HCT v2 container header on the host (no GPU): the library's layout and
-parser agree with the oracle's reading of containers built byte by byte."""
+"""HCT v2 container header on the host (no GPU): the library's native
+header functions (lt_hct2_layout / read_header / write_header, through the
+C ABI) agree with the oracle's reading of containers built byte by byte."""
 from __future__ import annotations
 
 import numpy as np
@@ -8,6 +9,7 @@ import pytest
 import oracle
 from tests._pins import hct2_build, libxxhash
 from weight_dequantization_b200 import hct
+from weight_dequantization_b200 import lt_decode as L
 
 pytestmark = pytest.mark.skipif(libxxhash() is None, reason="system libxxhash not present")
 RNG = np.random.default_rng(23)
@@ -30,8 +32,8 @@ def test_header_and_sections_match_the_oracle(idx):
     for k in ("compression", "quantization", "block_size", "rows", "cols", "group_size", "secret_len", "n_blocks",
               "payload_bytes", "n_groups", "version", "checksum"):
         assert getattr(h, k) == meta[k], k
-    assert h.sections() == sec
-    assert h.pack()[:56] == c[:56]
+    assert hct.sections(h) == sec
+    assert L.lt_hct2_write_header(h) == c[:64]
 
 
 def test_parser_rejects_what_the_oracle_rejects():

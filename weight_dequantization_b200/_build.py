@@ -15,7 +15,9 @@ CSRC = os.path.join(PKG, "csrc")
 DECODE_LIB = os.path.join(PKG, "liblt_decode.so")
 SYNTH_LIB = os.path.join(PKG, "synth", "liblt_synth.so")
 
-CUDA_SOURCES = ["lt_abi.cu", "lt_dequant.cu", "lt_dict.cu", "lt_zrle.cu", "lt_lz4.cu", "lt_xxh3.cu"]
+# CUDA sources, plus the host-only container header code (lt_hct.cpp, built
+# by nvcc's host compiler into the same library)
+CUDA_SOURCES = ["lt_abi.cu", "lt_dequant.cu", "lt_dict.cu", "lt_zrle.cu", "lt_lz4.cu", "lt_xxh3.cu", "lt_hct.cpp"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

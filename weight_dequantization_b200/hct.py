@@ -17,101 +17,56 @@ undesigned, so this layout is this library's):
      only), and the payload (the compressed blocks), which ends the file.
 
 meta_hash is XXH3-64 of every byte before the payload with the meta_hash
-field read as zero; block hash b covers the payload bytes of block b. All
-hashing runs on the device through ``lt_xxh3_blocks``; this module only
-lays out and parses bytes on the host.
+field read as zero; block hash b covers the payload bytes of block b. The
+header is laid out, parsed and written by the library's host functions
+(``lt_hct2_layout``, ``lt_hct2_read_header``, ``lt_hct2_write_header``) and
+all hashing runs on the device through ``lt_xxh3_blocks``; this module only
+moves bytes.
 """
 from __future__ import annotations
 
 import struct
-from dataclasses import dataclass
 
 import numpy as np
 
 from . import lt_decode as L
 
-MAGIC = b"HCT2"
-VERSION = 2
-HEADER_BYTES = 64
-SECRET_MIN = 136
+SECRET_MIN = L.LT_HCT2_SECRET_MIN
+HEADER_BYTES = L.LT_HCT2_HEADER_BYTES
 COMPRESSION_NONE, COMPRESSION_LZ4 = 0, 1
 QUANT_NONE, QUANT_INT4, QUANT_INT8 = 0, 1, 2
 CHECKSUM_XXH3 = 1
-_HEADER = struct.Struct("<4sHHBBBBIQQIIQQQ")
-
-
-def _r16(x: int) -> int:
-    return (x + 15) & ~15
-
-
-@dataclass(frozen=True)
-class Header:
-    compression: int
-    quantization: int
-    block_size: int
-    rows: int
-    cols: int
-    group_size: int
-    secret_len: int
-    n_blocks: int
-    payload_bytes: int
-    meta_hash: int = 0
-    version: int = VERSION
-    checksum: int = CHECKSUM_XXH3
-
-    @property
-    def n_groups(self) -> int:
-        if self.quantization == QUANT_INT4:
-            return self.rows * self.cols // self.group_size
-        if self.quantization == QUANT_INT8:
-            return self.rows
-        return 0
-
-    def sections(self) -> dict:
-        """Byte offsets of the sections (and the end of the container)."""
-        at = _r16(HEADER_BYTES + self.secret_len)
-        out = {"offsets": at}
-        at = _r16(at + 8 * (self.n_blocks + 1))
-        out["hashes"] = at
-        at = _r16(at + 8 * self.n_blocks)
-        out["scales"] = at
-        at = _r16(at + 2 * self.n_groups)
-        out["zeros"] = at
-        at = _r16(at + (self.n_groups if self.quantization == QUANT_INT4 else 0))
-        out["payload"] = at
-        out["end"] = at + self.payload_bytes
-        return out
-
-    def pack(self) -> bytes:
-        return _HEADER.pack(MAGIC, self.version, 0, self.compression, self.quantization, self.checksum, 0,
-                            self.block_size, self.rows, self.cols, self.group_size, self.secret_len, self.n_blocks,
-                            self.payload_bytes, self.meta_hash)
 
 
 class HctError(ValueError):
     pass
 
 
-def read_header(buf) -> Header:
-    """Parse and sanity-check the header (no checksum is checked here)."""
-    b = bytes(buf[:HEADER_BYTES])
-    if len(b) < HEADER_BYTES:
-        raise HctError("shorter than the 64-byte header")
-    (magic, version, _, compression, quantization, checksum, _, block_size, rows, cols, group_size, secret_len,
-     n_blocks, payload_bytes, meta_hash) = _HEADER.unpack(b)
-    if magic != MAGIC or version != VERSION:
-        raise HctError("not an HCT v2 container")
-    if compression > 1 or quantization > 2 or checksum != CHECKSUM_XXH3 or secret_len < SECRET_MIN:
-        raise HctError("unsupported header fields")
-    if block_size == 0 or n_blocks > (1 << 40) or (cols and rows > (1 << 50) // cols):
-        raise HctError("sizes out of range")
-    if quantization == QUANT_INT4 and (group_size == 0 or cols % group_size):
-        raise HctError("group_size must divide cols")
-    h = Header(compression, quantization, block_size, rows, cols, group_size, secret_len, n_blocks, payload_bytes,
-               meta_hash, version, checksum)
-    if h.sections()["end"] != len(buf):
-        raise HctError(f"container is {len(buf)} bytes, its header says {h.sections()['end']}")
-    return h
+def make_header(compression: int, quantization: int, block_size: int, rows: int, cols: int, group_size: int,
+                secret_len: int, n_blocks: int, payload_bytes: int, meta_hash: int = 0) -> L.LtHct2Header:
+    """A header with its sections laid out (lt_hct2_layout)."""
+    h = L.LtHct2Header(version=L.LT_HCT2_VERSION, compression=compression, quantization=quantization,
+                       checksum=CHECKSUM_XXH3, block_size=block_size, rows=rows, cols=cols, group_size=group_size,
+                       secret_len=secret_len, n_blocks=n_blocks, payload_bytes=payload_bytes, meta_hash=meta_hash)
+    try:
+        return L.lt_hct2_layout(h)
+    except L.LtError as e:
+        raise HctError(str(e)) from e
+
+
+def read_header(buf) -> L.LtHct2Header:
+    """Parse and check the header of a whole container (no checksum is
+    checked here)."""
+    try:
+        return L.lt_hct2_read_header(buf)
+    except L.LtError as e:
+        raise HctError(str(e)) from e
+
+
+def sections(h: L.LtHct2Header) -> dict:
+    """Byte offsets of the sections, and the end of the container."""
+    return {"offsets": h.offsets_at, "hashes": h.hashes_at, "scales": h.scales_at, "zeros": h.zeros_at,
+            "payload": h.payload_at, "end": h.total_bytes}
 
 
 def _device_hashes(data_dev, data_bytes: int, offsets, secret_dev, secret_len: int):
@@ -138,15 +93,15 @@ def write(blocks, block_size: int, rows: int, cols: int, quantization: int, grou
     payload = b"".join(bytes(x) for x in blocks)
     offs = np.zeros(len(blocks) + 1, np.uint64)
     offs[1:] = np.cumsum([len(x) for x in blocks], dtype=np.uint64)
-    hdr = Header(compression, quantization, block_size, rows, cols, group_size, len(secret), len(blocks),
-                 len(payload))
-    sec = hdr.sections()
+    hdr = make_header(compression, quantization, block_size, rows, cols, group_size, len(secret), len(blocks),
+                      len(payload))
+    sec = sections(hdr)
     sc = b"" if scales is None else np.ascontiguousarray(scales, np.uint16).tobytes()
     ze = b"" if zeros is None else np.ascontiguousarray(zeros, np.uint8).tobytes()
     if len(sc) != 2 * hdr.n_groups or len(ze) != (hdr.n_groups if quantization == QUANT_INT4 else 0):
         raise HctError("scales / zero points do not match the shape and quantization")
     meta = bytearray(sec["payload"])
-    meta[:HEADER_BYTES] = hdr.pack()
+    meta[:HEADER_BYTES] = L.lt_hct2_write_header(hdr)
     meta[HEADER_BYTES:HEADER_BYTES + len(secret)] = secret
     meta[sec["offsets"]:sec["offsets"] + offs.nbytes] = offs.tobytes()
     meta[sec["scales"]:sec["scales"] + len(sc)] = sc
@@ -168,7 +123,7 @@ def verify(buf):
     import torch
 
     h = read_header(buf)
-    sec = h.sections()
+    sec = sections(h)
     dev = torch.frombuffer(bytearray(bytes(buf)), dtype=torch.uint8).cuda()
     secret_dev = dev[HEADER_BYTES:HEADER_BYTES + h.secret_len]
     meta = bytearray(bytes(buf[:sec["payload"]]))

@@ -34,6 +34,7 @@ EXPORTED = (
     "lt_dequant_int4", "lt_dequant_int8", "lt_value_dict_decode", "lt_zrle_decode", "lt_lz4_int4_decode",
     "lt_lz4_int4_decode_batch", "lt_lz4_index_batch", "lt_lz4_int4_expand_batch", "lt_lz4_decode",
     "lt_lz4_workspace_bytes", "lt_lz4_int4_decode_noalloc", "lt_xxh3_blocks",
+    "lt_hct2_layout", "lt_hct2_read_header", "lt_hct2_write_header",
     "lt_status_string", "lt_abi_version",
 )
 LT_NOALLOC_MAX_BLOCKS = 512
@@ -53,6 +54,23 @@ class LtLz4Int4Desc(ctypes.Structure):
         ("block_bytes", ctypes.c_int32),
     ]
 
+
+class LtHct2Header(ctypes.Structure):
+    """lt_hct2_header: the stored header fields, then the derived ones."""
+    _fields_ = [
+        ("version", ctypes.c_uint16), ("compression", ctypes.c_uint8), ("quantization", ctypes.c_uint8),
+        ("checksum", ctypes.c_uint8), ("block_size", ctypes.c_uint32), ("rows", ctypes.c_uint64),
+        ("cols", ctypes.c_uint64), ("group_size", ctypes.c_uint32), ("secret_len", ctypes.c_uint32),
+        ("n_blocks", ctypes.c_uint64), ("payload_bytes", ctypes.c_uint64), ("meta_hash", ctypes.c_uint64),
+        ("n_groups", ctypes.c_uint64), ("offsets_at", ctypes.c_uint64), ("hashes_at", ctypes.c_uint64),
+        ("scales_at", ctypes.c_uint64), ("zeros_at", ctypes.c_uint64), ("payload_at", ctypes.c_uint64),
+        ("total_bytes", ctypes.c_uint64),
+    ]
+
+
+LT_HCT2_VERSION = 2
+LT_HCT2_HEADER_BYTES = 64
+LT_HCT2_SECRET_MIN = 136
 
 _lib = None
 
@@ -80,6 +98,11 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.lt_lz4_int4_decode_noalloc.restype = ctypes.c_int
     lib.lt_xxh3_blocks.argtypes = [P, U64, P, I64, P, I32, P, P, P, P, P]
     lib.lt_xxh3_blocks.restype = ctypes.c_int
+    lib.lt_hct2_layout.argtypes = [ctypes.POINTER(LtHct2Header)]
+    lib.lt_hct2_read_header.argtypes = [ctypes.c_char_p, U64, ctypes.POINTER(LtHct2Header)]
+    lib.lt_hct2_write_header.argtypes = [ctypes.POINTER(LtHct2Header), ctypes.c_char_p]
+    for f in ("lt_hct2_layout", "lt_hct2_read_header", "lt_hct2_write_header"):
+        getattr(lib, f).restype = ctypes.c_int
     lib.lt_lz4_workspace_bytes.argtypes = [I64]
     lib.lt_lz4_workspace_bytes.restype = U64
     for f in ("lt_dequant_int4", "lt_dequant_int8", "lt_value_dict_decode", "lt_zrle_decode", "lt_lz4_int4_decode",
@@ -246,3 +269,22 @@ def lt_lz4_int4_decode_noalloc(comp, comp_bytes: int, block_offsets, block_bytes
                                                      _ptr(scales), _ptr(zeros), rows, cols, group_size, _ptr(out),
                                                      _ptr(d_status), _stream(stream, out)),
            "lt_lz4_int4_decode_noalloc")
+
+
+# HCT v2 container header: host functions (host memory, no device)
+def lt_hct2_layout(h: LtHct2Header) -> LtHct2Header:
+    _check(load_library().lt_hct2_layout(ctypes.byref(h)), "lt_hct2_layout")
+    return h
+
+
+def lt_hct2_read_header(buf) -> LtHct2Header:
+    b = bytes(buf)
+    h = LtHct2Header()
+    _check(load_library().lt_hct2_read_header(b, len(b), ctypes.byref(h)), "lt_hct2_read_header")
+    return h
+
+
+def lt_hct2_write_header(h: LtHct2Header) -> bytes:
+    out = ctypes.create_string_buffer(LT_HCT2_HEADER_BYTES)
+    _check(load_library().lt_hct2_write_header(ctypes.byref(h), out), "lt_hct2_write_header")
+    return out.raw
