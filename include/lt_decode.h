@@ -22,9 +22,10 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- *  - Every data pointer is a DEVICE pointer owned by the caller (except the
- *    descriptor array of lt_lz4_int4_decode_batch, a host array read during
- *    the call). The library allocates no memory, frees nothing, never
+ *  - Every data pointer is a DEVICE pointer owned by the caller, except the
+ *    descriptor arrays of the LZ4 batch calls (host arrays read during the
+ *    call) and the buffers of the lt_hct2_* header functions, which are
+ *    host-only and touch no device. The library allocates no memory, frees nothing, never
  *    synchronizes and keeps no pointer after it returns.
  *  - All work is enqueued on `stream` (NULL = the legacy default stream).
  *    A call returns as soon as its kernel is enqueued.
