@@ -559,6 +559,22 @@ def cpu_baseline(hw, budget_s: float = 15.0):
     }
 
 
+def cpu_baseline_value_dict():
+    """The oracle on the whole value-dictionary workload, single-threaded."""
+    import oracle
+    from weight_dequantization_b200.synth import workloads as W
+
+    d = W.v_value_dict()
+    t0 = time.perf_counter()
+    _, st = oracle.value_dict_decode(d["packed"], d["bits"], d["dictionary"], d["n"])
+    dt = time.perf_counter() - t0
+    if st != 0:
+        raise RuntimeError("the oracle reported an error on the value-dictionary workload")
+    return {"value": 2 * d["n"] / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle", "cpu": cpu_model(),
+            "sample": f"the whole workload ({d['n']} elements, {2 * d['n'] / 1e6:.1f} MB decoded in {dt:.2f} s, "
+                      f"single-threaded plain C oracle)"}
+
+
 # ----------------------------------------------------------------------------
 # arms
 # ----------------------------------------------------------------------------
@@ -848,6 +864,8 @@ def run_lt(args, rank, world, local):
             cpu_thr = cpu_baseline_threads(hw, cpu["frac"])
         c1g = c1_graph_steady_state(hw, peak) if "C1" in hw else None
         vd = value_dict_timing(peak) if "V" in only else None
+        if vd is not None and world == 1 and not args.no_cpu_baseline:
+            vd["cpu_baseline"] = cpu_baseline_value_dict()
         result = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": elapsed / K * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

@@ -46,3 +46,9 @@ def test_zero_run_pieces_decode_like_one_call():
     assert st == 0 and nch > 3
     pieces = [t() for t, _ in bench.oracle_sample_tasks({"C3": c3}, frac, 4)]
     assert np.array_equal(np.concatenate([o for o, _ in pieces]), whole)
+
+
+def test_value_dictionary_oracle_baseline_covers_the_workload():
+    r = bench.cpu_baseline_value_dict()
+    assert r["kind"] == "oracle" and r["cores"] == 1 and r["value"] > 0
+    assert str(W.v_value_dict()["n"]) in r["sample"]
