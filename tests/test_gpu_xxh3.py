@@ -127,3 +127,50 @@ def test_container_verified_on_the_device():
     bad[100] ^= 0xFF  # a byte of the secret: the metadata hash no longer matches
     assert hct.verify(bytes(bad)) == (False, None, False)
     assert oracle.hct2_validate(bytes(bad))[0] == oracle.HCT_META_MISMATCH
+
+
+def _f16_bits(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16).ravel()
+
+
+def test_container_decodes_like_the_oracle():
+    from weight_dequantization_b200 import hct
+    blocks, bs, rows, cols, G, scales, zeros, secret = _container_parts()
+    c = hct.write(blocks, bs, rows, cols, hct.QUANT_INT4, G, scales, zeros, secret)
+    comp = np.frombuffer(b"".join(blocks), np.uint8)
+    offs = np.concatenate([[0], np.cumsum([len(b) for b in blocks])]).astype(np.uint64)
+    want, st = oracle.lz4_int4_decode(comp, offs, bs, scales, zeros, rows, cols, G)
+    assert st == 0
+    assert np.array_equal(_f16_bits(hct.decode(c)), want)
+    bad = bytearray(c)
+    bad[-1] ^= 0xFF
+    with pytest.raises(hct.HctError):
+        hct.decode(bytes(bad))
+
+
+def test_uncompressed_and_raw_containers_decode_like_the_oracle():
+    from weight_dequantization_b200 import hct
+    from weight_dequantization_b200.synth import fp16_uniform, int8_normal, relu_runs, u8_uniform
+    secret = RNG.integers(0, 256, 136, dtype=np.uint8).tobytes()
+    # INT4 without compression, payload in two checksummed blocks
+    rows, cols, G = 8, 1024, 64
+    packed = int4_gauss_groups_packed(8, rows * cols)
+    s4 = fp16_uniform(8, rows * cols // G, 0.001, 0.1, stream=1)
+    z4 = u8_uniform(8, rows * cols // G, 0, 15, stream=2)
+    c = hct.write([packed[:1000].tobytes(), packed[1000:].tobytes()], 4096, rows, cols, hct.QUANT_INT4, G, s4, z4,
+                  secret, compression=hct.COMPRESSION_NONE)
+    want, _ = oracle.dequant_int4(packed, s4, z4, rows, cols, G)
+    assert np.array_equal(_f16_bits(hct.decode(c)), want)
+    # INT8 per row without compression
+    q = int8_normal(9, 16 * 512, 32.0)
+    s8 = fp16_uniform(9, 16, 0.001, 0.02, stream=1)
+    c = hct.write([q.view(np.uint8).tobytes()], 8192, 16, 512, hct.QUANT_INT8, 0, s8, None, secret,
+                  compression=hct.COMPRESSION_NONE)
+    want, _ = oracle.dequant_int8(q, s8, None, True, 16, 512)
+    assert np.array_equal(_f16_bits(hct.decode(c)), want)
+    # raw fp16 in LZ4 blocks
+    x = relu_runs(10, 3 * 32768)
+    comp, offs = lz4_compress_blocks(x.view(np.uint8), 65536)
+    blocks = [comp[offs[b]:offs[b + 1]].tobytes() for b in range(len(offs) - 1)]
+    c = hct.write(blocks, 65536, 3, 32768, hct.QUANT_NONE, 0, None, None, secret)
+    assert np.array_equal(_f16_bits(hct.decode(c)), x)

@@ -64,3 +64,15 @@ def test_parser_rejects_each_bad_field(field, offset, value):
     with pytest.raises(hct.HctError):
         hct.read_header(bytes(c))
     assert oracle.hct2_validate(bytes(c))[0] == oracle.HCT_BAD_HEADER, field
+
+
+def test_decode_rejects_payloads_that_cannot_hold_the_shape():
+    sec = bytes(range(136))
+    # INT4 without compression: 4 x 64 codes need 128 payload bytes, 100 given
+    short = hct2_build([bytes(100)], 4096, 4, 64, 64, 1, bytes(2 * 4), bytes(4), sec, compression=0)
+    with pytest.raises(hct.HctError):
+        hct.decode(short, check=False)
+    # LZ4 + INT4: 4 x 65536 codes are 128 KB packed, two 64 KB blocks; one given
+    one_block = hct2_build([b"\x00" * 8], 65536, 4, 65536, 128, 1, bytes(2 * 2048), bytes(2048), sec)
+    with pytest.raises(hct.HctError):
+        hct.decode(one_block, check=False)

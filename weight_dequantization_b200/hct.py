@@ -149,3 +149,56 @@ def verify(buf):
     if st != L.LT_ERR_CHECKSUM:
         raise HctError(L.status_string(st))
     return False, int(first.item()), True
+
+
+def decode(buf, check: bool = True):
+    """Decode a container on the device into a new fp16 [rows, cols] tensor,
+    after checking its checksums (``check``). LZ4 + INT4 takes the fused
+    decode, INT4 and INT8 the dequant kernels, LZ4 of raw fp16 the LZ4
+    decoder. Raises HctError on a checksum mismatch, a corrupt stream or a
+    combination no kernel implements (LZ4 + INT8)."""
+    import torch
+
+    h = read_header(buf)
+    if check:
+        ok, bad, meta_ok = verify(buf)
+        if not ok:
+            raise HctError("metadata checksum mismatch" if not meta_ok else f"checksum mismatch in block {bad}")
+    sec = sections(h)
+    n = h.rows * h.cols
+    # bytes the decoded stream must hold: packed INT4, INT8 or raw fp16
+    need = {QUANT_INT4: (n + 1) // 2, QUANT_INT8: n, QUANT_NONE: 2 * n}[h.quantization]
+    if h.compression == COMPRESSION_LZ4:
+        if h.n_blocks != (need + h.block_size - 1) // h.block_size:
+            raise HctError(f"{h.n_blocks} blocks of {h.block_size} bytes cannot hold {need} bytes")
+    elif h.payload_bytes < need:
+        raise HctError(f"the payload holds {h.payload_bytes} bytes, the shape needs {need}")
+    dev = torch.frombuffer(bytearray(bytes(buf)), dtype=torch.uint8).cuda()
+    out = torch.empty((h.rows, h.cols), dtype=torch.float16, device="cuda")
+    if n == 0:
+        return out
+    payload = dev[sec["payload"]:]
+    offs = dev[sec["offsets"]:sec["offsets"] + 8 * (h.n_blocks + 1)].view(torch.int64)
+    scales = dev[sec["scales"]:sec["scales"] + 2 * h.n_groups].view(torch.float16)
+    zeros = dev[sec["zeros"]:sec["zeros"] + h.n_groups] if h.quantization == QUANT_INT4 else None
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if h.compression == COMPRESSION_LZ4 and h.quantization == QUANT_INT4:
+        ws = torch.empty(max(L.lt_lz4_workspace_bytes(h.n_blocks), 16), dtype=torch.uint8, device="cuda")
+        L.lt_lz4_int4_decode(payload, h.payload_bytes, offs, h.block_size, scales, zeros, h.rows, h.cols,
+                             h.group_size, out, ws, status)
+    elif h.compression == COMPRESSION_LZ4 and h.quantization == QUANT_NONE:
+        ws = torch.empty(max(L.lt_lz4_workspace_bytes(h.n_blocks), 16), dtype=torch.uint8, device="cuda")
+        L.lt_lz4_decode(payload, h.payload_bytes, offs, h.block_size, out.view(torch.uint8).view(-1), 2 * n, ws,
+                        status)
+    elif h.compression == COMPRESSION_NONE and h.quantization == QUANT_INT4:
+        L.lt_dequant_int4(payload, scales, zeros, h.rows, h.cols, h.group_size, out)
+    elif h.compression == COMPRESSION_NONE and h.quantization == QUANT_INT8:
+        L.lt_dequant_int8(payload, scales, None, L.LT_SCALE_PER_ROW, h.rows, h.cols, out)
+    elif h.compression == COMPRESSION_NONE and h.quantization == QUANT_NONE:
+        out.view(torch.uint8).view(-1).copy_(payload[:2 * n])
+    else:
+        raise HctError("LZ4-compressed INT8 has no decoder")
+    st = int(status.item())
+    if st != 0:
+        raise HctError(L.status_string(st))
+    return out
