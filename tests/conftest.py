@@ -12,9 +12,10 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
 
 
-# The checksum tests are collected after every other module, so that under
-# -x a failure in them leaves the decoders' parity tests already run.
-RUN_LAST = ("test_gpu_xxh3.py",)
+# The checksum and streaming tests are collected after every other module,
+# so that under -x a failure in them leaves the decoders' parity tests
+# already run.
+RUN_LAST = ("test_gpu_xxh3.py", "test_gpu_stream.py")
 
 
 def pytest_collection_modifyitems(config, items):
