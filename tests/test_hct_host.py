@@ -76,3 +76,9 @@ def test_decode_rejects_payloads_that_cannot_hold_the_shape():
     one_block = hct2_build([b"\x00" * 8], 65536, 4, 65536, 128, 1, bytes(2 * 2048), bytes(2048), sec)
     with pytest.raises(hct.HctError):
         hct.decode(one_block, check=False)
+
+
+def test_decode_refuses_lz4_int8_before_any_device_work():
+    c = hct2_build([b"\x00"], 65536, 2, 8, 0, 2, bytes(4), b"", bytes(range(136)))
+    with pytest.raises(hct.HctError):
+        hct.decode(c)

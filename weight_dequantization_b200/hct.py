@@ -160,6 +160,8 @@ def decode(buf, check: bool = True):
     import torch
 
     h = read_header(buf)
+    if h.compression == COMPRESSION_LZ4 and h.quantization == QUANT_INT8:
+        raise HctError("LZ4-compressed INT8 has no decoder")
     if check:
         ok, bad, meta_ok = verify(buf)
         if not ok:
@@ -194,10 +196,8 @@ def decode(buf, check: bool = True):
         L.lt_dequant_int4(payload, scales, zeros, h.rows, h.cols, h.group_size, out)
     elif h.compression == COMPRESSION_NONE and h.quantization == QUANT_INT8:
         L.lt_dequant_int8(payload, scales, None, L.LT_SCALE_PER_ROW, h.rows, h.cols, out)
-    elif h.compression == COMPRESSION_NONE and h.quantization == QUANT_NONE:
+    else:  # neither compressed nor quantized: the payload is the fp16 tensor
         out.view(torch.uint8).view(-1).copy_(payload[:2 * n])
-    else:
-        raise HctError("LZ4-compressed INT8 has no decoder")
     st = int(status.item())
     if st != 0:
         raise HctError(L.status_string(st))
