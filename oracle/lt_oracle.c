@@ -43,7 +43,13 @@
  * (u16 zero run, u16 literal count, fp16 literals)* record list with
  * little-endian fields; a value dictionary is one table of 2^bits fp16
  * entries per tensor, indexed by bits-wide fields packed least-significant
- * bits first (the INT4 nibble order).
+ * bits first (the INT4 nibble order); decode -> GEMM multiplies an fp16
+ * input by the decoded [K, N] weight.
+ *
+ * Parity unpinned by the pages (the tests pin this code's arithmetic, but
+ * the pages fix no value for these readings): the zero point for z != 0,
+ * the zero-run byte layout, the value-dictionary layout beyond the 4-bit
+ * order, and the HCT v2 byte layout.
  *
  * Status values returned by the decoders: 0 ok, 4 corrupt stream, 5 decoded
  * size differs from the declared size, 1 invalid argument. The container
