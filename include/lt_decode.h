@@ -14,6 +14,9 @@
  *                               64 KB blocks of Phase 3.1 / Phase 6.1
  *   block checksums             "GPU Compression Pipeline - TDD Roadmap",
  *                               Phase 6.1 HCT Format V2 (XXH3 checksums)
+ *   decode -> matrix multiply   "LoreToken-powered GPU memory layer", decode
+ *                               + GEMM; "GPU Compression Pipeline - TDD
+ *                               Roadmap", Phase 4.1
  *   value-dictionary decoding   "LoreToken-powered GPU memory layer",
  *                               compression strategies (value dictionary
  *                               compression), and the "GPU sidecar brain"
@@ -57,7 +60,7 @@
 extern "C" {
 #endif
 
-#define LT_ABI_VERSION 5
+#define LT_ABI_VERSION 6
 
 /* Same type as cudaStream_t. */
 typedef struct CUstream_st *lt_stream_t;
@@ -73,7 +76,7 @@ typedef enum {
   LT_ERR_CORRUPT_STREAM = 4, /* (device status) malformed LZ4 / zero-run data */
   LT_ERR_SIZE_MISMATCH = 5,  /* (device status) stream decodes to a different length */
   LT_ERR_CUDA = 6,           /* a CUDA launch failed */
-  LT_ERR_TIMEOUT = 7,        /* (device status) an internal on-chip wait ran out; reserved: no current kernel waits */
+  LT_ERR_TIMEOUT = 7,        /* (device status) an internal on-chip wait ran out (lt_int4_gemm) */
   LT_ERR_CHECKSUM = 8        /* (device status) a block's checksum differs from the stored one */
 } lt_status;
 
@@ -375,7 +378,10 @@ lt_status lt_lz4_decode(const uint8_t *comp, uint64_t comp_bytes, const uint64_t
  *  - The first call on each device looks up the scratch array's device
  *    address (cudaGetSymbolAddress) with that device current; make that
  *    first call before any stream capture. A failed lookup returns
- *    LT_ERR_CUDA.
+ *    LT_ERR_CUDA. The address is kept with the id of the CUDA context it
+ *    was taken in: after the context is destroyed and created again (e.g.
+ *    cudaDeviceReset), the next call is again a first call in the new
+ *    context and looks the address up again.
  *  - All calls on a device share the one scratch array and it keeps the
  *    last call's contents (nothing in it needs to start at zero). Calls whose
  *    work overlaps on the GPU -- on different streams, or from different host
@@ -387,6 +393,45 @@ lt_status lt_lz4_int4_decode_noalloc(const uint8_t *comp, uint64_t comp_bytes, c
                                      int32_t block_bytes, const lt_half *scales, const uint8_t *zeros, int64_t rows,
                                      int64_t cols, int32_t group_size, lt_half *out, int32_t *d_status,
                                      lt_stream_t stream);
+
+/*
+ * Fused INT4 decode -> matrix multiply on the tensor cores
+ * ("LoreToken-powered GPU memory layer": decode + GEMM, decoded weights
+ * feeding a matrix multiply; "GPU Compression Pipeline - TDD Roadmap",
+ * Phase 4.1: a decoded weight tensor used in input.matmul(weights)).
+ *
+ *   out[M, N] = x[M, K] . W[K, N]
+ *
+ *   x        M x K binary16, row-major (row stride K), 16-byte aligned.
+ *   packed, scales, zeros, group_size
+ *            W in the layout of lt_dequant_int4 with rows = K, cols = N:
+ *            ceil(K*N/2) bytes of codes (16-byte aligned), K*N/group_size
+ *            binary16 scales and uint8 zero points (or NULL) laid out
+ *            [K, N/group_size]. W[k, n] is exactly lt_dequant_int4's output
+ *            element k*N + n; it is never written to memory: each tile is
+ *            decoded into shared memory and fed to the tensor cores.
+ *   out      M x N binary16, row-major, 16-byte aligned: the fp32 sum of the
+ *            exact products x[m, k] * W[k, n] over k, rounded once to
+ *            binary16. The order of the fp32 additions is the hardware's
+ *            (and, with a split of K, partial sums are added in split
+ *            order), so out differs from the exact sum by at most about
+ *            K * 2^-23 * sum_k |x[m, k] W[k, n]| plus half an ulp of out.
+ *   workspace, workspace_bytes
+ *            optional fp32 scratch for splitting K across CTAs when the
+ *            output has few tiles (small M): lt_int4_gemm_workspace_bytes
+ *            gives the size the call would use (0: no split). NULL or a
+ *            smaller workspace computes without splitting (correct, fewer
+ *            CTAs). 16-byte aligned, caller-owned, reusable by the next
+ *            call on the same stream.
+ *   Shapes: M >= 1, K a multiple of 64, N a multiple of 256, group_size a
+ *   multiple of 32 that divides N, else LT_ERR_UNSUPPORTED.
+ *   Device status: LT_ERR_TIMEOUT if an on-chip wait of the kernel ran out
+ *   (an internal error; the output is then unspecified).
+ */
+uint64_t lt_int4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+lt_status lt_int4_gemm(const lt_half *x, int64_t M, int64_t K, const uint8_t *packed, const lt_half *scales,
+                       const uint8_t *zeros, int64_t N, int32_t group_size, lt_half *out, void *workspace,
+                       uint64_t workspace_bytes, int32_t *d_status, lt_stream_t stream);
 
 /* Static, human-readable name of a status code. */
 const char *lt_status_string(lt_status s);

@@ -40,8 +40,18 @@ def test_library_exports_every_declared_symbol(lib):
         assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
 
 
+def test_binding_constants_match_the_header():
+    text = open(HEADER).read()
+    for name in ("LT_NOALLOC_MAX_BLOCKS", "LT_LZ4_BATCH_MAX", "LT_ABI_VERSION"):
+        m = re.search(r"#define\s+%s\s+(\d+)" % name, text)
+        assert m, name
+        want = int(m.group(1))
+        got = L.abi_version() if name == "LT_ABI_VERSION" else getattr(L, name)
+        assert got == want, (name, got, want)
+
+
 def test_abi_version_and_status_strings(lib):
-    assert L.abi_version() == 5
+    assert L.abi_version() == 6
     for code in range(9):
         s = L.status_string(code)
         assert s and s != "unknown status"
@@ -120,3 +130,27 @@ def test_binding_rejects_host_tensors():
     x = torch.zeros(16, dtype=torch.uint8)
     with pytest.raises(TypeError):
         L.lt_dequant_int4(x, x, None, 1, 32, 32, x, stream=0)
+
+
+def test_gemm_host_argument_errors(lib):
+    P = 0x1000  # never dereferenced: every call below is refused before any CUDA call
+    ok = dict(x=P, M=4, K=128, packed=P, scales=P, zeros=None, N=512, G=128, out=P)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lib.lt_int4_gemm(a["x"], a["M"], a["K"], a["packed"], a["scales"], a["zeros"], a["N"], a["G"],
+                                a["out"], None, 0, None, None)
+
+    assert call(N=384) == L.LT_ERR_UNSUPPORTED     # N not a multiple of 256
+    assert call(K=96) == L.LT_ERR_UNSUPPORTED      # K not a multiple of 64
+    assert call(G=16) == L.LT_ERR_UNSUPPORTED      # group not a multiple of 32
+    assert call(G=96) == L.LT_ERR_UNSUPPORTED      # group does not divide N
+    assert call(M=-1) == L.LT_ERR_INVALID_ARG
+    assert call(x=None) == L.LT_ERR_INVALID_ARG
+    assert call(x=P + 8) == L.LT_ERR_MISALIGNED   # x must be 16-byte aligned (tiled copies)
+    assert call(out=P + 2) == L.LT_ERR_MISALIGNED
+    assert call(M=0) == L.LT_OK                    # empty: nothing enqueued
+    # a split of K is offered only when the output has fewer tiles than SMs
+    assert L.lt_int4_gemm_workspace_bytes(1, 8192, 8192) > 0
+    assert L.lt_int4_gemm_workspace_bytes(4096, 8192, 8192) == 0
+    assert L.lt_int4_gemm_workspace_bytes(1, 8192, 100) == 0

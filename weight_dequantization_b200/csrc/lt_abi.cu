@@ -45,6 +45,34 @@ int blocks_per_sm(const void *kernel, int threads, size_t dyn_smem) {
 
 lt_status launch_status() { return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA; }
 
+void *driver_fn(const char *name) {
+  // the CUDA driver API through the runtime's entry-point lookup, so that the
+  // library does not link libcuda itself (it loads on hosts without a GPU)
+  void *fn = nullptr;
+  cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+  if (cudaGetDriverEntryPointByVersion(name, &fn, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return fn;
+}
+
+bool current_context_id(unsigned long long *id) {
+  typedef int (*ctx_get_current_t)(void **);
+  typedef int (*ctx_get_id_t)(void *, unsigned long long *);
+  static ctx_get_current_t get_current = nullptr;
+  static ctx_get_id_t get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    get_current = (ctx_get_current_t)driver_fn("cuCtxGetCurrent");
+    get_id = (ctx_get_id_t)driver_fn("cuCtxGetId");
+  });
+  void *ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != 0 || !ctx) return false;
+  return get_id(ctx, id) == 0;
+}
+
 }  // namespace lt
 
 LT_API const char *lt_status_string(lt_status s) {

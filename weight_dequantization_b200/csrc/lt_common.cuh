@@ -136,5 +136,10 @@ int num_sms();
 // resident blocks per SM of a kernel (cached per kernel and device)
 int blocks_per_sm(const void *kernel, int threads, size_t dyn_smem);
 lt_status launch_status();
+// a CUDA driver API function by name (nullptr if unavailable)
+void *driver_fn(const char *name);
+// unique id of the calling thread's current CUDA context (false if none):
+// a context destroyed and created again (cudaDeviceReset) gets a new id
+bool current_context_id(unsigned long long *id);
 
 }  // namespace lt

@@ -1086,23 +1086,39 @@ constexpr uint64_t kNoAllocBytes = (uint64_t)LT_NOALLOC_MAX_BLOCKS * (16ull + 16
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
 std::mutex g_noalloc_mu;
-void *g_noalloc_addr[64] = {nullptr};
+struct NoAllocAddr {
+  unsigned long long ctx_id;  // the context the address belongs to
+  void *addr;
+};
+NoAllocAddr g_noalloc_addr[64] = {};
 
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device (the first call on a device does it).
+// Device address of g_noalloc_scratch in the current context. It is looked
+// up on the first call in a context (with that device current) and kept per
+// device together with the context's id; a call from a new context on that
+// device -- e.g. after cudaDeviceReset, which destroys the primary context
+// and with it this module's copy of the array -- looks it up again instead
+// of using the old address.
 lt_status noalloc_scratch(void **out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LT_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return LT_ERR_CUDA;
+  }
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
+  unsigned long long ctx = 0;
+  const bool have_ctx = current_context_id(&ctx);
+  if (!g_noalloc_addr[dev].addr || !have_ctx || g_noalloc_addr[dev].ctx_id != ctx) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
       cudaGetLastError();
       return LT_ERR_CUDA;
     }
-    g_noalloc_addr[dev] = p;
+    // cudaGetSymbolAddress made the primary context current if none was:
+    // record the id of the context the address was taken in
+    if (!have_ctx && !current_context_id(&ctx)) ctx = 0;
+    g_noalloc_addr[dev] = NoAllocAddr{ctx, p};
   }
-  *out = g_noalloc_addr[dev];
+  *out = g_noalloc_addr[dev].addr;
   return LT_OK;
 }
 
