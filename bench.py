@@ -6,6 +6,8 @@ One step = one pass of every decode workload over its synthetic input:
   C2  INT8 per-row dequant, 8192 x 8192
   C3  zero-run decode, 8 x 2048 x 11008 fp16 ReLU-like activations
   C4  fused LZ4 -> INT4 -> fp16, 4096 x 14336, group 128, 64 KB blocks
+  C4u INT4 group dequant of C4's matrix without the LZ4 layer (the
+      uncompressed variant at the large shape, 4096 x 14336, group 128)
   C5  8 Llama-2-70B-shaped layers (q, o, k, v, gate, up, down), fused LZ4 ->
       INT4 -> fp16: one index launch over the blocks of all layers, then each
       layer expanded (one launch) into one reused buffer
@@ -64,9 +66,13 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=8, help="C5 layers (8 is the workload)")
-    ap.add_argument("--only", default="C1,C2,C3,C4,C5,V",
+    ap.add_argument("--no-parity", action="store_true",
+                    help="skip the parity pass (profiling runs only: the line then says parity was not checked)")
+    ap.add_argument("--only", default="C1,C2,C3,C4,C4u,C5,V,S,G",
                     help="comma-separated subset of the workloads to run (profiling); the bench line uses all. "
-                         "C1-C5 form the timed step; V (value-dictionary decode) is timed on its own afterwards")
+                         "C1-C5 form the timed step; V (value-dictionary decode), S (the streaming API over "
+                         "the C5 layers) and G (fused decode -> GEMM on the C5 shapes) are timed on their own "
+                         "afterwards")
     return ap.parse_args()
 
 
@@ -174,7 +180,10 @@ def gpu_id_for(dev_index: int) -> str:
 # workloads
 # ----------------------------------------------------------------------------
 
-def build_host_workload(rank: int, layers: int, only=("C1", "C2", "C3", "C4", "C5")):
+STEP_CODECS = ("C1", "C2", "C3", "C4", "C4u")  # single-call units of a step, in order; then C5
+
+
+def build_host_workload(rank: int, layers: int, only=("C1", "C2", "C3", "C4", "C4u", "C5")):
     """Seeded host inputs; each rank gets its own seeds (weak scaling)."""
     from weight_dequantization_b200.synth import workloads as W
 
@@ -183,10 +192,18 @@ def build_host_workload(rank: int, layers: int, only=("C1", "C2", "C3", "C4", "C
         "C1": lambda: W.c1_int4(seed=1 + off),
         "C2": lambda: W.c2_int8(seed=2 + off),
         "C3": lambda: W.c3_zrle(seed=3 + off),
-        "C4": lambda: W.c4_lz4_int4(seed=4 + off),
+        "C4": lambda: W.c4_lz4_int4(seed=4 + off, keep_packed="C4u" in only),
         "C5": lambda: W.c5_layers(layers=layers, seed=5 + off),
     }
-    return {k: make[k]() for k in ("C1", "C2", "C3", "C4", "C5") if k in only}
+    hw = {k: make[k]() for k in ("C1", "C2", "C3", "C4", "C5") if k in only or (k == "C4" and "C4u" in only)}
+    if "C4u" in only:
+        # the same matrix, codes, scales and zero points as C4, not compressed
+        c4 = hw["C4"]
+        hw["C4u"] = dict(kind="int4", rows=c4["rows"], cols=c4["cols"], group_size=c4["group_size"],
+                         packed=c4.pop("packed"), scales=c4["scales"], zeros=c4["zeros"])
+        if "C4" not in only:
+            del hw["C4"]
+    return hw
 
 
 def nbytes(a) -> int:
@@ -209,6 +226,9 @@ def algorithmic_bytes(hw):
         c4 = hw["C4"]
         out["C4"] = (nbytes(c4["comp"]) + nbytes(c4["offsets"]) + nbytes(c4["scales"]) + nbytes(c4["zeros"]),
                      2 * c4["rows"] * c4["cols"])
+    if "C4u" in hw:
+        c = hw["C4u"]
+        out["C4u"] = (nbytes(c["packed"]) + nbytes(c["scales"]) + nbytes(c["zeros"]), 2 * c["rows"] * c["cols"])
     layer = []
     if "C5" in hw:
         for mats in hw["C5"]:
@@ -272,6 +292,11 @@ class DeviceWorkload:
             self.c4 = dict(comp=put(c4["comp"]), offsets=put(c4["offsets"]), scales=put(c4["scales"]),
                            zeros=put(c4["zeros"]))
             self.c4_out = torch.empty(c4["rows"] * c4["cols"], dtype=torch.float16, device="cuda")
+        if "C4u" in hw:
+            c = hw["C4u"]
+            unit[0] = "C4u"
+            self.c4u = dict(packed=put(c["packed"]), scales=put(c["scales"]), zeros=put(c["zeros"]))
+            self.c4u_out = torch.empty(c["rows"] * c["cols"], dtype=torch.float16, device="cuda")
         self.c5 = []
         if "C5" in hw:
             layer_elems = max(sum(m["rows"] * m["cols"] for m in mats) for mats in hw["C5"])
@@ -313,7 +338,7 @@ class DeviceWorkload:
         c5 = [("C5", i) for i in range(len(self.c5))]
         if two_step and c5:
             c5 = ["C5index"] + [("C5x", i) for i in range(len(self.c5))]
-        return [u for u in ("C1", "C2", "C3", "C4") if u in hw] + c5
+        return [u for u in STEP_CODECS if u in hw] + c5
 
     def run_unit(self, u, s):
         """Issue unit u's decode call on stream s."""
@@ -337,6 +362,10 @@ class DeviceWorkload:
             L.lt_lz4_int4_decode(self.c4["comp"], int(c4["comp"].size), self.c4["offsets"], c4["block_bytes"],
                                  self.c4["scales"], self.c4["zeros"], c4["rows"], c4["cols"], c4["group_size"],
                                  self.c4_out, self.ws, self.status, s)
+        elif u == "C4u":
+            c = hw["C4u"]
+            L.lt_dequant_int4(self.c4u["packed"], self.c4u["scales"], self.c4u["zeros"], c["rows"], c["cols"],
+                              c["group_size"], self.c4u_out, s)
         elif u == "C5index":
             L.lt_lz4_index_batch(self.c5_all, self.ws, s)
         elif u[0] == "C5x":
@@ -359,7 +388,7 @@ class DeviceWorkload:
         n = 0
         for u in self.units():
             self.run_unit(u, s)
-            mark(u if u in ("C1", "C2", "C3", "C4") else "C5")
+            mark(u if u in STEP_CODECS else "C5")
             n += 1
         return n  # kernel launches of this step
 
@@ -394,10 +423,11 @@ def launches_per_step(hw) -> int:
     # every call takes its vector path (no scalar tail launch): all element
     # counts are multiples of 8, groups multiples of 8, buffers 256-byte aligned
     n = 0
-    if "C1" in hw:
-        c1 = hw["C1"]
-        assert (c1["rows"] * c1["cols"]) % 8 == 0 and c1["group_size"] % 8 == 0
-        n += 1
+    for u in ("C1", "C4u"):
+        if u in hw:
+            c1 = hw[u]
+            assert (c1["rows"] * c1["cols"]) % 8 == 0 and c1["group_size"] % 8 == 0
+            n += 1
     if "C2" in hw:
         c2 = hw["C2"]
         assert (c2["rows"] * c2["cols"]) % 8 == 0 and c2["cols"] % 8 == 0
@@ -421,8 +451,10 @@ def oracle_sample_step(hw, frac: float):
 
     t0 = time.perf_counter()
     dec = 0
-    if "C1" in hw:
-        c1 = hw["C1"]
+    for u in ("C1", "C4u"):
+        if u not in hw:
+            continue
+        c1 = hw[u]
         r1 = max(1, int(c1["rows"] * frac))
         n1 = r1 * c1["cols"]
         g1 = n1 // c1["group_size"]
@@ -469,12 +501,14 @@ def oracle_sample_tasks(hw, frac: float, pieces: int):
         k = max(1, min(pieces, n))
         return [(n * i // k, n * (i + 1) // k) for i in range(k) if n * i // k < n * (i + 1) // k]
 
-    if "C1" in hw:
-        c1 = hw["C1"]
+    for u in ("C1", "C4u"):
+        if u not in hw:
+            continue
+        c1 = hw[u]
         r1 = max(1, int(c1["rows"] * frac))
         cols, G = c1["cols"], c1["group_size"]
         for a, b in split(r1):
-            tasks.append((lambda a=a, b=b: oracle.dequant_int4(
+            tasks.append((lambda a=a, b=b, c1=c1, cols=cols, G=G: oracle.dequant_int4(
                 c1["packed"][a * cols // 2:b * cols // 2], c1["scales"][a * cols // G:b * cols // G],
                 c1["zeros"][a * cols // G:b * cols // G], b - a, cols, G), 2 * (b - a) * cols))
     if "C2" in hw:
@@ -510,6 +544,157 @@ def oracle_sample_tasks(hw, frac: float, pieces: int):
         for m in mats:
             lz4_tasks(m)
     return tasks
+
+
+# ----------------------------------------------------------------------------
+# parity gate: one step's outputs against the oracle, every element
+# ----------------------------------------------------------------------------
+
+def _ulp_stats(got, want):
+    """(elements, elements that differ, max binary16 ulp distance); +0 == -0
+    and NaN == NaN as in the tests."""
+    import numpy as np
+
+    if got.shape != want.shape:
+        return want.size, want.size, 1 << 20
+    if np.array_equal(got, want):
+        return want.size, 0, 0
+    a, b = got.astype(np.int64), want.astype(np.int64)
+    oa = np.where(a & 0x8000, -(a & 0x7FFF), a)
+    ob = np.where(b & 0x8000, -(b & 0x7FFF), b)
+    nan_a = ((a & 0x7C00) == 0x7C00) & ((a & 0x3FF) != 0)
+    nan_b = ((b & 0x7C00) == 0x7C00) & ((b & 0x3FF) != 0)
+    d = np.abs(oa - ob)
+    d = np.where(nan_a & nan_b, 0, d)
+    d = np.where(nan_a ^ nan_b, 1 << 20, d)
+    return want.size, int((d > 0).sum()), int(d.max())
+
+
+def _lz4_block_tasks(m, base_elem: int, per: int = 64):
+    """(oracle call, first output element) per range of `per` blocks of
+    matrix m, whose output starts at element base_elem of its buffer."""
+    import numpy as np
+
+    import oracle
+
+    bb, G = m["block_bytes"], m["group_size"]
+    n = m["rows"] * m["cols"]
+    nb = len(m["offsets"]) - 1
+    tasks = []
+    for a in range(0, nb, per):
+        b = min(nb, a + per)
+        c0, c1 = 2 * a * bb, min(n, 2 * b * bb)
+        s0, s1 = int(m["offsets"][a]), int(m["offsets"][b])
+        offs = (m["offsets"][a:b + 1] - np.uint64(s0)).astype(np.uint64)
+        g0, g1 = c0 // G, (c1 + G - 1) // G
+        tasks.append((lambda m=m, s0=s0, s1=s1, offs=offs, g0=g0, g1=g1, c0=c0, c1=c1: oracle.lz4_int4_decode(
+            m["comp"][s0:s1], offs, bb, m["scales"][g0:g1], m["zeros"][g0:g1], 1, c1 - c0, G), base_elem + c0))
+    return tasks
+
+
+def _row_tasks(fn, rows: int, cols: int, per_rows: int):
+    return [(lambda a=a, b=min(rows, a + per_rows): fn(a, b), a * cols) for a in range(0, rows, per_rows)]
+
+
+def parity_pass(dw, hw):
+    """Issue one step's decode calls in order; after each call read its
+    output back and compare every element with the oracle's (computed on
+    all host cores, independent row / chunk / block ranges). Returns
+    ({unit: verdict}, ok). Dequantized outputs must be within 1 binary16
+    ulp of the oracle (0 expected), zero-run output bit for bit."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import numpy as np
+    import torch
+
+    import oracle
+
+    s = torch.cuda.current_stream()
+    threads = os.cpu_count() or 1
+    verdict, ok = {}, True
+
+    def host_bits(t):
+        return t.cpu().view(torch.int16).numpy().view(np.uint16)
+
+    def run(ex, tasks, got):
+        n = bad = worst = 0
+        for want_st, k0 in ex.map(lambda t: (t[0](), t[1]), tasks):
+            want, st = want_st
+            if st != 0:
+                return None
+            a, b, w = _ulp_stats(got[k0:k0 + want.size], want)
+            n, bad, worst = n + a, bad + b, max(worst, w)
+        return n, bad, worst
+
+    def record(name, res, total, exact):
+        nonlocal ok
+        if res is None:
+            verdict[name] = "oracle reported an error"
+            ok = False
+            return
+        n, bad, worst = res
+        good = n == total and worst <= (0 if exact else 1)
+        ok = ok and good
+        verdict[name] = (f"bit-exact, {n} of {total} elements" if bad == 0 and n == total else
+                         f"{bad} of {n} elements differ (max {worst} ulp){'' if good else ': FAILED'}")
+
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        for u in dw.units():
+            dw.run_unit(u, s)
+            torch.cuda.synchronize()
+            if u in ("C1", "C4u"):
+                c = hw[u]
+                cols, G = c["cols"], c["group_size"]
+                fn = (lambda a, b, c=c, cols=cols, G=G: oracle.dequant_int4(
+                    c["packed"][a * cols // 2:b * cols // 2], c["scales"][a * cols // G:b * cols // G],
+                    c["zeros"][a * cols // G:b * cols // G], b - a, cols, G))
+                out = dw.c1_out if u == "C1" else dw.c4u_out
+                record(u, run(ex, _row_tasks(fn, c["rows"], cols, 64), host_bits(out)), c["rows"] * cols, False)
+            elif u == "C2":
+                c = hw["C2"]
+                cols = c["cols"]
+                fn = (lambda a, b: oracle.dequant_int8(c["q"][a * cols:b * cols], c["scales"][a:b], None, True,
+                                                       b - a, cols))
+                record(u, run(ex, _row_tasks(fn, c["rows"], cols, 128), host_bits(dw.c2_out)), c["rows"] * cols,
+                       False)
+            elif u == "C3":
+                c = hw["C3"]
+                ce, nch = c["chunk_elems"], len(c["offsets"]) - 1
+                tasks = []
+                for a in range(0, nch, 512):
+                    b = min(nch, a + 512)
+                    n_sub = min(c["n"], b * ce) - a * ce
+                    tasks.append((lambda a=a, b=b, n_sub=n_sub: oracle.zrle_decode(c["enc"], c["offsets"][a:b + 1],
+                                                                                    n_sub, ce), a * ce))
+                record(u, run(ex, tasks, host_bits(dw.c3_out)), c["n"], True)
+            elif u == "C4":
+                c = hw["C4"]
+                record(u, run(ex, _lz4_block_tasks(c, 0), host_bits(dw.c4_out)), c["rows"] * c["cols"], False)
+            elif u == "C5index":
+                continue
+            else:  # one C5 layer, now in the reused buffer
+                li = u[1]
+                mats, base, tasks = hw["C5"][li], 0, []
+                for m in mats:
+                    tasks += _lz4_block_tasks(m, base)
+                    base += m["rows"] * m["cols"]
+                got = host_bits(dw.c5_out[:base])
+                res = run(ex, tasks, got)
+                prev = verdict.get("C5")
+                if res is not None and isinstance(prev, tuple):
+                    res = (prev[0] + res[0], prev[1] + res[1], max(prev[2], res[2]))
+                verdict["C5"] = res if res is not None else None
+                if li == len(hw["C5"]) - 1 or res is None:
+                    total = sum(m["rows"] * m["cols"] for ms in hw["C5"] for m in ms)
+                    record(f"C5 ({len(hw['C5'])} layers)", verdict.pop("C5"), total, False)
+                    if res is None:
+                        break
+    torch.cuda.synchronize()
+    st = int(dw.status.item())
+    if st != 0:
+        verdict["status"] = f"decoder status {st}"
+        ok = False
+    return verdict, ok
 
 
 def cpu_model() -> str:
@@ -589,13 +774,14 @@ def read_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def workload_config(hw, layers, only=("C1", "C2", "C3", "C4", "C5")):
+def workload_config(hw, layers, only=("C1", "C2", "C3", "C4", "C4u", "C5")):
     c5_codes = sum(m["rows"] * m["cols"] for mats in hw.get("C5", []) for m in mats)
     parts = {
         "C1": "C1 INT4 1M codes G256",
         "C2": "C2 INT8 8192x8192 per-row",
         "C3": "C3 zero-run 8x2048x11008",
         "C4": "C4 LZ4+INT4 4096x14336 G128",
+        "C4u": "C4u INT4 4096x14336 G128 (C4's matrix uncompressed)",
         "C5": f"C5 {layers}-layer Llama-2-70B-shaped LZ4+INT4 G128 sweep (one reused layer buffer)",
     }
     return {
@@ -720,6 +906,137 @@ def value_dict_timing(peak: float, reps: int = 30, warmup: int = 3):
             "hbm_frac_of_8TBps": (rd + wr) / med / 1e9 / NOMINAL_HBM_GBS}
 
 
+def read_tflops_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured (cuBLAS bf16 burst; fp16 runs at the same tensor rate)"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def gemm_timing(hbm_peak: float, reps: int = 10, warmup: int = 3,
+                shapes=(("q/o", 8192, 8192), ("k/v", 8192, 1024), ("gate/up", 8192, 28672), ("down", 28672, 8192)),
+                batch=(1, 16, 128, 4096)):
+    """Fused INT4 decode -> GEMM (lt_int4_gemm) on the C5 weight shapes
+    ([K, N] = [in, out], C4's code law, group 128) against decode-then-
+    cuBLAS (lt_dequant_int4 into an fp16 buffer, then torch.matmul). Device
+    time per call by CUDA events, median of `reps`, a 256 MB L2-flushing
+    write before each call (not timed). Roofline: HBM bytes (x + packed
+    codes + scales + zero points + out) against the measured copy peak, and
+    2 M N K flops against the measured dense 16-bit tensor peak; the bound
+    is whichever time is larger."""
+    import numpy as np
+    import torch
+
+    from weight_dequantization_b200 import lt_decode as L
+    from weight_dequantization_b200.synth import fp16_uniform, int4_gauss_groups_packed, u8_uniform
+
+    tpeak, tkind = read_tflops_peak()
+    s = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def timed(fn):
+        ts = []
+        for r in range(warmup + reps):
+            flush.fill_(r & 0xFF)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            fn()
+            e1.record(s)
+            torch.cuda.synchronize()
+            if r >= warmup:
+                ts.append(e0.elapsed_time(e1) / 1e3)
+        return statistics.median(ts)
+
+    rows = []
+    for name, K, N in shapes:
+        G = 128
+        packed = torch.from_numpy(int4_gauss_groups_packed(11, K * N)).cuda()
+        scales = torch.from_numpy(fp16_uniform(11, K * N // G, 0.001, 0.1, stream=1).view(np.int16)).cuda()
+        zeros = torch.from_numpy(u8_uniform(11, K * N // G, 0, 15, stream=2)).cuda()
+        wbuf = torch.empty(K * N, dtype=torch.float16, device="cuda")
+        for M in batch:
+            x = torch.from_numpy(fp16_uniform(12, M * K, -1.0, 1.0, stream=7).view(np.int16)).cuda()
+            x16 = x.view(torch.float16).view(M, K)
+            out = torch.empty(M * N, dtype=torch.float16, device="cuda")
+            wsb = L.lt_int4_gemm_workspace_bytes(M, N, K)
+            ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
+            st = torch.zeros(1, dtype=torch.int32, device="cuda")
+            t_fused = timed(lambda: L.lt_int4_gemm(x, M, K, packed, scales, zeros, N, G, out, ws, st, s))
+            out_ref = torch.empty(M, N, dtype=torch.float16, device="cuda")
+
+            def dec_then_mm():
+                L.lt_dequant_int4(packed, scales, zeros, K, N, G, wbuf, s)
+                torch.matmul(x16, wbuf.view(K, N), out=out_ref)
+
+            t_base = timed(dec_then_mm)
+            t_mm = timed(lambda: torch.matmul(x16, wbuf.view(K, N), out=out_ref))
+            torch.cuda.synchronize()
+            if int(st.item()) != 0:
+                raise RuntimeError(f"lt_int4_gemm reported status {int(st.item())}")
+            diff = (out.view(M, N).float() - out_ref.float()).abs()
+            scale = out_ref.float().abs().max().item()
+            byts = 2 * M * K + K * N // 2 + 3 * K * N // G + 2 * M * N
+            flops = 2.0 * M * N * K
+            t_hbm, t_tc = byts / (hbm_peak * 1e9), flops / (tpeak * 1e12)
+            rows.append({"shape": name, "M": M, "K": K, "N": N, "us_fused": t_fused * 1e6,
+                         "us_decode_then_cublas": t_base * 1e6, "us_cublas_alone": t_mm * 1e6,
+                         "speedup_vs_decode_then_cublas": t_base / t_fused,
+                         "TFLOPs_fused": flops / t_fused / 1e12, "GBps_fused": byts / t_fused / 1e9,
+                         "bound": "tensor" if t_tc > t_hbm else "hbm",
+                         "roofline_frac": max(t_hbm, t_tc) / t_fused, "splits_workspace_bytes": wsb,
+                         "max_abs_diff_vs_cublas": diff.max().item(), "max_abs_out": scale})
+            del x, out, out_ref, ws
+        del packed, scales, zeros, wbuf
+    del flush
+    return {"label": "fused INT4 decode -> tcgen05 GEMM (lt_int4_gemm) vs lt_dequant_int4 + torch.matmul (cuBLAS) "
+                     "on the C5 weight shapes; L2 flushed before each call; median of %d" % reps,
+            "tensor_peak_TFLOPs": tpeak, "tensor_peak_kind": tkind, "hbm_peak_GBps": hbm_peak, "rows": rows}
+
+
+def stream_api_timing(hw, reps: int = 3):
+    """The streaming API (LayerStreamer) over the C5 layers against
+    sequential loading: streamed = each layer's host-to-device copy overlaps
+    the previous layer's decode; sequential = each layer copied, then
+    decoded, one after the other on one stream. Device time by CUDA events,
+    median of `reps` runs each, inputs in pinned host memory."""
+    import torch
+
+    from weight_dequantization_b200.stream import LayerStreamer
+
+    st = LayerStreamer(hw["C5"])
+    s = torch.cuda.current_stream()
+
+    def timed(fn):
+        ts = []
+        for r in range(reps + 1):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(s)
+            fn()
+            e1.record(s)
+            torch.cuda.synchronize()
+            if r:
+                ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    t_stream = timed(lambda: st.run(stream=s))
+    t_seq = timed(lambda: st.run_sequential(stream=s))
+    status = st.status()
+    h2d = sum(nb for _, nb, _ in st.layers)
+    dec = sum(2 * m["rows"] * m["cols"] for mats in hw["C5"] for m in mats)
+    res = {"label": f"LayerStreamer over {len(hw['C5'])} C5 layers from pinned host memory (two device slots, one "
+                    f"reused output buffer) vs sequential copy-then-decode per layer; median of {reps} runs",
+           "streamed_ms": t_stream, "sequential_ms": t_seq, "speedup": t_seq / t_stream,
+           "h2d_bytes": h2d, "decoded_GBps_streamed": dec / t_stream / 1e6,
+           "h2d_GBps_streamed": h2d / t_stream / 1e6, "status": status}
+    del st
+    return res
+
+
 def run_lt(args, rank, world, local):
     import torch
 
@@ -741,6 +1058,22 @@ def run_lt(args, rank, world, local):
     torch.cuda.synchronize()
     if int(dw.status.item()) != 0:
         raise RuntimeError(f"decode reported status {int(dw.status.item())} on the benchmark input")
+
+    # parity gate: one more step, every output compared with the oracle; a
+    # mismatch means no bench value
+    if args.no_parity:
+        parity, parity_ok = "not checked (--no-parity)", True
+    else:
+        t_par = time.perf_counter()
+        parity, parity_ok = parity_pass(dw, hw)
+        parity["seconds"] = round(time.perf_counter() - t_par, 1)
+        parity["how"] = ("one step's calls in order, each output read back and compared element by element with "
+                         "the oracle (all host cores); dequantized outputs within 1 binary16 ulp, zero-run bit for bit")
+    if not parity_ok:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": None, "unit": "GB/s", "n_gpus": world, "impl": "lt",
+                              "parity": parity, "error": "parity failed: no bench value"}), flush=True)
+        raise SystemExit(1)
 
     # timed region: K steps, device time by CUDA events on the launching stream
     clocks = ClockSampler(gpu_id_for(local))
@@ -767,7 +1100,7 @@ def run_lt(args, rank, world, local):
     # per codec (device time of the launches, summed over steps): events are
     # recorded at the step start and after every launch, in launch order
     K = args.steps
-    order = [c for c in ("C1", "C2", "C3", "C4") if c in hw] + ["C5"] * ((1 + len(dw.c5)) if dw.c5 else 0)
+    order = [c for c in STEP_CODECS if c in hw] + ["C5"] * ((1 + len(dw.c5)) if dw.c5 else 0)
     t_c = {c: 0.0 for c in alg}
     per_step = {c: [] for c in alg}  # device ms of the codec's launches in each step
     layer_t = []
@@ -864,6 +1197,8 @@ def run_lt(args, rank, world, local):
             cpu_thr = cpu_baseline_threads(hw, cpu["frac"])
         c1g = c1_graph_steady_state(hw, peak) if "C1" in hw else None
         vd = value_dict_timing(peak) if "V" in only else None
+        sapi = stream_api_timing(hw) if ("S" in only and hw.get("C5")) else None
+        gemm = gemm_timing(peak) if "G" in only else None
         if vd is not None and world == 1 and not args.no_cpu_baseline:
             vd["cpu_baseline"] = cpu_baseline_value_dict()
         result = {
@@ -874,6 +1209,7 @@ def run_lt(args, rank, world, local):
             "gpu_launches": nlaunch * K, "clocks": {"sm_mhz": ck["sm_mhz"], "sm_max_mhz": ck["sm_max_mhz"],
                                                      "reasons": ck["reasons"], "samples": ck["samples"]},
             "per_codec": per_codec, "c1_graph": c1g, "value_dict": vd, "cpu_baseline_threads": cpu_thr,
+            "parity": parity, "stream_api": sapi, "gemm": gemm,
             "impl": "lt",
         }
     if dist is not None:

@@ -124,6 +124,24 @@ class LayerStreamer:
                 with torch.cuda.stream(s):
                     consume(i, views)
 
+    def run_sequential(self, consume=None, stream=None):
+        """Sequential loading, the baseline the roadmap's streaming test
+        compares against: each layer is copied into slot 0 and then decoded,
+        both on the compute stream, so no copy overlaps a decode. Same
+        results as ``run``."""
+        torch = self.torch
+        s = stream if stream is not None else torch.cuda.current_stream()
+        slot = self.slots[0]
+        for i, (host, nbytes, _) in enumerate(self.layers):
+            with torch.cuda.stream(s):
+                if nbytes:
+                    slot[:nbytes].copy_(host[:nbytes], non_blocking=True)
+            descs, views = self._descs(i, slot)
+            L.lt_lz4_int4_decode_batch(descs, self.ws, self.d_status, s)
+            if consume is not None:
+                with torch.cuda.stream(s):
+                    consume(i, views)
+
     def status(self) -> int:
         """The first error status of the decodes so far (0: none); waits for
         the device."""
