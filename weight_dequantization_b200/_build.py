@@ -17,7 +17,8 @@ SYNTH_LIB = os.path.join(PKG, "synth", "liblt_synth.so")
 
 # CUDA sources, plus the host-only container header code (lt_hct.cpp, built
 # by nvcc's host compiler into the same library)
-CUDA_SOURCES = ["lt_abi.cu", "lt_dequant.cu", "lt_dict.cu", "lt_zrle.cu", "lt_lz4.cu", "lt_xxh3.cu", "lt_hct.cpp"]
+CUDA_SOURCES = ["lt_abi.cu", "lt_dequant.cu", "lt_dict.cu", "lt_zrle.cu", "lt_lz4.cu", "lt_xxh3.cu", "lt_gemm.cu",
+                "lt_hct.cpp"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -33,7 +33,8 @@ LT_LZ4_BATCH_MAX = 64
 EXPORTED = (
     "lt_dequant_int4", "lt_dequant_int8", "lt_value_dict_decode", "lt_zrle_decode", "lt_lz4_int4_decode",
     "lt_lz4_int4_decode_batch", "lt_lz4_index_batch", "lt_lz4_int4_expand_batch", "lt_lz4_decode",
-    "lt_lz4_workspace_bytes", "lt_lz4_int4_decode_noalloc", "lt_xxh3_blocks",
+    "lt_lz4_workspace_bytes", "lt_lz4_int4_decode_noalloc", "lt_xxh3_blocks", "lt_int4_gemm",
+    "lt_int4_gemm_workspace_bytes",
     "lt_hct2_layout", "lt_hct2_read_header", "lt_hct2_write_header",
     "lt_status_string", "lt_abi_version",
 )
@@ -103,6 +104,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.lt_hct2_write_header.argtypes = [ctypes.POINTER(LtHct2Header), ctypes.c_char_p]
     for f in ("lt_hct2_layout", "lt_hct2_read_header", "lt_hct2_write_header"):
         getattr(lib, f).restype = ctypes.c_int
+    lib.lt_int4_gemm.argtypes = [P, I64, I64, P, P, P, I64, I32, P, P, U64, P, P]
+    lib.lt_int4_gemm.restype = ctypes.c_int
+    lib.lt_int4_gemm_workspace_bytes.argtypes = [I64, I64, I64]
+    lib.lt_int4_gemm_workspace_bytes.restype = U64
     lib.lt_lz4_workspace_bytes.argtypes = [I64]
     lib.lt_lz4_workspace_bytes.restype = U64
     for f in ("lt_dequant_int4", "lt_dequant_int8", "lt_value_dict_decode", "lt_zrle_decode", "lt_lz4_int4_decode",
@@ -269,6 +274,22 @@ def lt_lz4_int4_decode_noalloc(comp, comp_bytes: int, block_offsets, block_bytes
                                                      _ptr(scales), _ptr(zeros), rows, cols, group_size, _ptr(out),
                                                      _ptr(d_status), _stream(stream, out)),
            "lt_lz4_int4_decode_noalloc")
+
+
+def lt_int4_gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(load_library().lt_int4_gemm_workspace_bytes(int(M), int(N), int(K)))
+
+
+def lt_int4_gemm(x, M: int, K: int, packed, scales, zeros, N: int, group_size: int, out, workspace=None,
+                 d_status=None, stream=None) -> None:
+    """out[M, N] = x[M, K] @ W[K, N], W the INT4 dequant of ``packed`` /
+    ``scales`` / ``zeros`` (lt_dequant_int4's layout with rows = K, cols =
+    N), decoded tile by tile into shared memory and multiplied on the tensor
+    cores. ``workspace``: optional CUDA tensor (or (address, bytes)) of at
+    least lt_int4_gemm_workspace_bytes(M, N, K) bytes for splitting K."""
+    wp, wb = _ws(workspace)
+    _check(load_library().lt_int4_gemm(_ptr(x), M, K, _ptr(packed), _ptr(scales), _ptr(zeros), N, group_size,
+                                       _ptr(out), wp, wb, _ptr(d_status), _stream(stream, out)), "lt_int4_gemm")
 
 
 # HCT v2 container header: host functions (host memory, no device)
