@@ -996,6 +996,68 @@ def gemm_timing(hbm_peak: float, reps: int = 10, warmup: int = 3,
             "tensor_peak_TFLOPs": tpeak, "tensor_peak_kind": tkind, "hbm_peak_GBps": hbm_peak, "rows": rows}
 
 
+def checksum_timing(dw, hw, peak: float, reps: int = 20, warmup: int = 3):
+    """Per-block XXH3-64 on C4's compressed stream (448 blocks): the
+    standalone verifier (lt_xxh3_blocks, one warp per block) and the decode
+    with the check fused in (lt_lz4_int4_decode_checked) against the plain
+    fused decode. Device time by CUDA events, median of `reps`, a 256 MB
+    L2-flushing write before each call (not timed)."""
+    import numpy as np
+    import torch
+
+    from weight_dequantization_b200 import lt_decode as L
+
+    c4 = hw["C4"]
+    nb = len(c4["offsets"]) - 1
+    secret = torch.from_numpy(np.random.default_rng(99).integers(0, 256, 192, dtype=np.uint8)).cuda()
+    hashes = torch.zeros(nb, dtype=torch.int64, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    first = torch.full((1,), -1, dtype=torch.int64, device="cuda")
+    s = torch.cuda.current_stream()
+    comp_bytes = int(c4["comp"].size)
+    L.lt_xxh3_blocks(dw.c4["comp"], comp_bytes, dw.c4["offsets"], nb, secret, 192, hashes, None, st, first, s)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def timed(fn):
+        ts = []
+        for r in range(warmup + reps):
+            flush.fill_(r & 0xFF)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            fn()
+            e1.record(s)
+            torch.cuda.synchronize()
+            if r >= warmup:
+                ts.append(e0.elapsed_time(e1) / 1e3)
+        return statistics.median(ts)
+
+    def plain():
+        L.lt_lz4_int4_decode(dw.c4["comp"], comp_bytes, dw.c4["offsets"], c4["block_bytes"], dw.c4["scales"],
+                             dw.c4["zeros"], c4["rows"], c4["cols"], c4["group_size"], dw.c4_out, dw.ws, st, s)
+
+    def checked():
+        L.lt_lz4_int4_decode_checked(dw.c4["comp"], comp_bytes, dw.c4["offsets"], c4["block_bytes"],
+                                     dw.c4["scales"], dw.c4["zeros"], c4["rows"], c4["cols"], c4["group_size"],
+                                     dw.c4_out, secret, 192, hashes, dw.ws, st, first, s)
+
+    t_hash = timed(lambda: L.lt_xxh3_blocks(dw.c4["comp"], comp_bytes, dw.c4["offsets"], nb, secret, 192, None,
+                                            hashes, st, first, s))
+    t_plain = timed(plain)
+    t_checked = timed(checked)
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"checksum leg: status {int(st.item())}")
+    hb = comp_bytes + 8 * (nb + 1) + 8 * nb
+    del flush
+    return {"label": f"XXH3-64 per LZ4 block of C4 ({nb} blocks, {comp_bytes} compressed bytes, 192-byte secret); "
+                     f"L2 flushed before each of {reps} calls",
+            "kernel": "k_xxh3_blocks (warp per block)", "us_verify": t_hash * 1e6, "verify_GBps": hb / t_hash / 1e9,
+            "verify_hbm_frac_of_measured": hb / t_hash / 1e9 / peak,
+            "us_decode_plain": t_plain * 1e6, "us_decode_checked": t_checked * 1e6,
+            "checked_overhead": t_checked / t_plain - 1.0}
+
+
 def stream_api_timing(hw, reps: int = 3):
     """The streaming API (LayerStreamer) over the C5 layers against
     sequential loading: streamed = each layer's host-to-device copy overlaps
@@ -1199,6 +1261,7 @@ def run_lt(args, rank, world, local):
         vd = value_dict_timing(peak) if "V" in only else None
         sapi = stream_api_timing(hw) if ("S" in only and hw.get("C5")) else None
         gemm = gemm_timing(peak) if "G" in only else None
+        csum = checksum_timing(dw, hw, peak) if "C4" in hw else None
         if vd is not None and world == 1 and not args.no_cpu_baseline:
             vd["cpu_baseline"] = cpu_baseline_value_dict()
         result = {
@@ -1209,7 +1272,7 @@ def run_lt(args, rank, world, local):
             "gpu_launches": nlaunch * K, "clocks": {"sm_mhz": ck["sm_mhz"], "sm_max_mhz": ck["sm_max_mhz"],
                                                      "reasons": ck["reasons"], "samples": ck["samples"]},
             "per_codec": per_codec, "c1_graph": c1g, "value_dict": vd, "cpu_baseline_threads": cpu_thr,
-            "parity": parity, "stream_api": sapi, "gemm": gemm,
+            "parity": parity, "stream_api": sapi, "gemm": gemm, "checksum": csum,
             "impl": "lt",
         }
     if dist is not None:

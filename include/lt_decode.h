@@ -286,6 +286,32 @@ lt_status lt_lz4_int4_decode(const uint8_t *comp, uint64_t comp_bytes, const uin
                              uint64_t workspace_bytes, int32_t *d_status, lt_stream_t stream);
 
 /*
+ * The fused decode of lt_lz4_int4_decode with each compressed block checked
+ * first ("GPU Compression Pipeline - TDD Roadmap", Phase 6.1 HCT Format V2:
+ * XXH3 checksums; a flipped byte is reported as a checksum mismatch).
+ *
+ * Before decoding block b, the kernel computes the XXH3-64 (seed 0, the
+ * given secret, as lt_xxh3_blocks) of comp[block_offsets[b],
+ * block_offsets[b + 1]) and compares it with expected_hashes[b]. A block
+ * that differs is not decoded (its output is left unspecified), sets
+ * LT_ERR_CHECKSUM in *d_status (which then takes precedence over any other
+ * error of that block) and lowers *d_first_bad (caller-initialised, e.g. to
+ * UINT64_MAX; may be NULL) to b. Other blocks decode as in
+ * lt_lz4_int4_decode. The hash is computed while the block is read for
+ * decoding (one warp of the expanding CTA), so the compressed stream is not
+ * read by a separate pass.
+ *   secret, secret_len  device, secret_len >= 136; expected_hashes: n_blocks
+ *                       uint64 (device, 8-byte aligned). All other arguments
+ *                       as lt_lz4_int4_decode.
+ */
+lt_status lt_lz4_int4_decode_checked(const uint8_t *comp, uint64_t comp_bytes, const uint64_t *block_offsets,
+                                     int32_t block_bytes, const lt_half *scales, const uint8_t *zeros, int64_t rows,
+                                     int64_t cols, int32_t group_size, lt_half *out, void *workspace,
+                                     uint64_t workspace_bytes, const uint8_t *secret, int32_t secret_len,
+                                     const uint64_t *expected_hashes, int32_t *d_status, uint64_t *d_first_bad,
+                                     lt_stream_t stream);
+
+/*
  * Several fused LZ4 -> INT4 decodes in one launch (the weight matrices of a
  * transformer layer decoded into one reused buffer). Each descriptor has
  * the meaning of the lt_lz4_int4_decode arguments of the same name. The

@@ -142,9 +142,15 @@ def test_container_decodes_like_the_oracle():
     want, st = oracle.lz4_int4_decode(comp, offs, bs, scales, zeros, rows, cols, G)
     assert st == 0
     assert np.array_equal(_f16_bits(hct.decode(c)), want)
+    # a damaged payload byte: the checked decode names its block
     bad = bytearray(c)
     bad[-1] ^= 0xFF
-    with pytest.raises(hct.HctError):
+    with pytest.raises(hct.HctError, match=f"checksum mismatch in block {len(blocks) - 1}$"):
+        hct.decode(bytes(bad))
+    # a damaged byte of the secret: the metadata hash no longer matches
+    bad = bytearray(c)
+    bad[100] ^= 0xFF
+    with pytest.raises(hct.HctError, match="metadata checksum mismatch"):
         hct.decode(bytes(bad))
 
 
@@ -174,3 +180,47 @@ def test_uncompressed_and_raw_containers_decode_like_the_oracle():
     blocks = [comp[offs[b]:offs[b + 1]].tobytes() for b in range(len(offs) - 1)]
     c = hct.write(blocks, 65536, 3, 32768, hct.QUANT_NONE, 0, None, None, secret)
     assert np.array_equal(_f16_bits(hct.decode(c)), x)
+
+
+# --------------------------------------------------------------------------- checked decode
+
+def _checked(comp, offs, m, secret, expected, ws=True, shift=0):
+    n = m["rows"] * m["cols"]
+    out = torch.full((n,), float("nan"), dtype=torch.float16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    first = torch.from_numpy(np.array([NONE]).view(np.int64)).cuda()
+    buf = dev(np.concatenate([np.zeros(shift, np.uint8), comp]))[shift:]
+    nb = offs.size - 1
+    work = torch.empty(L.lt_lz4_workspace_bytes(nb), dtype=torch.uint8, device="cuda") if ws else None
+    L.lt_lz4_int4_decode_checked(buf, comp.size, dev(offs), 65536, dev(m["scales"]), dev(m["zeros"]), m["rows"],
+                                 m["cols"], m["group_size"], out, dev(secret), secret.size, dev(expected), work,
+                                 status, first)
+    torch.cuda.synchronize()
+    bits = out.cpu().view(torch.int16).numpy().view(np.uint16)
+    return bits, int(status.item()), int(first.cpu().numpy().view(np.uint64)[0])
+
+
+@pytest.mark.parametrize("ws,shift", [(True, 0), (False, 0), (True, 5)])
+def test_checked_decode_matches_the_oracle_and_stops_a_damaged_block(ws, shift):
+    from weight_dequantization_b200.synth import workloads as W
+    m = W.c4_lz4_int4(scale=16 * 8 / 4096, seed=21)  # 16 blocks of 64 KB, C4's law
+    comp, offs = m["comp"], m["offsets"]
+    secret = RNG.integers(0, 256, 192, dtype=np.uint8)
+    stored = oracle_hashes(comp, offs, secret)
+    want, st = oracle.lz4_int4_decode(comp, offs, 65536, m["scales"], m["zeros"], m["rows"], m["cols"],
+                                      m["group_size"])
+    assert st == 0
+    got, st, first = _checked(comp, offs, m, secret, stored, ws, shift)
+    assert (st, first) == (0, int(NONE))
+    assert np.array_equal(got, want)
+    # one flipped byte in block 5: reported as a checksum mismatch at block 5
+    # (not as whatever stream error the damage causes); every other block
+    # still decodes exactly
+    bad = comp.copy()
+    bad[int(offs[5]) + 7] ^= 0xFF
+    got, st, first = _checked(bad, offs, m, secret, stored, ws, shift)
+    assert (st, first) == (L.LT_ERR_CHECKSUM, 5)
+    per = 2 * 65536
+    keep = np.ones(want.size, bool)
+    keep[5 * per:6 * per] = False
+    assert np.array_equal(got[keep], want[keep])

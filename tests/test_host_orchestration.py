@@ -83,6 +83,25 @@ def _fake_lz4_int4(comp, comp_bytes, offs, bs, scales, zeros, rows, cols, G, out
         st[0] = s
 
 
+def _fake_lz4_checked(comp, comp_bytes, offs, bs, scales, zeros, rows, cols, G, out, secret, secret_len, expected,
+                      ws=None, st=None, first=None, stream=None):
+    assert secret_len >= 136 and expected is not None and expected.data_ptr() % 8 == 0
+    nb = ((rows * cols + 1) // 2 + bs - 1) // bs
+    d = _u8(comp)[:comp_bytes]
+    o = offs.numpy().view(np.uint64)[:nb + 1]
+    sec = _u8(secret)[:secret_len]
+    bad = [b for b in range(nb) if oracle.xxh3_64(d[int(o[b]):int(o[b + 1])], sec) !=
+           int(expected.numpy().view(np.uint64)[b])]
+    if bad:
+        if st is not None and st[0] == 0:
+            st[0] = 8
+        if first is not None:
+            fb = first.numpy().view(np.uint64)
+            fb[0] = min(int(fb[0]), bad[0])
+        return
+    _fake_lz4_int4(comp, comp_bytes, offs, bs, scales, zeros, rows, cols, G, out, ws, st, stream)
+
+
 def _fake_lz4(comp, comp_bytes, offs, bs, out, out_bytes, ws=None, st=None, stream=None):
     nb = (out_bytes + bs - 1) // bs
     w, s = oracle.lz4_decode_blocks(_u8(comp)[:comp_bytes], offs.numpy().view(np.uint64)[:nb + 1], bs, out_bytes)
@@ -156,6 +175,7 @@ def cpu_device(monkeypatch):
     monkeypatch.setattr(torch.cuda, "stream", lambda s: contextlib.nullcontext())
     monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
     for name, fake in (("lt_xxh3_blocks", _fake_xxh3), ("lt_lz4_int4_decode", _fake_lz4_int4),
+                       ("lt_lz4_int4_decode_checked", _fake_lz4_checked),
                        ("lt_lz4_decode", _fake_lz4), ("lt_dequant_int4", _fake_int4),
                        ("lt_dequant_int8", _fake_int8), ("lt_lz4_int4_decode_batch", _fake_batch)):
         monkeypatch.setattr(L, name, fake)

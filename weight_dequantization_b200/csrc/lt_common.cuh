@@ -39,6 +39,28 @@ __device__ __forceinline__ uint4 ld_stream_u128(const void *p) {
                : "l"(p));
   return v;
 }
+// 8 little-endian bytes at p, any alignment, inside a caller's buffer
+// [lo, hi): two aligned 8-byte loads when both aligned words lie inside the
+// buffer, byte loads at its edges (never a byte outside [lo, hi)).
+struct GlobalBytes {
+  const uint8_t *lo, *hi;
+  __device__ __forceinline__ uint64_t rd64(const uint8_t *p) const {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p) & ~uintptr_t(7);
+    const uint32_t sh = (uint32_t)(reinterpret_cast<uintptr_t>(p) & 7) * 8;
+    const uint64_t *w = reinterpret_cast<const uint64_t *>(a);
+    if (sh == 0) return __ldg(reinterpret_cast<const unsigned long long *>(w));
+    if (a >= reinterpret_cast<uintptr_t>(lo) && a + 16 <= reinterpret_cast<uintptr_t>(hi)) {
+      const uint64_t x = __ldg(reinterpret_cast<const unsigned long long *>(w));
+      const uint64_t y = __ldg(reinterpret_cast<const unsigned long long *>(w + 1));
+      return (x >> sh) | (y << (64 - sh));
+    }
+    uint64_t v = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v |= (uint64_t)__ldg(p + i) << (8 * i);
+    return v;
+  }
+};
+
 // Output written once and not read back by this kernel.
 __device__ __forceinline__ void st_u128(void *p, uint4 v) {
   asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)

@@ -30,6 +30,7 @@
 #include <mutex>
 
 #include "lt_common.cuh"
+#include "lt_xxh3.cuh"
 
 namespace lt {
 namespace {
@@ -72,6 +73,12 @@ struct Batch {
   int32_t n_jobs;
   int32_t max_block_bytes;
   int64_t total_blocks;
+  // checked decode (one job): each compressed block's XXH3-64 with this
+  // secret must equal expected[block] before the block is decoded
+  const uint8_t *secret;
+  uint32_t secret_len;
+  const uint64_t *expected;
+  unsigned long long *first_bad;
 };
 
 __device__ __forceinline__ const Job &find_job(const Batch &batch, int64_t blk, int64_t &b) {
@@ -750,7 +757,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
   extern __shared__ uint4 smem_u4[];
   uint8_t *win = reinterpret_cast<uint8_t *>(smem_u4) + kPad;
   __shared__ Seqs S;
-  __shared__ uint32_t s_n, s_st, s_lmax;
+  __shared__ uint32_t s_n, s_st, s_lmax, s_badsum;
   const uint32_t wcap = win_cap(batch.max_block_bytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -759,6 +766,33 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
     const Job &jb = find_job(batch, blk, b);
     const int64_t d0 = b * (int64_t)jb.block_bytes;
     const uint32_t olen = block_len(jb, b);
+    if (batch.secret != nullptr && warp == 0) {
+      // checked decode: the block's checksum first, so that a damaged block
+      // is reported as a checksum mismatch (and not decoded) whatever else is
+      // wrong with it
+      const uint64_t c0 = jb.offsets[b], c1 = jb.offsets[b + 1];
+      bool bad = false;
+      if (c0 <= c1 && c1 <= jb.comp_bytes) {
+        const uint64_t len = c1 - c0;
+        const uint8_t *in = jb.comp + c0;
+        const GlobalBytes din{jb.comp, jb.comp + jb.comp_bytes}, dsec{batch.secret, batch.secret + batch.secret_len};
+        uint64_t h;
+        if (len > 240)
+          h = xxh3::hash64_long_warp([&](uint64_t off) { return din.rd64(in + off); },
+                                     [&](uint64_t off) { return dsec.rd64(batch.secret + off); }, len,
+                                     batch.secret_len, lane);
+        else
+          h = lane == 0 ? xxh3::hash64(in, len, batch.secret, batch.secret_len) : 0;
+        bad = h != batch.expected[blk];
+      }  // (an offset pair outside the stream is reported by the decode below)
+      if (lane == 0) {
+        s_badsum = bad ? 1u : 0u;
+        if (bad) {
+          report(d_status, LT_ERR_CHECKSUM);
+          if (batch.first_bad) atomicMin(batch.first_bad, (unsigned long long)blk);
+        }
+      }
+    }
     if (threadIdx.x == 0) {
       const uint4 h = hdr ? hdr[blk] : make_uint4(0u, kNoIndex, 0u, 0u);
       s_n = h.x;
@@ -769,6 +803,10 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
     __syncthreads();
     const uint32_t n = s_n, lmax = s_lmax;
     uint32_t st = s_st;
+    if (batch.secret != nullptr && s_badsum) {  // checksum mismatch: not decoded (output unspecified)
+      __syncthreads();
+      continue;
+    }
     if (st != 0 && st != kOverflow && st != kNoIndex && st != kNoInPlace) {
       // the parse found a malformed block: report it; its output stays unwritten
       if (threadIdx.x == 0) report(d_status, (int32_t)st);
@@ -994,6 +1032,26 @@ LT_API lt_status lt_lz4_int4_decode_batch(const lt_lz4_int4_desc *descs, int32_t
                                 d.rows, d.cols, d.group_size, d.out);
     if (s != LT_OK) return s;
   }
+  return launch(batch, true, workspace, workspace_bytes, d_status, (cudaStream_t)stream);
+}
+
+LT_API lt_status lt_lz4_int4_decode_checked(const uint8_t *comp, uint64_t comp_bytes, const uint64_t *block_offsets,
+                                            int32_t block_bytes, const lt_half *scales, const uint8_t *zeros,
+                                            int64_t rows, int64_t cols, int32_t group_size, lt_half *out,
+                                            void *workspace, uint64_t workspace_bytes, const uint8_t *secret,
+                                            int32_t secret_len, const uint64_t *expected_hashes, int32_t *d_status,
+                                            uint64_t *d_first_bad, lt_stream_t stream) {
+  if (!aligned(d_status, 4) || !aligned(workspace, 16) || !aligned(d_first_bad, 8)) return LT_ERR_MISALIGNED;
+  if (!secret || secret_len < (int32_t)xxh3::kSecretMin || !expected_hashes) return LT_ERR_INVALID_ARG;
+  if (!aligned(expected_hashes, 8)) return LT_ERR_MISALIGNED;
+  Batch batch = empty_batch();
+  lt_status s = add_fused_job(batch, comp, comp_bytes, block_offsets, block_bytes, scales, zeros, rows, cols,
+                              group_size, out);
+  if (s != LT_OK) return s;
+  batch.secret = secret;
+  batch.secret_len = (uint32_t)secret_len;
+  batch.expected = expected_hashes;
+  batch.first_bad = reinterpret_cast<unsigned long long *>(d_first_bad);
   return launch(batch, true, workspace, workspace_bytes, d_status, (cudaStream_t)stream);
 }
 

@@ -153,5 +153,61 @@ LT_HD uint64_t hash64(const uint8_t *in, uint64_t len, const uint8_t *sec, uint6
   return avalanche3(h);
 }
 
+#ifdef __CUDACC__
+// ---------------------------------------------------------------------------
+// The long class (len > 240) computed by one warp. Within one scramble
+// interval the accumulator updates of the stripes are plain sums modulo
+// 2^64, so they can be split among lanes and added up: lane l takes the
+// 8-byte word i = l % 8 of stripes l / 8, l / 8 + 4, ...; a butterfly over
+// the four lanes with the same i adds their terms; acc[i] takes its product
+// terms and the data terms of word i ^ 1 (one shuffle). The scramble, the
+// tail stripes, the last stripe and the merge then follow the sequential
+// definition above, each lane holding acc[l % 8]. `rd(off)` returns the 8
+// input bytes at offset off (little-endian, any alignment); `rk(off)` the 8
+// secret bytes at offset off. Every lane returns the hash.
+// ---------------------------------------------------------------------------
+template <typename RD, typename RK>
+__device__ __forceinline__ uint64_t hash64_long_warp(RD rd, RK rk, uint64_t len, uint64_t sec_len, int lane) {
+  const int i = lane & 7;
+  // the initial accumulators kP32_3, kP64_1, kP64_2, kP64_3, kP64_4, kP32_2, kP64_5, kP32_1, by i
+  uint64_t acc = (i & 4) ? ((i & 2) ? ((i & 1) ? kP32_1 : kP64_5) : ((i & 1) ? kP32_2 : kP64_4))
+                         : ((i & 2) ? ((i & 1) ? kP64_3 : kP64_2) : ((i & 1) ? kP64_1 : kP32_3));
+  const uint64_t per_block = (sec_len - 64) / 8;
+  const uint64_t block_len = 64 * per_block;
+  const uint64_t n_blocks = (len - 1) / block_len;
+  const uint64_t scr = rk(sec_len - 64 + 8 * (uint64_t)i);
+  // stripes [0, ns) starting at input offset base, stripe s keyed at secret offset key0 + 8 s
+  auto stripes = [&](uint64_t base, uint64_t ns, uint64_t key0) {
+    uint64_t m = 0, d = 0;
+    for (uint64_t st = (uint64_t)(lane >> 3); st < ns; st += 4) {
+      const uint64_t v = rd(base + 64 * st + 8 * (uint64_t)i);
+      const uint64_t k = v ^ rk(key0 + 8 * st + 8 * (uint64_t)i);
+      d += v;
+      m += (k & 0xFFFFFFFFull) * (k >> 32);
+    }
+    m += __shfl_xor_sync(0xFFFFFFFFu, m, 8);
+    m += __shfl_xor_sync(0xFFFFFFFFu, m, 16);
+    d += __shfl_xor_sync(0xFFFFFFFFu, d, 8);
+    d += __shfl_xor_sync(0xFFFFFFFFu, d, 16);
+    acc += m + __shfl_xor_sync(0xFFFFFFFFu, d, 1);
+  };
+  for (uint64_t b = 0; b < n_blocks; ++b) {
+    stripes(b * block_len, per_block, 0);
+    acc ^= acc >> 47;
+    acc ^= scr;
+    acc *= kP32_1;
+  }
+  stripes(n_blocks * block_len, ((len - 1) - block_len * n_blocks) / 64, 0);
+  stripes(len - 64, 1, sec_len - 64 - 7);
+  // merge: term j (lanes 0..3) from acc[2j] and acc[2j + 1]
+  const uint64_t a_even = __shfl_sync(0xFFFFFFFFu, acc, (2 * lane) & 7);
+  const uint64_t a_odd = __shfl_sync(0xFFFFFFFFu, acc, (2 * lane + 1) & 7);
+  uint64_t t = lane < 4 ? mul_fold(a_even ^ rk(11 + 16 * (uint64_t)lane), a_odd ^ rk(19 + 16 * (uint64_t)lane)) : 0;
+  t += __shfl_xor_sync(0xFFFFFFFFu, t, 1);
+  t += __shfl_xor_sync(0xFFFFFFFFu, t, 2);
+  return avalanche3(len * kP64_1 + __shfl_sync(0xFFFFFFFFu, t, 0));
+}
+#endif
+
 }  // namespace xxh3
 }  // namespace lt

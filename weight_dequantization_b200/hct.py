@@ -117,6 +117,21 @@ def write(blocks, block_size: int, rows: int, cols: int, quantization: int, grou
     return bytes(meta) + payload
 
 
+def _meta_ok(buf, h, sec, dev):
+    """The metadata hash (every byte before the payload, meta_hash read as
+    zero) checked on the device, and the block offsets' consistency."""
+    import torch
+
+    secret_dev = dev[HEADER_BYTES:HEADER_BYTES + h.secret_len]
+    meta = bytearray(bytes(buf[:sec["payload"]]))
+    meta[56:64] = bytes(8)
+    meta_dev = torch.frombuffer(meta, dtype=torch.uint8).cuda()
+    (mh,) = _device_hashes(meta_dev, len(meta), [0, len(meta)], secret_dev, h.secret_len)
+    offs = np.frombuffer(bytes(buf[sec["offsets"]:sec["offsets"] + 8 * (h.n_blocks + 1)]), np.uint64)
+    return (mh == h.meta_hash and offs[0] == 0 and offs[-1] == h.payload_bytes
+            and not np.any(np.diff(offs.astype(np.int64)) < 0))
+
+
 def verify(buf):
     """Check a container's checksums on the device (PyTorch's current
     stream). Returns (ok, first bad block or None, meta_ok)."""
@@ -125,17 +140,11 @@ def verify(buf):
     h = read_header(buf)
     sec = sections(h)
     dev = torch.frombuffer(bytearray(bytes(buf)), dtype=torch.uint8).cuda()
-    secret_dev = dev[HEADER_BYTES:HEADER_BYTES + h.secret_len]
-    meta = bytearray(bytes(buf[:sec["payload"]]))
-    meta[56:64] = bytes(8)
-    meta_dev = torch.frombuffer(meta, dtype=torch.uint8).cuda()
-    (mh,) = _device_hashes(meta_dev, len(meta), [0, len(meta)], secret_dev, h.secret_len)
-    meta_ok = mh == h.meta_hash
-    offs = np.frombuffer(bytes(buf[sec["offsets"]:sec["offsets"] + 8 * (h.n_blocks + 1)]), np.uint64)
-    if not meta_ok or offs[0] != 0 or offs[-1] != h.payload_bytes or np.any(np.diff(offs.astype(np.int64)) < 0):
+    if not _meta_ok(buf, h, sec, dev):
         return False, None, False
     if h.n_blocks == 0:
         return True, None, True
+    secret_dev = dev[HEADER_BYTES:HEADER_BYTES + h.secret_len]
     payload = dev[sec["payload"]:]
     stored = dev[sec["hashes"]:sec["hashes"] + 8 * h.n_blocks].view(torch.int64)
     offs_dev = dev[sec["offsets"]:sec["offsets"] + 8 * (h.n_blocks + 1)].view(torch.int64)
@@ -162,11 +171,15 @@ def decode(buf, check: bool = True):
     h = read_header(buf)
     if h.compression == COMPRESSION_LZ4 and h.quantization == QUANT_INT8:
         raise HctError("LZ4-compressed INT8 has no decoder")
-    if check:
+    sec = sections(h)
+    # LZ4 + INT4: the payload blocks are checked inside the decode itself
+    # (lt_lz4_int4_decode_checked: each block's hash while it is read for
+    # decoding); every other kind is verified first
+    fused_check = check and h.compression == COMPRESSION_LZ4 and h.quantization == QUANT_INT4
+    if check and not fused_check:
         ok, bad, meta_ok = verify(buf)
         if not ok:
             raise HctError("metadata checksum mismatch" if not meta_ok else f"checksum mismatch in block {bad}")
-    sec = sections(h)
     n = h.rows * h.cols
     # bytes the decoded stream must hold: packed INT4, INT8 or raw fp16
     need = {QUANT_INT4: (n + 1) // 2, QUANT_INT8: n, QUANT_NONE: 2 * n}[h.quantization]
@@ -176,6 +189,8 @@ def decode(buf, check: bool = True):
     elif h.payload_bytes < need:
         raise HctError(f"the payload holds {h.payload_bytes} bytes, the shape needs {need}")
     dev = torch.frombuffer(bytearray(bytes(buf)), dtype=torch.uint8).cuda()
+    if fused_check and not _meta_ok(buf, h, sec, dev):
+        raise HctError("metadata checksum mismatch")
     out = torch.empty((h.rows, h.cols), dtype=torch.float16, device="cuda")
     if n == 0:
         return out
@@ -184,10 +199,18 @@ def decode(buf, check: bool = True):
     scales = dev[sec["scales"]:sec["scales"] + 2 * h.n_groups].view(torch.float16)
     zeros = dev[sec["zeros"]:sec["zeros"] + h.n_groups] if h.quantization == QUANT_INT4 else None
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    first = None
     if h.compression == COMPRESSION_LZ4 and h.quantization == QUANT_INT4:
         ws = torch.empty(max(L.lt_lz4_workspace_bytes(h.n_blocks), 16), dtype=torch.uint8, device="cuda")
-        L.lt_lz4_int4_decode(payload, h.payload_bytes, offs, h.block_size, scales, zeros, h.rows, h.cols,
-                             h.group_size, out, ws, status)
+        if fused_check:
+            stored = dev[sec["hashes"]:sec["hashes"] + 8 * h.n_blocks].view(torch.int64)
+            first = torch.full((1,), -1, dtype=torch.int64, device="cuda")  # all ones: no block yet
+            L.lt_lz4_int4_decode_checked(payload, h.payload_bytes, offs, h.block_size, scales, zeros, h.rows, h.cols,
+                                         h.group_size, out, dev[HEADER_BYTES:HEADER_BYTES + h.secret_len],
+                                         h.secret_len, stored, ws, status, first)
+        else:
+            L.lt_lz4_int4_decode(payload, h.payload_bytes, offs, h.block_size, scales, zeros, h.rows, h.cols,
+                                 h.group_size, out, ws, status)
     elif h.compression == COMPRESSION_LZ4 and h.quantization == QUANT_NONE:
         ws = torch.empty(max(L.lt_lz4_workspace_bytes(h.n_blocks), 16), dtype=torch.uint8, device="cuda")
         L.lt_lz4_decode(payload, h.payload_bytes, offs, h.block_size, out.view(torch.uint8).view(-1), 2 * n, ws,
@@ -199,6 +222,8 @@ def decode(buf, check: bool = True):
     else:  # neither compressed nor quantized: the payload is the fp16 tensor
         out.view(torch.uint8).view(-1).copy_(payload[:2 * n])
     st = int(status.item())
+    if st == L.LT_ERR_CHECKSUM and first is not None:
+        raise HctError(f"checksum mismatch in block {int(first.item())}")
     if st != 0:
         raise HctError(L.status_string(st))
     return out

@@ -33,7 +33,8 @@ LT_LZ4_BATCH_MAX = 64
 EXPORTED = (
     "lt_dequant_int4", "lt_dequant_int8", "lt_value_dict_decode", "lt_zrle_decode", "lt_lz4_int4_decode",
     "lt_lz4_int4_decode_batch", "lt_lz4_index_batch", "lt_lz4_int4_expand_batch", "lt_lz4_decode",
-    "lt_lz4_workspace_bytes", "lt_lz4_int4_decode_noalloc", "lt_xxh3_blocks", "lt_int4_gemm",
+    "lt_lz4_workspace_bytes", "lt_lz4_int4_decode_noalloc", "lt_lz4_int4_decode_checked", "lt_xxh3_blocks",
+    "lt_int4_gemm",
     "lt_int4_gemm_workspace_bytes",
     "lt_hct2_layout", "lt_hct2_read_header", "lt_hct2_write_header",
     "lt_status_string", "lt_abi_version",
@@ -96,6 +97,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.lt_lz4_int4_expand_batch.argtypes = [ctypes.POINTER(LtLz4Int4Desc), I32, P, U64, I64, I64, P, P]
     lib.lt_lz4_decode.argtypes = [P, U64, P, I32, P, U64, P, U64, P, P]
     lib.lt_lz4_int4_decode_noalloc.argtypes = [P, U64, P, I32, P, P, I64, I64, I32, P, P, P]
+    lib.lt_lz4_int4_decode_checked.argtypes = [P, U64, P, I32, P, P, I64, I64, I32, P, P, U64, P, I32, P, P, P, P]
+    lib.lt_lz4_int4_decode_checked.restype = ctypes.c_int
     lib.lt_lz4_int4_decode_noalloc.restype = ctypes.c_int
     lib.lt_xxh3_blocks.argtypes = [P, U64, P, I64, P, I32, P, P, P, P, P]
     lib.lt_xxh3_blocks.restype = ctypes.c_int
@@ -209,6 +212,19 @@ def lt_lz4_int4_decode(comp, comp_bytes: int, block_offsets, block_bytes: int, s
     _check(load_library().lt_lz4_int4_decode(_ptr(comp), comp_bytes, _ptr(block_offsets), block_bytes,
                                              _ptr(scales), _ptr(zeros), rows, cols, group_size, _ptr(out), wp, wb,
                                              _ptr(d_status), _stream(stream, out)), "lt_lz4_int4_decode")
+
+
+def lt_lz4_int4_decode_checked(comp, comp_bytes: int, block_offsets, block_bytes: int, scales, zeros, rows: int,
+                               cols: int, group_size: int, out, secret, secret_len: int, expected_hashes,
+                               workspace=None, d_status=None, d_first_bad=None, stream=None) -> None:
+    """lt_lz4_int4_decode with every compressed block's XXH3-64 checked
+    against ``expected_hashes`` first (LT_ERR_CHECKSUM and the first bad
+    block in ``d_first_bad``)."""
+    wp, wb = _ws(workspace)
+    _check(load_library().lt_lz4_int4_decode_checked(
+        _ptr(comp), comp_bytes, _ptr(block_offsets), block_bytes, _ptr(scales), _ptr(zeros), rows, cols, group_size,
+        _ptr(out), wp, wb, _ptr(secret), secret_len, _ptr(expected_hashes), _ptr(d_status), _ptr(d_first_bad),
+        _stream(stream, out)), "lt_lz4_int4_decode_checked")
 
 
 def lt_lz4_int4_decode_batch(descs: Sequence[dict], workspace=None, d_status=None, stream=None) -> None:
