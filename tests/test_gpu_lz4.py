@@ -462,3 +462,27 @@ def test_index_then_expand_in_slices_matches_oracle():
     _, st_o = oracle_fused(bad)
     assert int(stat0.item()) == 0
     assert int(stat1.item()) == st_o != 0
+
+
+# --------------------------------------------------------------------------- both parse paths
+
+@pytest.mark.parametrize("n_blocks", [40, 700])
+def test_lz4_parse_paths_agree_with_the_oracle_and_report_the_same_errors(n_blocks):
+    # A launch with few blocks per SM walks each block staged whole in shared
+    # memory; one with many blocks per SM (more than 4 per SM here) streams
+    # each block through a small ring. Both must decode every regime exactly
+    # and report a damaged block with the oracle's status.
+    from tests._lz4gen import random_blocks
+    comp, offs, raw = random_blocks(60 + n_blocks, n_blocks, 4096)
+    got, st = run_raw(comp, offs, 4096, raw.size, "ws")
+    assert st == 0 and np.array_equal(got, raw)
+    for blk, pos in ((n_blocks - 3, 0), (n_blocks // 2, 17)):
+        bad = comp.copy()
+        s0, s1 = int(offs[blk]), int(offs[blk + 1])
+        bad[s0 + pos:s1] = 0xFF  # every token claims a long literal run past the block
+        want, st_o = oracle.lz4_decode_blocks(bad, offs, 4096, raw.size)
+        got, st_g = run_raw(bad, offs, 4096, raw.size, "ws")
+        assert st_o != 0 and st_g == st_o
+        keep = np.ones(raw.size, bool)
+        keep[blk * 4096:(blk + 1) * 4096] = False
+        assert np.array_equal(got[keep], raw[keep])

@@ -125,7 +125,10 @@ template <int BITS>
 void launch_vec(const uint8_t *packed, const uint16_t *dict, int64_t n_words, void *out, cudaStream_t st) {
   auto k = k_dict_vec<BITS>;
   const int64_t need = (n_words + (int64_t)kThreads * kUnroll - 1) / ((int64_t)kThreads * kUnroll);
-  const int64_t cap = (int64_t)num_sms() * blocks_per_sm((const void *)k, kThreads, 0);
+  // one CTA per tile (the kernel loops, so any grid is correct): as for the
+  // dequant streams, fresh CTAs keep more loads in flight than one resident
+  // wave that loops; the table build is 256 shared-memory stores per CTA
+  const int64_t cap = 1ll << 30;
   const int64_t g = need < cap ? need : cap;
   k<<<(int)(g < 1 ? 1 : g), kThreads, 0, st>>>(reinterpret_cast<const uint32_t *>(packed), dict, n_words, out);
 }

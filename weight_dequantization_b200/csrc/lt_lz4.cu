@@ -301,7 +301,8 @@ struct Leveler {
 // by the slow path, which checks the bounds the oracle checks in the same
 // order, so statuses agree. A match's level is worked out one sequence
 // later, right after the next token is read, so it overlaps that read.
-__device__ __forceinline__ uint32_t parse_block(WarpRing &r, uint32_t olen, uint32_t wcap, uint8_t *lmap,
+template <typename R>
+__device__ __forceinline__ uint32_t parse_block(R &r, uint32_t olen, uint32_t wcap, uint8_t *lmap,
                                                 uint4 *__restrict__ out, uint32_t &n_out, uint32_t &lmax_out) {
   n_out = 0;
   lmax_out = 0;
@@ -458,6 +459,75 @@ __global__ void __launch_bounds__(kParseWarps * 32) k_lz4_parse(const __grid_con
       st = parse_block(r, olen, win_cap(batch.max_block_bytes), lmaps[warp], desc + blk * kCap, n, lmax);
     }
     if (lane == 0) hdr[blk] = make_uint4(n, st, lmax, win_cap(batch.max_block_bytes));  // the window checked against
+  }
+}
+
+// The whole compressed block staged in shared memory: the same walk with
+// none of the ring's bookkeeping (every byte is readable from the start).
+// For launches with few blocks per SM, where each warp's walk is a latency
+// chain and the ring's per-sequence work sits on it.
+struct StagedBlock {
+  const uint8_t *buf;  // rel byte x at buf[x] (rel 0 = a0)
+  const uint8_t *a0, *beg, *end;
+  int lane;
+  __device__ __forceinline__ void need(uint32_t, uint32_t) const {}
+  __device__ __forceinline__ void top_up(uint32_t) const {}
+  __device__ __forceinline__ uint32_t at(uint32_t rel) const { return buf[rel]; }
+};
+
+// bytes a compressed block of a block_bytes-byte output can take in a valid
+// stream (literal-only worst case plus length bytes), plus the 16-byte lead
+__host__ __device__ constexpr uint32_t staged_cap(int32_t block_bytes) {
+  return ((uint32_t)block_bytes + (uint32_t)block_bytes / 255u + 64u + 15u) / 16u * 16u;
+}
+constexpr uint32_t kTooLong = 0x103;  // parse status: the block does not fit the staging buffer (walked by the expand)
+
+__global__ void __launch_bounds__(32) k_lz4_parse_staged(const __grid_constant__ Batch batch, uint4 *__restrict__ hdr,
+                                                          uint4 *__restrict__ desc) {
+  extern __shared__ __align__(16) uint8_t psm[];
+  uint8_t *lmap = psm;                      // kMaxWindow / 16 level granules
+  uint8_t *buf = psm + kMaxWindow / 16;     // the staged block
+  const uint32_t cap = staged_cap(batch.max_block_bytes);
+  const int lane = threadIdx.x;
+  for (int64_t blk = blockIdx.x; blk < batch.total_blocks; blk += gridDim.x) {
+    int64_t b;
+    const Job &jb = find_job(batch, blk, b);
+    const uint32_t olen = block_len(jb, b);
+    const uint64_t s0 = jb.offsets[b], s1 = jb.offsets[b + 1];
+    uint32_t n = 0, st, lmax = 0;
+    if (s1 < s0 || s1 > jb.comp_bytes) {
+      st = LT_ERR_CORRUPT_STREAM;
+    } else {
+      StagedBlock r;
+      r.buf = buf;
+      r.lane = lane;
+      r.beg = jb.comp + s0;
+      r.end = jb.comp + s1;
+      r.a0 = reinterpret_cast<const uint8_t *>(reinterpret_cast<uintptr_t>(r.beg) & ~uintptr_t(15));
+      const uint64_t span = (uint64_t)(r.end - r.a0);
+      if (span > cap) {
+        st = kTooLong;
+      } else {
+        const uint32_t nch = (uint32_t)((span + 15) / 16);
+        for (uint32_t c = (uint32_t)lane; c < nch; c += 32) {
+          const uint8_t *src = r.a0 + 16 * c;
+          uint8_t *dst = buf + 16 * c;
+          if (src >= r.beg) {
+            const uint32_t nb = (uint32_t)((r.end - src) < 16 ? (r.end - src) : 16);
+            cp_async16(dst, src, nb);  // the rest of the 16 bytes is zero-filled
+          } else {
+            for (uint32_t i = 0; i < 16; ++i)
+              if (src + i >= r.beg && src + i < r.end) dst[i] = __ldg(src + i);
+          }
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncwarp();
+        st = parse_block(r, olen, win_cap(batch.max_block_bytes), lmap, desc + blk * kCap, n, lmax);
+      }
+    }
+    if (lane == 0) hdr[blk] = make_uint4(n, st, lmax, win_cap(batch.max_block_bytes));
+    __syncwarp();  // the buffer is refilled for the next block only after every lane is done with it
   }
 }
 
@@ -750,7 +820,27 @@ __device__ __forceinline__ bool resolve_block(uint8_t *win, Seqs &S, const uint8
   return true;
 }
 
-template <bool FUSED>
+// Checked decode: does block b's XXH3-64 (batch's secret) differ from the
+// expected value? One warp; every lane returns the answer. An offset pair
+// outside the stream is not hashed (the decode reports it). Kept out of
+// line so that the hash's registers do not weigh on the expand loop.
+__device__ __noinline__ bool block_hash_differs(const Batch &batch, const Job &jb, int64_t b, int64_t blk, int lane) {
+  const uint64_t c0 = jb.offsets[b], c1 = jb.offsets[b + 1];
+  if (c0 > c1 || c1 > jb.comp_bytes) return false;
+  const uint64_t len = c1 - c0;
+  const uint8_t *in = jb.comp + c0;
+  const GlobalBytes din{jb.comp, jb.comp + jb.comp_bytes}, dsec{batch.secret, batch.secret + batch.secret_len};
+  uint64_t h;
+  if (len > 240)
+    h = xxh3::hash64_long_warp([&](uint64_t off) { return din.rd64(in + off); },
+                               [&](uint64_t off) { return dsec.rd64(batch.secret + off); }, len, batch.secret_len,
+                               lane);
+  else
+    h = __shfl_sync(0xFFFFFFFFu, lane == 0 ? xxh3::hash64(in, len, batch.secret, batch.secret_len) : 0ull, 0);
+  return h != batch.expected[blk];
+}
+
+template <bool FUSED, bool CHECKED>
 __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constant__ Batch batch,
                                                           const uint4 *__restrict__ hdr,
                                                           const uint4 *__restrict__ desc, int32_t *d_status) {
@@ -766,25 +856,11 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
     const Job &jb = find_job(batch, blk, b);
     const int64_t d0 = b * (int64_t)jb.block_bytes;
     const uint32_t olen = block_len(jb, b);
-    if (batch.secret != nullptr && warp == 0) {
+    if (CHECKED && warp == 0) {
       // checked decode: the block's checksum first, so that a damaged block
       // is reported as a checksum mismatch (and not decoded) whatever else is
       // wrong with it
-      const uint64_t c0 = jb.offsets[b], c1 = jb.offsets[b + 1];
-      bool bad = false;
-      if (c0 <= c1 && c1 <= jb.comp_bytes) {
-        const uint64_t len = c1 - c0;
-        const uint8_t *in = jb.comp + c0;
-        const GlobalBytes din{jb.comp, jb.comp + jb.comp_bytes}, dsec{batch.secret, batch.secret + batch.secret_len};
-        uint64_t h;
-        if (len > 240)
-          h = xxh3::hash64_long_warp([&](uint64_t off) { return din.rd64(in + off); },
-                                     [&](uint64_t off) { return dsec.rd64(batch.secret + off); }, len,
-                                     batch.secret_len, lane);
-        else
-          h = lane == 0 ? xxh3::hash64(in, len, batch.secret, batch.secret_len) : 0;
-        bad = h != batch.expected[blk];
-      }  // (an offset pair outside the stream is reported by the decode below)
+      const bool bad = block_hash_differs(batch, jb, b, blk, lane);
       if (lane == 0) {
         s_badsum = bad ? 1u : 0u;
         if (bad) {
@@ -803,11 +879,11 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
     __syncthreads();
     const uint32_t n = s_n, lmax = s_lmax;
     uint32_t st = s_st;
-    if (batch.secret != nullptr && s_badsum) {  // checksum mismatch: not decoded (output unspecified)
+    if (CHECKED && s_badsum) {  // checksum mismatch: not decoded (output unspecified)
       __syncthreads();
       continue;
     }
-    if (st != 0 && st != kOverflow && st != kNoIndex && st != kNoInPlace) {
+    if (st != 0 && st != kOverflow && st != kNoIndex && st != kNoInPlace && st != kTooLong) {
       // the parse found a malformed block: report it; its output stays unwritten
       if (threadIdx.x == 0) report(d_status, (int32_t)st);
       __syncthreads();
@@ -920,6 +996,24 @@ void index_arrays(const void *ws, int64_t total, uint4 *&hdr, uint4 *&desc) {
 }
 
 void launch_parse(const Batch &batch, uint4 *hdr, uint4 *desc, cudaStream_t st) {
+  // Few blocks per SM (e.g. one 4096 x 14336 matrix: 448 blocks): each
+  // block's walk is a latency chain, so the lean walk over a fully staged
+  // block wins. Many blocks per SM (a whole model's layers): the walks are
+  // issue-bound and the ring's small footprint keeps 36 of them per SM.
+  const int64_t sms = num_sms();
+  if (batch.total_blocks <= 4 * sms) {
+    const size_t smem = kMaxWindow / 16 + staged_cap(batch.max_block_bytes);
+    static int attr_set[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+      cudaFuncSetAttribute(k_lz4_parse_staged, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)(kMaxWindow / 16 + staged_cap(kMaxWindow)));
+      attr_set[dev] = 1;
+    }
+    k_lz4_parse_staged<<<(int)batch.total_blocks, 32, smem, st>>>(batch, hdr, desc);
+    return;
+  }
   const int64_t need = (batch.total_blocks + kParseWarps - 1) / kParseWarps;
   const int64_t cap = (int64_t)num_sms() * blocks_per_sm((const void *)k_lz4_parse, kParseWarps * 32, 0);
   k_lz4_parse<<<(int)(need < cap ? need : cap), kParseWarps * 32, 0, st>>>(batch, hdr, desc);
@@ -943,20 +1037,25 @@ lt_status launch_expand(const Batch &batch, bool fused, const uint4 *hdr, const 
                         cudaStream_t st) {
   if (batch.total_blocks == 0) return LT_OK;
   const size_t smem = (size_t)win_cap(batch.max_block_bytes) + 2 * kPad;
-  const void *k = fused ? (const void *)k_lz4_expand<true> : (const void *)k_lz4_expand<false>;
-  static int attr_set[2][64] = {{0}};
+  const bool checked = fused && batch.secret != nullptr;
+  const int variant = checked ? 2 : (fused ? 1 : 0);
+  const void *k = checked ? (const void *)k_lz4_expand<true, true>
+                          : (fused ? (const void *)k_lz4_expand<true, false> : (const void *)k_lz4_expand<false, false>);
+  static int attr_set[3][64] = {{0}};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[fused][dev]) {
+  if (dev >= 0 && dev < 64 && !attr_set[variant][dev]) {
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)win_cap(kMaxWindow) + 2 * kPad);
-    attr_set[fused][dev] = 1;
+    attr_set[variant][dev] = 1;
   }
   const int64_t cap = (int64_t)num_sms() * blocks_per_sm(k, kThreads, smem);
   const int grid = (int)(batch.total_blocks < cap ? batch.total_blocks : cap);
-  if (fused)
-    k_lz4_expand<true><<<grid, kThreads, smem, st>>>(batch, hdr, desc, d_status);
+  if (checked)
+    k_lz4_expand<true, true><<<grid, kThreads, smem, st>>>(batch, hdr, desc, d_status);
+  else if (fused)
+    k_lz4_expand<true, false><<<grid, kThreads, smem, st>>>(batch, hdr, desc, d_status);
   else
-    k_lz4_expand<false><<<grid, kThreads, smem, st>>>(batch, hdr, desc, d_status);
+    k_lz4_expand<false, false><<<grid, kThreads, smem, st>>>(batch, hdr, desc, d_status);
   return launch_status();
 }
 
