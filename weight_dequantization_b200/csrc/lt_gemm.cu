@@ -14,18 +14,19 @@
 //               the x tile (128 x 64 fp16, 128-byte swizzle) and one of the
 //               packed INT4 tile (64 rows x 128 bytes, 128-byte swizzle) into
 //               a 4-deep ring, completion counted on an mbarrier;
-//   warps 2..5  decoders: turn the packed tile into the fp16 B operand in
+//   warps 2..9  decoders: turn the packed tile into the fp16 B operand in
 //               shared memory (N-major, 128-byte swizzle), with the exact
 //               half2 arithmetic of lt_dequant_int4 (bit-identical to it), in
-//               a 2-deep ring; scales and zero points of the next step are
+//               a 3-deep ring; scales and zero points of the next step are
 //               loaded while the current one is decoded;
 //   warp 1      MMA issuer: one thread issues tcgen05.mma kind::f16 (fp32
 //               accumulator in tensor memory, 128 x 256 = 256 columns), four
 //               K = 16 instructions per step, and tcgen05.commit releases the
 //               ring slots;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads lanes
-//               32 (w % 4) ...), conversion to binary16 (or the fp32 partial
-//               of a split), 16-byte stores.
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator (warp w reads lanes
+//               32 (w % 4) ..., warps 2..5 columns 0..127, warps 6..9
+//               columns 128..255), conversion to binary16 (or the fp32
+//               partial of a split), 16-byte stores.
 // Every mbarrier wait is bounded (about a second of clock); a wait that runs
 // out sets LT_ERR_TIMEOUT in the status word and the CTA winds down: the
 // producer waits (bounded) for its copies in flight, the tensor memory is
@@ -40,8 +41,9 @@ namespace {
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kStagesIn = 4;  // x + packed-W slots (TMA)
-constexpr int kStagesB = 2;   // decoded-B slots
-constexpr int kDecWarps = 4;
+constexpr int kStagesB = 3;   // decoded-B slots
+constexpr int kDecWarps = 8;
+constexpr int kUnits = (kBK * kBN / 32) / (kDecWarps * 32);  // 16-byte packed chunks per decoder thread per step
 constexpr int kGemmThreads = (2 + kDecWarps) * 32;
 constexpr uint32_t kABytes = kBM * kBK * 2;   // 16384
 constexpr uint32_t kWBytes = kBK * kBN / 2;   // 8192
@@ -49,7 +51,7 @@ constexpr uint32_t kBBytes = kBN * kBK * 2;   // 32768
 constexpr uint32_t kSmemA = 0;
 constexpr uint32_t kSmemW = kSmemA + kStagesIn * kABytes;
 constexpr uint32_t kSmemB = kSmemW + kStagesIn * kWBytes;
-constexpr uint32_t kSmemTotal = kSmemB + kStagesB * kBBytes;  // 160 KB
+constexpr uint32_t kSmemTotal = kSmemB + kStagesB * kBBytes;  // 192 KB
 constexpr uint32_t kSmemDyn = kSmemTotal + 1024;              // + alignment slack
 constexpr uint32_t kTmemCols = 256;
 // B operand (N-major, 128-byte swizzle): 1 KB atoms of 64 n x 8 k; atoms
@@ -241,20 +243,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
     }
   } else {
     // ---------------- decoders (then epilogue) ----------------
-    const int dt = tid - 64;  // 0 .. 127
-    const int klo = dt & 7, h = (dt >> 3) & 7, khi0 = dt >> 6;
+    const int dt = tid - 64;  // 0 .. 32 kDecWarps - 1
+    const int klo = dt & 7, h = (dt >> 3) & 7, khi0 = dt >> 6;  // unit i: row klo + 8 (khi0 + (kDecWarps / 2) i)
     const int64_t NG = a.N / a.group_size;
     const int64_t gcol = (n0 + 32 * h) / a.group_size;  // this thread's group column
     // scales / zero points of this thread's 4 rows of step `it`
-    auto load_sz = [&](int it, uint32_t (&sc)[4], uint32_t (&zr)[4]) {
+    auto load_sz = [&](int it, uint32_t (&sc)[kUnits], uint32_t (&zr)[kUnits]) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int64_t k = (int64_t)(it_begin + it) * kBK + klo + 8 * (khi0 + 2 * i);
+      for (int i = 0; i < kUnits; ++i) {
+        const int64_t k = (int64_t)(it_begin + it) * kBK + klo + 8 * (khi0 + (kDecWarps / 2) * i);
         sc[i] = __ldg(a.scales + k * NG + gcol);
         zr[i] = a.zeros ? __ldg(a.zeros + k * NG + gcol) : 0u;
       }
     };
-    uint32_t sc[4], zr[4], sc_n[4] = {0, 0, 0, 0}, zr_n[4] = {0, 0, 0, 0};
+    uint32_t sc[kUnits], zr[kUnits], sc_n[kUnits], zr_n[kUnits];
+#pragma unroll
+    for (int i = 0; i < kUnits; ++i) sc_n[i] = zr_n[i] = 0;
     if (n_it > 0) load_sz(0, sc, zr);
     bool ok = true;
     for (int it = 0; it < n_it && ok; ++it) {
@@ -270,8 +274,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
       const uint8_t *wsrc = sm + kSmemW + s * kWBytes;
       uint8_t *bdst = sm + kSmemB + b * kBBytes;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int kk = klo + 8 * (khi0 + 2 * i);  // row of the step, 0..63
+      for (int i = 0; i < kUnits; ++i) {
+        const int kk = klo + 8 * (khi0 + (kDecWarps / 2) * i);  // row of the step, 0..63
         // packed row kk: 128 bytes (256 codes), 16-byte chunk h at chunk h ^ (kk & 7)
         const uint4 v = *reinterpret_cast<const uint4 *>(wsrc + kk * 128 + ((h ^ klo) << 4));
         const uint32_t s2 = bcast_half((uint16_t)sc[i]);
@@ -287,7 +291,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
         }
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < kUnits; ++i) {
         sc[i] = sc_n[i];
         zr[i] = zr_n[i];
       }
@@ -306,7 +310,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
     if (acc_ok && !*(volatile int *)&s_abort && n_it > 0) {
       const int quarter = warp & 3;  // tensor-memory lanes 32 quarter .. + 31
       const int64_t m = m0 + 32 * quarter + lane;
-      for (int c0 = 0; c0 < kBN; c0 += 32) {
+      const int cbeg = warp < 6 ? 0 : kBN / 2;  // each quarter's columns split between two warps
+      for (int c0 = cbeg; c0 < cbeg + kBN / 2; c0 += 32) {
         uint32_t r[32];
         tmem_ld32(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0, r);
         if (m < a.M) {

@@ -594,6 +594,8 @@ __device__ __forceinline__ uint32_t upper_bound(const uint32_t *a, uint32_t n, i
   return lo;
 }
 
+constexpr int kResolved = 0, kResolveFallback = 1, kResolveSkip = 2;
+
 // Per-block state of the expansion, in shared memory.
 struct Seqs {
   uint32_t op[kCap + 1];  // output position of sequence k's literals; op[n] = block length
@@ -626,10 +628,15 @@ struct Seqs {
 //  c. matches, one level at a time (levels come from the parse: a match
 //     reads only literals and matches of lower levels), 8 lanes per match,
 //     a CTA barrier between levels.
-// Returns false before any output byte is written if the index is not one
-// the parse can have written (the caller then walks the block itself).
-__device__ __forceinline__ bool resolve_block(uint8_t *win, Seqs &S, const uint8_t *beg, uint32_t ilen, uint32_t olen,
-                                              uint32_t n, uint32_t lmax, uint32_t wcap, const uint4 *__restrict__ dsc) {
+// Returns kResolveFallback before any output byte is written if the index is
+// not one the parse can have written (the caller then walks the block
+// itself), kResolveSkip if `check_staged` (given the window index of the
+// staged block's first byte and its length, called by every thread once the
+// block is staged) says the block is not to be decoded, else kResolved.
+template <typename Check>
+__device__ __forceinline__ int resolve_block(uint8_t *win, Seqs &S, const uint8_t *beg, uint32_t ilen, uint32_t olen,
+                                             uint32_t n, uint32_t lmax, uint32_t wcap, const uint4 *__restrict__ dsc,
+                                             Check &&check_staged) {
   const uint32_t tid = threadIdx.x;
   const int lane = tid & 31;
   // a. stage
@@ -680,7 +687,10 @@ __device__ __forceinline__ bool resolve_block(uint8_t *win, Seqs &S, const uint8
     S.u.seg[sg] = (uint16_t)(u ? u - 1 : 0u);
   }
   cp_async_wait<0>();
-  if (__syncthreads_or(bad)) return false;
+  if (__syncthreads_or(bad)) return kResolveFallback;
+  // checked decode: the staged copy of the block is hashed here, before the
+  // literal rounds overwrite it
+  if (check_staged(S0, ilen)) return kResolveSkip;
 
   // b. literals. A 4-byte output word holds literals of at most one run
   // (two runs are separated by a match of at least 4 bytes), so each word
@@ -740,7 +750,7 @@ __device__ __forceinline__ bool resolve_block(uint8_t *win, Seqs &S, const uint8
         }
       }
     }
-    return true;
+    return kResolved;
   }
   // counting sort of the matches by level into S.u.m.order
   for (uint32_t i = tid; i <= kLevelCap; i += kThreads) S.u.m.start[i] = 0;
@@ -817,7 +827,7 @@ __device__ __forceinline__ bool resolve_block(uint8_t *win, Seqs &S, const uint8
       }
     }
   }
-  return true;
+  return kResolved;
 }
 
 // Checked decode: does block b's XXH3-64 (batch's secret) differ from the
@@ -840,6 +850,27 @@ __device__ __noinline__ bool block_hash_differs(const Batch &batch, const Job &j
   return h != batch.expected[blk];
 }
 
+// The same check on the block's staged copy in shared memory: window bytes
+// [S0, S0 + ilen). Out of line for the same reason.
+__device__ __noinline__ bool staged_hash_differs(const Batch &batch, const uint8_t *win, uint32_t S0, uint32_t ilen,
+                                                 int64_t blk, int lane) {
+  // 8 bytes of the staged block at offset off: two aligned 8-byte loads (the
+  // window is 16-byte aligned and padded past its end)
+  auto rd = [&](uint64_t off) -> uint64_t {
+    const uint32_t x = S0 + (uint32_t)off, sh = (x & 7u) * 8u;
+    const uint64_t *w = reinterpret_cast<const uint64_t *>(win + (x & ~7u));
+    return sh ? (w[0] >> sh) | (w[1] << (64u - sh)) : w[0];
+  };
+  const GlobalBytes dsec{batch.secret, batch.secret + batch.secret_len};
+  uint64_t h;
+  if (ilen > 240)
+    h = xxh3::hash64_long_warp(rd, [&](uint64_t off) { return dsec.rd64(batch.secret + off); }, ilen,
+                               batch.secret_len, lane);
+  else
+    h = __shfl_sync(0xFFFFFFFFu, lane == 0 ? xxh3::hash64(win + S0, ilen, batch.secret, batch.secret_len) : 0ull, 0);
+  return h != batch.expected[blk];
+}
+
 template <bool FUSED, bool CHECKED>
 __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constant__ Batch batch,
                                                           const uint4 *__restrict__ hdr,
@@ -856,19 +887,6 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
     const Job &jb = find_job(batch, blk, b);
     const int64_t d0 = b * (int64_t)jb.block_bytes;
     const uint32_t olen = block_len(jb, b);
-    if (CHECKED && warp == 0) {
-      // checked decode: the block's checksum first, so that a damaged block
-      // is reported as a checksum mismatch (and not decoded) whatever else is
-      // wrong with it
-      const bool bad = block_hash_differs(batch, jb, b, blk, lane);
-      if (lane == 0) {
-        s_badsum = bad ? 1u : 0u;
-        if (bad) {
-          report(d_status, LT_ERR_CHECKSUM);
-          if (batch.first_bad) atomicMin(batch.first_bad, (unsigned long long)blk);
-        }
-      }
-    }
     if (threadIdx.x == 0) {
       const uint4 h = hdr ? hdr[blk] : make_uint4(0u, kNoIndex, 0u, 0u);
       s_n = h.x;
@@ -879,9 +897,30 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
     __syncthreads();
     const uint32_t n = s_n, lmax = s_lmax;
     uint32_t st = s_st;
-    if (CHECKED && s_badsum) {  // checksum mismatch: not decoded (output unspecified)
+    const uint64_t s0 = jb.offsets[b], s1 = jb.offsets[b + 1];
+    const uint32_t lead = (uint32_t)(reinterpret_cast<uintptr_t>(jb.comp + s0) & 15);
+    if (st == 0 && (n > kCap || s1 < s0 || s1 > jb.comp_bytes || s1 - s0 + lead > wcap))
+      st = kNoIndex;  // never from the parse
+    // Checked decode: each block's checksum comes first, so that a damaged
+    // block is reported as a checksum mismatch (and not decoded) whatever
+    // else is wrong with it. A block that is staged for decoding is hashed
+    // from its staged copy (resolve_block); any other from global memory here.
+    auto mismatch = [&](bool bad) {
+      if (lane == 0) {
+        s_badsum = bad ? 1u : 0u;
+        if (bad) {
+          report(d_status, LT_ERR_CHECKSUM);
+          if (batch.first_bad) atomicMin(batch.first_bad, (unsigned long long)blk);
+        }
+      }
+    };
+    if (CHECKED && st != 0) {
+      if (warp == 0) mismatch(block_hash_differs(batch, jb, b, blk, lane));
       __syncthreads();
-      continue;
+      if (s_badsum) {  // not decoded (output unspecified)
+        __syncthreads();
+        continue;
+      }
     }
     if (st != 0 && st != kOverflow && st != kNoIndex && st != kNoInPlace && st != kTooLong) {
       // the parse found a malformed block: report it; its output stays unwritten
@@ -889,12 +928,21 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
       __syncthreads();
       continue;
     }
-    const uint64_t s0 = jb.offsets[b], s1 = jb.offsets[b + 1];
-    const uint32_t lead = (uint32_t)(reinterpret_cast<uintptr_t>(jb.comp + s0) & 15);
-    if (st == 0 && (n > kCap || s1 < s0 || s1 > jb.comp_bytes || s1 - s0 + lead > wcap))
-      st = kNoIndex;  // never from the parse
-    if (st == 0 && !resolve_block(win, S, jb.comp + s0, (uint32_t)(s1 - s0), olen, n, lmax, wcap, desc + blk * kCap))
-      st = kNoIndex;
+    if (st == 0) {
+      auto check_staged = [&](uint32_t S0, uint32_t ilen) -> bool {
+        if (!CHECKED) return false;
+        if (warp == 0) mismatch(staged_hash_differs(batch, win, S0, ilen, blk, lane));
+        __syncthreads();
+        return s_badsum != 0;
+      };
+      const int rs = resolve_block(win, S, jb.comp + s0, (uint32_t)(s1 - s0), olen, n, lmax, wcap,
+                                   desc + blk * kCap, check_staged);
+      if (rs == kResolveSkip) {  // checksum mismatch: not decoded (output unspecified)
+        __syncthreads();
+        continue;
+      }
+      if (rs == kResolveFallback) st = kNoIndex;
+    }
     if (st != 0 && warp == 0) {
       int err = LT_ERR_CORRUPT_STREAM;
       if (s0 <= s1 && s1 <= jb.comp_bytes) err = walk_block_warp(jb.comp + s0, s1 - s0, win, olen, lane);

@@ -166,39 +166,47 @@ LT_HD uint64_t hash64(const uint8_t *in, uint64_t len, const uint8_t *sec, uint6
 // input bytes at offset off (little-endian, any alignment); `rk(off)` the 8
 // secret bytes at offset off. Every lane returns the hash.
 // ---------------------------------------------------------------------------
+
+// the initial accumulator i: kP32_3, kP64_1, kP64_2, kP64_3, kP64_4, kP32_2, kP64_5, kP32_1
+__device__ __forceinline__ uint64_t acc_init(int i) {
+  return (i & 4) ? ((i & 2) ? ((i & 1) ? kP32_1 : kP64_5) : ((i & 1) ? kP32_2 : kP64_4))
+                 : ((i & 2) ? ((i & 1) ? kP64_3 : kP64_2) : ((i & 1) ? kP64_1 : kP32_3));
+}
+
+// what stripes [0, ns) starting at input offset base (stripe s keyed at
+// secret offset key0 + 8 s) add to acc[lane % 8]; every lane returns its sum
 template <typename RD, typename RK>
-__device__ __forceinline__ uint64_t hash64_long_warp(RD rd, RK rk, uint64_t len, uint64_t sec_len, int lane) {
-  const int i = lane & 7;
-  // the initial accumulators kP32_3, kP64_1, kP64_2, kP64_3, kP64_4, kP32_2, kP64_5, kP32_1, by i
-  uint64_t acc = (i & 4) ? ((i & 2) ? ((i & 1) ? kP32_1 : kP64_5) : ((i & 1) ? kP32_2 : kP64_4))
-                         : ((i & 2) ? ((i & 1) ? kP64_3 : kP64_2) : ((i & 1) ? kP64_1 : kP32_3));
-  const uint64_t per_block = (sec_len - 64) / 8;
-  const uint64_t block_len = 64 * per_block;
-  const uint64_t n_blocks = (len - 1) / block_len;
-  const uint64_t scr = rk(sec_len - 64 + 8 * (uint64_t)i);
-  // stripes [0, ns) starting at input offset base, stripe s keyed at secret offset key0 + 8 s
-  auto stripes = [&](uint64_t base, uint64_t ns, uint64_t key0) {
-    uint64_t m = 0, d = 0;
-    for (uint64_t st = (uint64_t)(lane >> 3); st < ns; st += 4) {
-      const uint64_t v = rd(base + 64 * st + 8 * (uint64_t)i);
-      const uint64_t k = v ^ rk(key0 + 8 * st + 8 * (uint64_t)i);
-      d += v;
-      m += (k & 0xFFFFFFFFull) * (k >> 32);
-    }
-    m += __shfl_xor_sync(0xFFFFFFFFu, m, 8);
-    m += __shfl_xor_sync(0xFFFFFFFFu, m, 16);
-    d += __shfl_xor_sync(0xFFFFFFFFu, d, 8);
-    d += __shfl_xor_sync(0xFFFFFFFFu, d, 16);
-    acc += m + __shfl_xor_sync(0xFFFFFFFFu, d, 1);
-  };
-  for (uint64_t b = 0; b < n_blocks; ++b) {
-    stripes(b * block_len, per_block, 0);
-    acc ^= acc >> 47;
-    acc ^= scr;
-    acc *= kP32_1;
+__device__ __forceinline__ uint64_t stripe_terms(RD &rd, RK &rk, uint64_t base, uint64_t ns, uint64_t key0,
+                                                 int lane) {
+  const uint64_t i = (uint64_t)(lane & 7);
+  uint64_t m = 0, d = 0;
+  for (uint64_t st = (uint64_t)(lane >> 3); st < ns; st += 4) {
+    const uint64_t v = rd(base + 64 * st + 8 * i);
+    const uint64_t k = v ^ rk(key0 + 8 * st + 8 * i);
+    d += v;
+    m += (k & 0xFFFFFFFFull) * (k >> 32);
   }
-  stripes(n_blocks * block_len, ((len - 1) - block_len * n_blocks) / 64, 0);
-  stripes(len - 64, 1, sec_len - 64 - 7);
+  m += __shfl_xor_sync(0xFFFFFFFFu, m, 8);
+  m += __shfl_xor_sync(0xFFFFFFFFu, m, 16);
+  d += __shfl_xor_sync(0xFFFFFFFFu, d, 8);
+  d += __shfl_xor_sync(0xFFFFFFFFu, d, 16);
+  return m + __shfl_xor_sync(0xFFFFFFFFu, d, 1);
+}
+
+__device__ __forceinline__ uint64_t scramble(uint64_t acc, uint64_t scr) {
+  acc ^= acc >> 47;
+  acc ^= scr;
+  return acc * kP32_1;
+}
+
+// tail stripes, last stripe and merge, after the n_blocks full scramble
+// intervals have been added into acc (lane l holds acc[l % 8])
+template <typename RD, typename RK>
+__device__ __forceinline__ uint64_t finish_long(RD &rd, RK &rk, uint64_t acc, uint64_t len, uint64_t sec_len,
+                                                uint64_t n_blocks, int lane) {
+  const uint64_t block_len = 64 * ((sec_len - 64) / 8);
+  acc += stripe_terms(rd, rk, n_blocks * block_len, ((len - 1) - block_len * n_blocks) / 64, 0, lane);
+  acc += stripe_terms(rd, rk, len - 64, 1, sec_len - 64 - 7, lane);
   // merge: term j (lanes 0..3) from acc[2j] and acc[2j + 1]
   const uint64_t a_even = __shfl_sync(0xFFFFFFFFu, acc, (2 * lane) & 7);
   const uint64_t a_odd = __shfl_sync(0xFFFFFFFFu, acc, (2 * lane + 1) & 7);
@@ -206,6 +214,17 @@ __device__ __forceinline__ uint64_t hash64_long_warp(RD rd, RK rk, uint64_t len,
   t += __shfl_xor_sync(0xFFFFFFFFu, t, 1);
   t += __shfl_xor_sync(0xFFFFFFFFu, t, 2);
   return avalanche3(len * kP64_1 + __shfl_sync(0xFFFFFFFFu, t, 0));
+}
+
+template <typename RD, typename RK>
+__device__ __forceinline__ uint64_t hash64_long_warp(RD rd, RK rk, uint64_t len, uint64_t sec_len, int lane) {
+  uint64_t acc = acc_init(lane & 7);
+  const uint64_t per_block = (sec_len - 64) / 8;
+  const uint64_t block_len = 64 * per_block;
+  const uint64_t n_blocks = (len - 1) / block_len;
+  const uint64_t scr = rk(sec_len - 64 + 8 * (uint64_t)(lane & 7));
+  for (uint64_t b = 0; b < n_blocks; ++b) acc = scramble(acc + stripe_terms(rd, rk, b * block_len, per_block, 0, lane), scr);
+  return finish_long(rd, rk, acc, len, sec_len, n_blocks, lane);
 }
 #endif
 
