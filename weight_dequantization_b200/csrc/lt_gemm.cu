@@ -256,21 +256,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
         zr[i] = a.zeros ? __ldg(a.zeros + k * NG + gcol) : 0u;
       }
     };
-    uint32_t sc[kUnits], zr[kUnits], sc_n[kUnits], zr_n[kUnits];
-#pragma unroll
-    for (int i = 0; i < kUnits; ++i) sc_n[i] = zr_n[i] = 0;
-    if (n_it > 0) load_sz(0, sc, zr);
+    // Scales and zero points arrive through three register sets, each loaded
+    // three steps before its use and reloaded right after it (no register
+    // moves: a move would wait for the load it copies).
+    uint32_t scA[kUnits], zrA[kUnits], scB[kUnits], zrB[kUnits], scC[kUnits], zrC[kUnits];
+    if (n_it > 0) load_sz(0, scA, zrA);
+    if (n_it > 1) load_sz(1, scB, zrB);
+    if (n_it > 2) load_sz(2, scC, zrC);
     bool ok = true;
-    for (int it = 0; it < n_it && ok; ++it) {
+    // one K step: wait for its packed tile and a free B slot, decode with
+    // (sc, zr), refill (sc, zr) for step it + 3, hand the slot to the MMA
+    auto step = [&](int it, uint32_t(&sc)[kUnits], uint32_t(&zr)[kUnits]) -> bool {
       const int s = it % kStagesIn, b = it % kStagesB;
-      if (it + 1 < n_it) load_sz(it + 1, sc_n, zr_n);
       if (!mbar_wait(smem_u32(&bar_full[s]), (it / kStagesIn) & 1) ||
           (it >= kStagesB && !mbar_wait(smem_u32(&bar_bempty[b]), ((it / kStagesB) - 1) & 1))) {
         fail();
-        ok = false;
-        break;
+        return false;
       }
-      if (*(volatile int *)&s_abort) break;
+      if (*(volatile int *)&s_abort) return false;
       const uint8_t *wsrc = sm + kSmemW + s * kWBytes;
       uint8_t *bdst = sm + kSmemB + b * kBBytes;
 #pragma unroll
@@ -290,11 +293,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
           *reinterpret_cast<uint4 *>(atom + ((c ^ klo) << 4)) = o[j];
         }
       }
-#pragma unroll
-      for (int i = 0; i < kUnits; ++i) {
-        sc[i] = sc_n[i];
-        zr[i] = zr_n[i];
-      }
+      if (it + 3 < n_it) load_sz(it + 3, sc, zr);
       // generic-proxy writes of B become visible to the tensor core's async proxy
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
@@ -302,6 +301,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
         mbar_arrive(smem_u32(&bar_aempty[s]));
         mbar_arrive(smem_u32(&bar_bfull[b]));
       }
+      return true;
+    };
+    for (int it = 0; it < n_it && ok; it += 3) {
+      ok = step(it, scA, zrA);
+      if (ok && it + 1 < n_it) ok = step(it + 1, scB, zrB);
+      if (ok && it + 2 < n_it) ok = step(it + 2, scC, zrC);
     }
     // ---------------- epilogue ----------------
     const bool acc_ok = mbar_wait(smem_u32(&bar_acc), 0);

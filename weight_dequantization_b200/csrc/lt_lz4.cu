@@ -475,19 +475,18 @@ struct StagedBlock {
   __device__ __forceinline__ uint32_t at(uint32_t rel) const { return buf[rel]; }
 };
 
-// bytes a compressed block of a block_bytes-byte output can take in a valid
-// stream (literal-only worst case plus length bytes), plus the 16-byte lead
-__host__ __device__ constexpr uint32_t staged_cap(int32_t block_bytes) {
-  return ((uint32_t)block_bytes + (uint32_t)block_bytes / 255u + 64u + 15u) / 16u * 16u;
-}
-constexpr uint32_t kTooLong = 0x103;  // parse status: the block does not fit the staging buffer (walked by the expand)
+// Staging buffer of a CTA of k_lz4_parse_staged: 51 KB, so that four CTAs
+// (with their level maps) fit in an SM's shared memory. Compressible 64 KB
+// blocks fit (the INT4 workloads' largest is 50.5 KB); a block that does not
+// (e.g. incompressible data) streams through the first 2 KB of the buffer as
+// the ring of k_lz4_parse instead.
+constexpr uint32_t kStageCap = 51 * 1024;
 
 __global__ void __launch_bounds__(32) k_lz4_parse_staged(const __grid_constant__ Batch batch, uint4 *__restrict__ hdr,
                                                           uint4 *__restrict__ desc) {
   extern __shared__ __align__(16) uint8_t psm[];
   uint8_t *lmap = psm;                      // kMaxWindow / 16 level granules
-  uint8_t *buf = psm + kMaxWindow / 16;     // the staged block
-  const uint32_t cap = staged_cap(batch.max_block_bytes);
+  uint8_t *buf = psm + kMaxWindow / 16;     // the staged block (kStageCap bytes)
   const int lane = threadIdx.x;
   for (int64_t blk = blockIdx.x; blk < batch.total_blocks; blk += gridDim.x) {
     int64_t b;
@@ -505,8 +504,18 @@ __global__ void __launch_bounds__(32) k_lz4_parse_staged(const __grid_constant__
       r.end = jb.comp + s1;
       r.a0 = reinterpret_cast<const uint8_t *>(reinterpret_cast<uintptr_t>(r.beg) & ~uintptr_t(15));
       const uint64_t span = (uint64_t)(r.end - r.a0);
-      if (span > cap) {
-        st = kTooLong;
+      if (span > kStageCap) {  // too long to stage: the ring walk, in the buffer's first 2 KB
+        WarpRing w;
+        w.buf = buf;
+        w.lane = lane;
+        w.beg = r.beg;
+        w.end = r.end;
+        w.a0 = r.a0;
+        w.total = (uint32_t)((w.end - w.a0 + kPChunk - 1) / kPChunk);
+        w.issued = 0;
+        w.done = 0;
+        w.top_up(0);
+        st = parse_block(w, olen, win_cap(batch.max_block_bytes), lmap, desc + blk * kCap, n, lmax);
       } else {
         const uint32_t nch = (uint32_t)((span + 15) / 16);
         for (uint32_t c = (uint32_t)lane; c < nch; c += 32) {
@@ -922,7 +931,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
         continue;
       }
     }
-    if (st != 0 && st != kOverflow && st != kNoIndex && st != kNoInPlace && st != kTooLong) {
+    if (st != 0 && st != kOverflow && st != kNoIndex && st != kNoInPlace) {
       // the parse found a malformed block: report it; its output stays unwritten
       if (threadIdx.x == 0) report(d_status, (int32_t)st);
       __syncthreads();
@@ -1050,13 +1059,12 @@ void launch_parse(const Batch &batch, uint4 *hdr, uint4 *desc, cudaStream_t st) 
   // issue-bound and the ring's small footprint keeps 36 of them per SM.
   const int64_t sms = num_sms();
   if (batch.total_blocks <= 4 * sms) {
-    const size_t smem = kMaxWindow / 16 + staged_cap(batch.max_block_bytes);
+    const size_t smem = kMaxWindow / 16 + kStageCap;
     static int attr_set[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-      cudaFuncSetAttribute(k_lz4_parse_staged, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)(kMaxWindow / 16 + staged_cap(kMaxWindow)));
+      cudaFuncSetAttribute(k_lz4_parse_staged, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       attr_set[dev] = 1;
     }
     k_lz4_parse_staged<<<(int)batch.total_blocks, 32, smem, st>>>(batch, hdr, desc);

@@ -39,6 +39,55 @@ __device__ __forceinline__ uint32_t rd16(const uint8_t *__restrict__ base, uint6
   return (uint32_t)__ldg(base + p) | ((uint32_t)__ldg(base + p + 1) << 8);
 }
 
+// A lane's sequential reader over its chunk: three aligned 16-byte windows in
+// registers, the two after the current one loaded ahead of use, so a lane
+// issues one 16-byte load per 16 bytes it consumes (not one per field) and
+// its next loads are in flight while it works. Windows that reach outside
+// the encoded buffer are read byte by byte, inside it only.
+struct LaneReader {
+  uintptr_t lo, hi;  // the encoded buffer [enc, enc + enc_bytes)
+  uintptr_t wb;      // address of window 0 (16-byte aligned)
+  uint4 w0, w1, w2;
+  __device__ __forceinline__ uint4 load(uintptr_t a) const {
+    if (a >= lo && a + 16 <= hi) return ld_stream_u128(reinterpret_cast<const void *>(a));
+    uint32_t b0 = 0, b1 = 0, b2 = 0, b3 = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uintptr_t x = a + (uintptr_t)i;
+      const uint32_t v = (x >= lo && x < hi) ? (uint32_t)__ldg(reinterpret_cast<const uint8_t *>(x)) : 0u;
+      const uint32_t sh = 8u * (uint32_t)(i & 3);
+      if (i < 4) b0 |= v << sh;
+      else if (i < 8) b1 |= v << sh;
+      else if (i < 12) b2 |= v << sh;
+      else b3 |= v << sh;
+    }
+    return make_uint4(b0, b1, b2, b3);
+  }
+  __device__ __forceinline__ void start(uintptr_t a) {
+    wb = a & ~uintptr_t(15);
+    w0 = load(wb);
+    w1 = load(wb + 16);
+    w2 = load(wb + 32);
+  }
+  // the little-endian u16 at even address a (a >= the current window)
+  __device__ __forceinline__ uint32_t get16(uintptr_t a) {
+    uintptr_t off = a - wb;
+    if (off >= 48) {  // a jump past the windows held (a long literal run): start again there
+      start(a);
+      off = a - wb;
+    }
+    while (off >= 16) {
+      w0 = w1;
+      w1 = w2;
+      w2 = load(wb + 48);
+      wb += 16;
+      off -= 16;
+    }
+    const uint32_t word = (off & 8) ? ((off & 4) ? w0.w : w0.z) : ((off & 4) ? w0.y : w0.x);
+    return (off & 2) ? (word >> 16) : (word & 0xFFFFu);
+  }
+};
+
 template <bool VEC>
 __global__ void __launch_bounds__(kZThreads) k_zrle(const uint8_t *__restrict__ enc, uint64_t enc_bytes,
                                                       const uint64_t *__restrict__ offsets, int64_t n, int32_t chunk,
@@ -68,6 +117,15 @@ __global__ void __launch_bounds__(kZThreads) k_zrle(const uint8_t *__restrict__ 
   }
   const uint8_t *src = enc + b0;
   const bool even = ((reinterpret_cast<uintptr_t>(src)) & 1) == 0;
+  LaneReader rdr;
+  rdr.lo = reinterpret_cast<uintptr_t>(enc);
+  rdr.hi = reinterpret_cast<uintptr_t>(enc) + enc_bytes;
+  if (even && nb) rdr.start(reinterpret_cast<uintptr_t>(src));
+  // the u16 at chunk byte q: through the window reader, or byte by byte for
+  // a chunk at an odd address
+  auto field = [&](uint64_t q) -> uint32_t {
+    return even ? rdr.get16(reinterpret_cast<uintptr_t>(src) + (uintptr_t)q) : rd16(src, q, false);
+  };
   uint64_t p = 0;          // next unread byte of the chunk
   uint32_t pos = 0;        // elements produced
   uint32_t zrem = 0, lrem = 0;  // zeros / literals of the current record still to produce
@@ -90,7 +148,7 @@ __global__ void __launch_bounds__(kZThreads) k_zrle(const uint8_t *__restrict__ 
       }
       if (lrem) {
         const uint32_t t = lrem < s_end - pos ? lrem : s_end - pos;
-        for (uint32_t i = 0; i < t; ++i) mine[pos - s0 + i] = (uint16_t)rd16(src, lsrc + 2 * i, even);
+        for (uint32_t i = 0; i < t; ++i) mine[pos - s0 + i] = (uint16_t)field(lsrc + 2 * i);
         lsrc += 2 * (uint64_t)t;
         pos += t;
         lrem -= t;
@@ -107,7 +165,8 @@ __global__ void __launch_bounds__(kZThreads) k_zrle(const uint8_t *__restrict__ 
         walking = false;
         break;
       }
-      const uint32_t zr = rd16(src, p, even), nl = rd16(src, p + 2, even);
+      const uint32_t zr = field(p);
+      const uint32_t nl = field(p + 2);
       p += 4;
       if ((uint64_t)pos + zr + nl > len || p + 2 * (uint64_t)nl > nb) {
         err = LT_ERR_CORRUPT_STREAM;
