@@ -66,6 +66,9 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=8, help="C5 layers (8 is the workload)")
+    ap.add_argument("--gemm-shapes", default="q/o,k/v,gate/up,down",
+                    help="C5 weight shapes of the GEMM leg (G): comma-separated subset of q/o, k/v, gate/up, down")
+    ap.add_argument("--gemm-m", default="1,16,128,4096", help="batch sizes M of the GEMM leg (G)")
     ap.add_argument("--no-parity", action="store_true",
                     help="skip the parity pass (profiling runs only: the line then says parity was not checked)")
     ap.add_argument("--only", default="C1,C2,C3,C4,C4u,C5,V,S,G",
@@ -915,9 +918,10 @@ def read_tflops_peak():
         return 1590.0, "fallback"
 
 
-def gemm_timing(hbm_peak: float, reps: int = 10, warmup: int = 3,
-                shapes=(("q/o", 8192, 8192), ("k/v", 8192, 1024), ("gate/up", 8192, 28672), ("down", 28672, 8192)),
-                batch=(1, 16, 128, 4096)):
+GEMM_SHAPES = (("q/o", 8192, 8192), ("k/v", 8192, 1024), ("gate/up", 8192, 28672), ("down", 28672, 8192))
+
+
+def gemm_timing(hbm_peak: float, reps: int = 10, warmup: int = 3, shapes=GEMM_SHAPES, batch=(1, 16, 128, 4096)):
     """Fused INT4 decode -> GEMM (lt_int4_gemm) on the C5 weight shapes
     ([K, N] = [in, out], C4's code law, group 128) against decode-then-
     cuBLAS (lt_dequant_int4 into an fp16 buffer, then torch.matmul). Device
@@ -1260,7 +1264,9 @@ def run_lt(args, rank, world, local):
         c1g = c1_graph_steady_state(hw, peak) if "C1" in hw else None
         vd = value_dict_timing(peak) if "V" in only else None
         sapi = stream_api_timing(hw) if ("S" in only and hw.get("C5")) else None
-        gemm = gemm_timing(peak) if "G" in only else None
+        gshapes = tuple(x for x in GEMM_SHAPES if x[0] in args.gemm_shapes.split(","))
+        gemm = gemm_timing(peak, shapes=gshapes, batch=tuple(int(m) for m in args.gemm_m.split(","))) \
+            if "G" in only else None
         csum = checksum_timing(dw, hw, peak) if "C4" in hw else None
         if vd is not None and world == 1 and not args.no_cpu_baseline:
             vd["cpu_baseline"] = cpu_baseline_value_dict()

@@ -2,205 +2,203 @@
 // ("LoreToken-powered GPU memory layer", compression strategies: zero-run
 // encoding for ReLU outputs).
 //
-// The work of a chunk is a serial walk over its records (where a record's
-// header sits depends on every literal count before it) plus a dense fp16
-// output that is mostly zeros. So each LANE walks one chunk, and each warp
-// writes its 32 chunks' output together:
-//  - lane l of a warp owns chunk 32 w + l and a 256-element stripe tile in
-//    shared memory that starts out zero;
-//  - round r: every lane walks its records until its output position reaches
-//    the end of stripe r of its chunk, skipping zero runs (the tile is
-//    already zero) and writing literals into its tile; a zero run or literal
-//    run that crosses the stripe end carries over to the next round;
-//  - then the warp stores the 32 stripes one after the other, each as 32
-//    16-byte pieces (512 contiguous bytes per store instruction), zeroing the
-//    tile behind it.
-// So a record costs a few instructions of one lane (32 chunks walk side by
-// side) and the output leaves with fully coalesced 16-byte stores. Every
-// walk is bounded by its chunk's bytes; the checks are the oracle's, in its
-// order.
+// One warp per chunk, no shared memory (so up to 64 warps per SM keep the
+// HBM streams busy):
+//  1. the chunk's output is zero-filled with 16-byte stores;
+//  2. the encoded bytes are read 128 at a time into registers (two 16-bit
+//     fields per lane), realigned to the chunk's 16-bit grid with funnel
+//     shifts;
+//  3. in each window the warp walks the record chain -- one shuffle per
+//     record reads its (zero run, literal count) -- and parks record k's
+//     position and header in lane k; then all records of the window are
+//     finished in parallel: a warp scan gives each record's output offset,
+//     a vote finds the first bad record (the oracle's checks, in its order),
+//     and every lane stores the literals it holds (L2 merges them with the
+//     zero fill before HBM sees them).
+// A record whose literals run past the 128-byte window carries over into
+// the next window. Every loop is bounded by the chunk's byte range.
 #include "lt_common.cuh"
 
 namespace lt {
 namespace {
 
-constexpr int kZWarps = 2;                 // warps per CTA (33 KB of tiles: six CTAs per SM)
-constexpr int kZThreads = kZWarps * 32;
-constexpr uint32_t kStripe = 256;          // elements per stripe
-constexpr uint32_t kPitch = 2 * kStripe + 16;  // bytes per lane tile (padded: lanes' tiles start on different banks)
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr uint32_t kWin = 128;  // bytes per window = 64 u16 slots, 2 per lane
 
-// the little-endian u16 at chunk byte p (the chunk may start at an odd address)
-__device__ __forceinline__ uint32_t rd16(const uint8_t *__restrict__ base, uint64_t p, bool even) {
-  if (even) {
-    uint16_t v;
-    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(base + p));
-    return v;
-  }
-  return (uint32_t)__ldg(base + p) | ((uint32_t)__ldg(base + p + 1) << 8);
+// aligned 4-byte word at byte address a (a % 4 == 0) of enc; bytes past
+// `limit` (the end of the encoded buffer) read as 0
+__device__ __forceinline__ uint32_t load_word(const uint8_t *__restrict__ enc, uint64_t a, uint64_t limit) {
+  if (a + 4 <= limit) return __ldg(reinterpret_cast<const uint32_t *>(enc + a));
+  uint32_t v = 0;
+  for (int j = 0; j < 4; ++j)
+    if (a + j < limit) v |= (uint32_t)__ldg(enc + a + j) << (8 * j);
+  return v;
 }
 
-// A lane's sequential reader over its chunk: three aligned 16-byte windows in
-// registers, the two after the current one loaded ahead of use, so a lane
-// issues one 16-byte load per 16 bytes it consumes (not one per field) and
-// its next loads are in flight while it works. Windows that reach outside
-// the encoded buffer are read byte by byte, inside it only.
-struct LaneReader {
-  uintptr_t lo, hi;  // the encoded buffer [enc, enc + enc_bytes)
-  uintptr_t wb;      // address of window 0 (16-byte aligned)
-  uint4 w0, w1, w2;
-  __device__ __forceinline__ uint4 load(uintptr_t a) const {
-    if (a >= lo && a + 16 <= hi) return ld_stream_u128(reinterpret_cast<const void *>(a));
-    uint32_t b0 = 0, b1 = 0, b2 = 0, b3 = 0;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uintptr_t x = a + (uintptr_t)i;
-      const uint32_t v = (x >= lo && x < hi) ? (uint32_t)__ldg(reinterpret_cast<const uint8_t *>(x)) : 0u;
-      const uint32_t sh = 8u * (uint32_t)(i & 3);
-      if (i < 4) b0 |= v << sh;
-      else if (i < 8) b1 |= v << sh;
-      else if (i < 12) b2 |= v << sh;
-      else b3 |= v << sh;
-    }
-    return make_uint4(b0, b1, b2, b3);
+// zero-fill out[0, len)
+__device__ __forceinline__ void zero_fill(uint16_t *out, uint32_t len, int lane) {
+  uint32_t i0 = 0;
+  const uintptr_t mis = reinterpret_cast<uintptr_t>(out) & 15;
+  if (mis & 1) {  // not even 2-byte aligned cannot happen (checked on the host)
+    for (uint32_t i = lane; i < len; i += 32) out[i] = 0;
+    return;
   }
-  __device__ __forceinline__ void start(uintptr_t a) {
-    wb = a & ~uintptr_t(15);
-    w0 = load(wb);
-    w1 = load(wb + 16);
-    w2 = load(wb + 32);
-  }
-  // the little-endian u16 at even address a (a >= the current window)
-  __device__ __forceinline__ uint32_t get16(uintptr_t a) {
-    uintptr_t off = a - wb;
-    if (off >= 48) {  // a jump past the windows held (a long literal run): start again there
-      start(a);
-      off = a - wb;
-    }
-    while (off >= 16) {
-      w0 = w1;
-      w1 = w2;
-      w2 = load(wb + 48);
-      wb += 16;
-      off -= 16;
-    }
-    const uint32_t word = (off & 8) ? ((off & 4) ? w0.w : w0.z) : ((off & 4) ? w0.y : w0.x);
-    return (off & 2) ? (word >> 16) : (word & 0xFFFFu);
-  }
-};
+  // elements up to the first 16-byte boundary
+  const uint32_t head = mis ? (uint32_t)((16 - mis) / 2) : 0u;
+  for (uint32_t i = lane; i < head && i < len; i += 32) out[i] = 0;
+  i0 = head < len ? head : len;
+  const uint32_t n16 = (len - i0) / 8;
+  uint4 *o4 = reinterpret_cast<uint4 *>(out + i0);
+  for (uint32_t i = lane; i < n16; i += 32) st_u128(o4 + i, make_uint4(0u, 0u, 0u, 0u));
+  for (uint32_t i = i0 + 8 * n16 + lane; i < len; i += 32) out[i] = 0;
+}
 
-template <bool VEC>
-__global__ void __launch_bounds__(kZThreads) k_zrle(const uint8_t *__restrict__ enc, uint64_t enc_bytes,
-                                                      const uint64_t *__restrict__ offsets, int64_t n, int32_t chunk,
-                                                      int64_t n_chunks, uint16_t *__restrict__ out,
-                                                      int32_t *d_status) {
-  __shared__ __align__(16) uint8_t tiles[kZWarps][32 * kPitch];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint8_t *wt = tiles[warp];
-  uint16_t *mine = reinterpret_cast<uint16_t *>(wt + lane * kPitch);
-  const int64_t c0 = ((int64_t)blockIdx.x * kZWarps + warp) * 32;  // the warp's first chunk
-  const int64_t c = c0 + lane;
+__global__ void __launch_bounds__(kThreads, 6) k_zrle(const uint8_t *__restrict__ enc, uint64_t enc_bytes,
+                                                   const uint64_t *__restrict__ offsets, int64_t n, int32_t chunk,
+                                                   int64_t n_chunks, uint16_t *__restrict__ out,
+                                                   int32_t *d_status) {
+  const uint32_t lane = threadIdx.x & 31;
+  const int64_t warp_global = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int64_t warps_total = (int64_t)gridDim.x * kWarps;
 
-  for (uint32_t i = (uint32_t)lane; i < 32 * kPitch / 16; i += 32)
-    reinterpret_cast<uint4 *>(wt)[i] = make_uint4(0u, 0u, 0u, 0u);
-
-  // this lane's chunk
-  uint32_t len = 0;
-  uint64_t b0 = 0, nb = 0;
-  int err = 0;
-  if (c < n_chunks) {
+  for (int64_t c = warp_global; c < n_chunks; c += warps_total) {
     const int64_t e0 = c * (int64_t)chunk;
-    len = (uint32_t)((n - e0) < chunk ? (n - e0) : chunk);
-    b0 = offsets[c];
-    const uint64_t b1 = offsets[c + 1];
-    if (b1 < b0 || b1 > enc_bytes) err = LT_ERR_CORRUPT_STREAM;
-    else nb = b1 - b0;
-  }
-  const uint8_t *src = enc + b0;
-  const bool even = ((reinterpret_cast<uintptr_t>(src)) & 1) == 0;
-  LaneReader rdr;
-  rdr.lo = reinterpret_cast<uintptr_t>(enc);
-  rdr.hi = reinterpret_cast<uintptr_t>(enc) + enc_bytes;
-  if (even && nb) rdr.start(reinterpret_cast<uintptr_t>(src));
-  // the u16 at chunk byte q: through the window reader, or byte by byte for
-  // a chunk at an odd address
-  auto field = [&](uint64_t q) -> uint32_t {
-    return even ? rdr.get16(reinterpret_cast<uintptr_t>(src) + (uintptr_t)q) : rd16(src, q, false);
-  };
-  uint64_t p = 0;          // next unread byte of the chunk
-  uint32_t pos = 0;        // elements produced
-  uint32_t zrem = 0, lrem = 0;  // zeros / literals of the current record still to produce
-  uint64_t lsrc = 0;       // byte of the next literal
-  bool walking = err == 0 && len > 0;
-  const uint32_t stripes = (len + kStripe - 1) / kStripe;
-  const uint32_t rounds = __reduce_max_sync(0xFFFFFFFFu, stripes);
-  __syncwarp();
+    const uint32_t len = (uint32_t)((n - e0) < chunk ? (n - e0) : chunk);
+    uint16_t *o = out + e0;
+    zero_fill(o, len, (int)lane);
+    __syncwarp();  // the literal stores below land after the zero fill
 
-  for (uint32_t r = 0; r < rounds; ++r) {
-    const uint32_t s0 = r * kStripe;
-    const uint32_t s_end = (s0 + kStripe) < len ? (s0 + kStripe) : len;
-    // 1. walk this lane's records up to the end of its stripe r
-    while (walking && pos < s_end) {
-      if (zrem) {  // zeros: the tile is zero already
-        const uint32_t t = zrem < s_end - pos ? zrem : s_end - pos;
-        pos += t;
-        zrem -= t;
-        if (zrem) break;
-      }
-      if (lrem) {
-        const uint32_t t = lrem < s_end - pos ? lrem : s_end - pos;
-        for (uint32_t i = 0; i < t; ++i) mine[pos - s0 + i] = (uint16_t)field(lsrc + 2 * i);
-        lsrc += 2 * (uint64_t)t;
-        pos += t;
-        lrem -= t;
-        if (lrem) break;
-      }
-      if (pos >= len) {
-        walking = false;
-        break;
-      }
-      if (pos >= s_end) break;
-      // the next record's header (the oracle's checks, in its order)
-      if (p + 4 > nb) {
+    const uint64_t b0 = offsets[c], b1 = offsets[c + 1];
+    if (b1 < b0 || b1 > enc_bytes) {
+      if (lane == 0) report(d_status, LT_ERR_CORRUPT_STREAM);
+      continue;
+    }
+    const uint64_t nbytes = b1 - b0;  // the chunk's bytes
+    uint32_t done = 0;                // elements accounted for (zero runs and literals)
+    uint64_t q = 0;                   // byte offset of the window in the chunk (even)
+    uint32_t p = 0;                   // next record start, in 16-bit slots from q
+    uint32_t lit_rem = 0, lit_out = 0;  // literals carried over from the previous window
+    int err = 0;
+    // every iteration moves q forward by at least 4 bytes: bounded by nbytes
+    while (done < len || lit_rem) {
+      if (q >= nbytes) {
         err = LT_ERR_SIZE_MISMATCH;
-        walking = false;
         break;
       }
-      const uint32_t zr = field(p);
-      const uint32_t nl = field(p + 2);
-      p += 4;
-      if ((uint64_t)pos + zr + nl > len || p + 2 * (uint64_t)nl > nb) {
-        err = LT_ERR_CORRUPT_STREAM;
-        walking = false;
-        break;
-      }
-      zrem = zr;
-      lrem = nl;
-      lsrc = p;
-      p += 2 * (uint64_t)nl;
-    }
-    __syncwarp();
-    // 2. the warp stores stripe r of each of its 32 chunks: 32 x 16 bytes each
-    for (int j = 0; j < 32; ++j) {
-      const uint32_t len_j = __shfl_sync(0xFFFFFFFFu, len, j);
-      if (s0 >= len_j) continue;  // warp-uniform
-      const uint32_t m = (len_j - s0) < kStripe ? (len_j - s0) : kStripe;
-      uint16_t *dst = out + (c0 + j) * (int64_t)chunk + s0;
-      uint4 *tv = reinterpret_cast<uint4 *>(wt + j * kPitch) + lane;
-      const uint32_t e = 8 * (uint32_t)lane;
-      if (e < m) {
-        const uint4 v = *tv;
-        if (VEC && e + 8 <= m) {
-          st_u128(dst + e, v);
-        } else {
-          const uint16_t *h = reinterpret_cast<const uint16_t *>(&v);
-          for (uint32_t q = 0; q < 8 && e + q < m; ++q) dst[e + q] = h[q];
+      // window: chunk bytes [q, q + 128) as 64 u16 slots; lane l holds slots
+      // 2l, 2l + 1 in `pair` and slots 2l + 1, 2l + 2 in `podd`
+      const uint64_t A = b0 + q;  // absolute byte index of slot 0
+      const uint64_t al = A & ~uint64_t(3);
+      const uint32_t sh = (uint32_t)(A & 3) * 8;
+      const uint32_t w0 = load_word(enc, al + 4 * (uint64_t)lane, enc_bytes);
+      const uint32_t w33 = (lane == 31) ? load_word(enc, al + 128, enc_bytes) : 0u;
+      const uint32_t w34 = (lane == 31) ? load_word(enc, al + 132, enc_bytes) : 0u;
+      uint32_t w1 = __shfl_down_sync(0xFFFFFFFFu, w0, 1);
+      if (lane == 31) w1 = w33;
+      const uint32_t pair = __funnelshift_r(w0, w1, sh);  // slots 2*lane, 2*lane + 1
+      uint32_t pnext = __shfl_down_sync(0xFFFFFFFFu, pair, 1);
+      if (lane == 31) pnext = __funnelshift_r(w33, w34, sh);  // slots 64, 65
+      const uint32_t podd = __funnelshift_r(pair, pnext, 16);  // slots 2*lane + 1, 2*lane + 2
+      const uint64_t win_bytes = (nbytes - q) < kWin ? (nbytes - q) : kWin;
+      const uint32_t win_slots = (uint32_t)(win_bytes / 2);
+
+      // 1. literals carried over from a record that began in an earlier window
+      if (lit_rem) {
+        const uint32_t take = lit_rem < win_slots ? lit_rem : win_slots;
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t s = 2 * lane + h;
+          if (s < take) o[lit_out + s] = (uint16_t)(h ? (pair >> 16) : (pair & 0xFFFFu));
         }
-        *tv = make_uint4(0u, 0u, 0u, 0u);
+        lit_rem -= take;
+        lit_out += take;
+        if (lit_rem) {  // the whole window was literals
+          if (win_slots < 64) {
+            err = LT_ERR_CORRUPT_STREAM;
+            break;
+          }
+          q += kWin;
+          p -= 64;
+          continue;
+        }
+      }
+      // 2. walk the records whose header lies in this window and in the
+      //    chunk's bytes, until the chunk is accounted for; record k's slot
+      //    and header go to lane k
+      const int32_t lim = nbytes >= q + 4 ? (int32_t)((nbytes - q - 4) / 2 < 62 ? (nbytes - q - 4) / 2 : 62) : -1;
+      const uint32_t rem = len - done;
+      uint32_t pp = p, k = 0, dsum = 0, myP = 0, myV = 0;
+      while ((int32_t)pp <= lim && dsum < rem) {  // at most 32 records: each takes >= 2 slots
+        const uint32_t v = __shfl_sync(0xFFFFFFFFu, (pp & 1) ? podd : pair, (int)(pp >> 1));
+        if (lane == k) {
+          myP = pp;
+          myV = v;
+        }
+        ++k;
+        dsum += (v & 0xFFFFu) + (v >> 16);
+        pp += 2 + (v >> 16);
+      }
+      // 3. the walked records, in parallel
+      const bool rec = lane < k;
+      const uint32_t zr = myV & 0xFFFFu, nl = myV >> 16;
+      const uint32_t lk = rec ? zr + nl : 0u;
+      uint32_t incl = lk;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if ((int)lane >= off) incl += t;
+      }
+      const uint32_t before = incl - lk;  // elements of the window's earlier records
+      const bool bad = rec && ((uint64_t)done + before + lk > len || q + 2 * ((uint64_t)myP + 2 + nl) > nbytes);
+      const unsigned badm = __ballot_sync(0xFFFFFFFFu, bad);
+      const uint32_t ok = badm ? (uint32_t)(__ffs(badm) - 1) : k;  // records before the first bad one
+      const bool live = lane < ok;
+      const uint32_t mlo = __reduce_or_sync(0xFFFFFFFFu, live && myP < 32 ? 1u << myP : 0u);
+      const uint32_t mhi = __reduce_or_sync(0xFFFFFFFFu, live && myP >= 32 ? 1u << (myP - 32) : 0u);
+      const uint32_t lend = myP + 2 + nl < 64 ? myP + 2 + nl : 64u;
+      const uint32_t span = (myP + 2) | (lend << 16);     // the record's literal slots in this window
+      const uint32_t obase = done + before + zr - (myP + 2);  // output index of literal slot s: obase + s
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t s = 2 * lane + h;  // the slot this lane holds
+        const uint32_t cnt = __popc(mlo & (s >= 31 ? 0xFFFFFFFFu : (2u << s) - 1u)) +
+                             (s >= 32 ? __popc(mhi & (s == 63 ? 0xFFFFFFFFu : (2u << (s - 32)) - 1u)) : 0);
+        const int r = cnt ? (int)cnt - 1 : 0;  // the last record starting at or before s
+        const uint32_t sp = __shfl_sync(0xFFFFFFFFu, span, r);
+        const uint32_t ob = __shfl_sync(0xFFFFFFFFu, obase, r);
+        if (cnt && s >= (sp & 0xFFFFu) && s < (sp >> 16)) o[ob + s] = (uint16_t)(h ? (pair >> 16) : (pair & 0xFFFFu));
+      }
+      if (badm) {
+        err = LT_ERR_CORRUPT_STREAM;
+        break;
+      }
+      // 4. carry-over from the window's last record, and the next window
+      if (k) {
+        const uint32_t lastP = __shfl_sync(0xFFFFFFFFu, myP, (int)k - 1);
+        const uint32_t lastV = __shfl_sync(0xFFFFFFFFu, myV, (int)k - 1);
+        const uint32_t lastB = __shfl_sync(0xFFFFFFFFu, before, (int)k - 1);
+        const uint32_t lend_all = lastP + 2 + (lastV >> 16);
+        if (lend_all > 64) {
+          lit_rem = lend_all - 64;
+          lit_out = done + lastB + (lastV & 0xFFFFu) + (64 - lastP - 2);
+        }
+      }
+      done += dsum;
+      if (done >= len && !lit_rem) break;
+      if (done < len && (int32_t)pp <= 62 && (int32_t)pp > lim) {  // the next header does not fit in the chunk's bytes
+        err = LT_ERR_SIZE_MISMATCH;
+        break;
+      }
+      if (lit_rem) {
+        q += kWin;
+        p = pp - 64;
+      } else {
+        q += 2 * (uint64_t)pp;
+        p = 0;
       }
     }
-    __syncwarp();
+    if (err && lane == 0) report(d_status, err);
   }
-  if (err) report(d_status, err);
 }
 
 }  // namespace
@@ -218,14 +216,10 @@ LT_API lt_status lt_zrle_decode(const uint8_t *enc, uint64_t enc_bytes, const ui
   if (!aligned(chunk_offsets, 8) || !aligned(out, 2) || !aligned(d_status, 4)) return LT_ERR_MISALIGNED;
   cudaStream_t st = (cudaStream_t)stream;
   const int64_t n_chunks = (n_elements + chunk_elems - 1) / chunk_elems;
-  const int64_t grid = (n_chunks + kZThreads - 1) / kZThreads;  // one chunk per lane
-  if (grid > INT32_MAX) return LT_ERR_UNSUPPORTED;
-  // 16-byte stores when every chunk's output starts on a 16-byte boundary
-  if (aligned(out, 16) && chunk_elems % 8 == 0)
-    k_zrle<true><<<(int)grid, kZThreads, 0, st>>>(enc, enc_bytes, chunk_offsets, n_elements, chunk_elems, n_chunks,
-                                                  out, d_status);
-  else
-    k_zrle<false><<<(int)grid, kZThreads, 0, st>>>(enc, enc_bytes, chunk_offsets, n_elements, chunk_elems, n_chunks,
-                                                   out, d_status);
+  const int64_t need = (n_chunks + kWarps - 1) / kWarps;
+  const int64_t cap = (int64_t)num_sms() * blocks_per_sm((const void *)k_zrle, kThreads, 0);
+  const int grid = (int)(need < cap ? need : cap);
+  k_zrle<<<grid, kThreads, 0, st>>>(enc, enc_bytes, chunk_offsets, n_elements, chunk_elems, n_chunks, out,
+                                    d_status);
   return launch_status();
 }
