@@ -156,39 +156,6 @@ __device__ __forceinline__ void copy_match(uint8_t *win, uint32_t op, uint32_t d
   }
 }
 
-// Window bytes [dst, dst + M) = the bytes at src repeated with period P
-// (P >= M: a plain copy; P == 1: one byte), with NL cooperating lanes. The
-// source bytes [src, src + min(P, M)) lie wholly before dst and are final, so
-// every destination byte is independent of the others. Never writes a byte
-// outside [dst, dst + M).
-template <int NL>
-__device__ __forceinline__ void copy_src(uint8_t *win, uint32_t dst, uint32_t src, uint32_t P, uint32_t M, int lid) {
-  if (P >= M) {
-    const uint32_t sh = src - dst;  // modulo 2^32: x + sh = x - (dst - src)
-    write_span<NL>(
-        win, dst, dst + M, lid, [&](uint32_t x) { return win[x + sh]; },
-        [&](uint32_t x) { return gather4_window(win, (int32_t)(x + sh)); });
-  } else if (P == 1) {
-    const uint32_t bv = win[src];
-    const uint32_t v = 0x01010101u * bv;
-    write_span<NL>(
-        win, dst, dst + M, lid, [&](uint32_t) { return (uint8_t)bv; }, [&](uint32_t) { return v; });
-  } else {
-    write_span<NL>(
-        win, dst, dst + M, lid, [&](uint32_t x) { return win[src + (x - dst) % P]; },
-        [&](uint32_t x) {
-          const uint32_t u = (x - dst) % P;
-          if (u + 4 <= P) return gather4_window(win, (int32_t)(src + u));
-          uint32_t w = 0, uu = u;
-          for (int i = 0; i < 4; ++i) {
-            w |= (uint32_t)win[src + uu] << (8 * i);
-            if (++uu == P) uu = 0;
-          }
-          return w;
-        });
-  }
-}
-
 // ---------------------------------------------------------------------------
 // 1. parse: one warp walks one block
 // ---------------------------------------------------------------------------
@@ -653,11 +620,7 @@ struct Seqs {
     } m;
   } u;
   uint32_t tail_level;  // levels from here on hold at most kTailMatches matches in all
-  uint32_t lmax_now;    // the highest level left after the sources are resolved
 };
-
-constexpr uint32_t kRle = 0x80000000u;  // resolved source flag: period 1 (one byte repeated)
-constexpr int kResolveRounds = 16;
 
 // Rebuild one block whose sequence index is in the workspace (n <= kCap
 // sequences, staged in place by the parse's rule). All threads of the CTA.
@@ -798,56 +761,6 @@ __device__ __forceinline__ int resolve_block(uint8_t *win, Seqs &S, const uint8_
     }
     return kResolved;
   }
-  // c0. Resolve each match's source through the matches that produced it.
-  // Match j copies its bytes from [dst - d, ...) with period d. When that
-  // source lies wholly inside the output of an earlier match k, the same
-  // bytes are k's source bytes: j's source moves there (keeping j's period,
-  // or period 1 when k repeats one byte). Rounds of this (each reads the
-  // others' current sources; an old and a new source describe the same
-  // bytes) move sources back until they lie in literals -- such a match only
-  // needs the literal rounds and goes to level 1 -- or straddle sequences.
-  // A moved source is still inside the bytes the old one depended on, so the
-  // parse's levels stay valid for every other match. S.le (free after the
-  // literal rounds) holds the source start, with kRle for period 1.
-  __syncthreads();
-  for (uint32_t j = tid; j < n; j += kThreads) {
-    const uint32_t d = S.dist[j];
-    S.le[j] = d ? ((S.md[j] - d) | (d == 1 ? kRle : 0u)) : 0u;
-  }
-  if (tid == 0) S.lmax_now = 0;
-  __syncthreads();
-  for (int round = 0; round < kResolveRounds; ++round) {
-    bool changed = false;
-    for (uint32_t j = tid; j < n; j += kThreads) {
-      if (!S.dist[j] || S.lvl[j] <= 1) continue;
-      const uint32_t mj = S.le[j];
-      const uint32_t src = mj & ~kRle;
-      const uint32_t P = (mj & kRle) ? 1u : S.dist[j];
-      const uint32_t M = S.op[j + 1] - S.md[j];
-      const uint32_t need = P < M ? P : M;
-      const uint32_t k = upper_bound(S.op, n, src) - 1;  // the sequence whose output holds src (op[0] = 0)
-      if (src + need <= S.md[k]) {  // inside k's literals: only the literal rounds before it
-        S.lvl[j] = 1;
-        changed = true;
-        continue;
-      }
-      if (src < S.md[k] || src + need > S.op[k + 1] || !S.dist[k]) continue;  // straddles: stays
-      const uint32_t mk = S.le[k];
-      const uint32_t off = src - S.md[k];
-      if (mk & kRle) {  // k repeats one byte: so does j's source
-        S.le[j] = mk;
-        changed = true;
-      } else if (off + need <= S.dist[k]) {  // within one period of k's source
-        S.le[j] = ((mk & ~kRle) + off) | (mj & kRle);
-        changed = true;
-      }
-    }
-    if (!__syncthreads_or(changed)) break;
-  }
-  for (uint32_t j = tid; j < n; j += kThreads)
-    if (S.dist[j]) atomicMax(&S.lmax_now, (uint32_t)S.lvl[j]);
-  __syncthreads();
-  lmax = S.lmax_now;
   // counting sort of the matches by level into S.u.m.order
   for (uint32_t i = tid; i <= kLevelCap; i += kThreads) S.u.m.start[i] = 0;
   __syncthreads();
@@ -902,8 +815,8 @@ __device__ __forceinline__ int resolve_block(uint8_t *win, Seqs &S, const uint8_
       const uint32_t i = base + (uint32_t)sub;
       if (i < end) {
         const uint32_t j = S.u.m.order[i];
-        const uint32_t md = S.md[j], mj = S.le[j];
-        copy_src<8>(win, md, mj & ~kRle, (mj & kRle) ? 1u : S.dist[j], S.op[j + 1] - md, lane & 7);
+        const uint32_t md = S.md[j];
+        copy_match<8>(win, md, S.dist[j], S.op[j + 1] - md, lane & 7, 0xFFu << (8 * sub));
       }
       __syncwarp();
     }
@@ -916,8 +829,8 @@ __device__ __forceinline__ int resolve_block(uint8_t *win, Seqs &S, const uint8_
         const uint32_t i = base + (uint32_t)sub;
         if (i < end) {
           const uint32_t j = S.u.m.order[i];
-          const uint32_t md = S.md[j], mj = S.le[j];
-          copy_src<8>(win, md, mj & ~kRle, (mj & kRle) ? 1u : S.dist[j], S.op[j + 1] - md, lane & 7);
+          const uint32_t md = S.md[j];
+          copy_match<8>(win, md, S.dist[j], S.op[j + 1] - md, lane & 7, 0xFFu << (8 * sub));
         }
         __syncwarp();
       }
