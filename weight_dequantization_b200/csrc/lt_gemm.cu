@@ -10,23 +10,26 @@
 // One CTA computes a 128 x 256 tile of out over a range of K (the whole of
 // K, or a split of it whose fp32 partial sums a second kernel adds in a
 // fixed order). Warp roles:
-//   warp 0      TMA producer: for each 64-wide K step, one tiled bulk copy of
-//               the x tile (128 x 64 fp16, 128-byte swizzle) and one of the
-//               packed INT4 tile (64 rows x 128 bytes, 128-byte swizzle) into
-//               a 4-deep ring, completion counted on an mbarrier;
-//   warps 2..9  decoders: turn the packed tile into the fp16 B operand in
+//   warp 0      packed-W producer: for each 64-wide K step one tiled bulk
+//               copy (TMA) of the packed INT4 tile (64 rows x 128 bytes,
+//               128-byte swizzle) into an 8-deep ring, completion counted on
+//               an mbarrier; a slot is refilled as soon as the decoders are
+//               done with it, so this stream runs well ahead of the MMAs;
+//   warp 2      x producer: the x tile (128 x 64 fp16, 128-byte swizzle) of
+//               each step into a 3-deep ring, refilled when the MMAs that
+//               read a slot have completed;
+//   warps 3..18 decoders: turn the packed tile into the fp16 B operand in
 //               shared memory (N-major, 128-byte swizzle), with the exact
 //               half2 arithmetic of lt_dequant_int4 (bit-identical to it), in
-//               a 3-deep ring; scales and zero points of the next step are
-//               loaded while the current one is decoded;
+//               a 2-deep ring; scales and zero points are loaded three steps
+//               before their use;
 //   warp 1      MMA issuer: one thread issues tcgen05.mma kind::f16 (fp32
 //               accumulator in tensor memory, 128 x 256 = 256 columns), four
 //               K = 16 instructions per step, and tcgen05.commit releases the
 //               ring slots;
-//   warps 2..9  epilogue: tcgen05.ld of the accumulator (warp w reads lanes
-//               32 (w % 4) ..., warps 2..5 columns 0..127, warps 6..9
-//               columns 128..255), conversion to binary16 (or the fp32
-//               partial of a split), 16-byte stores.
+//   warps 3..18 epilogue: tcgen05.ld of the accumulator (warp w reads lanes
+//               32 (w % 4) ... and a quarter of the columns), conversion to
+//               binary16 (or the fp32 partial of a split), 16-byte stores.
 // Every mbarrier wait is bounded (about a second of clock); a wait that runs
 // out sets LT_ERR_TIMEOUT in the status word and the CTA winds down: the
 // producer waits (bounded) for its copies in flight, the tensor memory is
@@ -35,23 +38,27 @@
 
 #include <cuda.h>
 #include <mutex>
+#include <type_traits>
 
 namespace lt {
 namespace {
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
-constexpr int kStagesIn = 4;  // x + packed-W slots (TMA)
-constexpr int kStagesB = 3;   // decoded-B slots
-constexpr int kDecWarps = 8;
+constexpr int kStagesW = 8;  // packed-W slots (TMA; freed by the decoders)
+constexpr int kStagesX = 3;  // x slots (TMA; freed by the MMAs)
+constexpr int kStagesB = 2;  // decoded-B slots
+constexpr int kDecWarps = 16;
+constexpr int kDec0 = 3;     // first decoder warp (0: packed-W producer, 1: MMA, 2: x producer)
 constexpr int kUnits = (kBK * kBN / 32) / (kDecWarps * 32);  // 16-byte packed chunks per decoder thread per step
-constexpr int kGemmThreads = (2 + kDecWarps) * 32;
+static_assert(kUnits * kDecWarps * 32 == kBK * kBN / 32, "decoder units must cover a packed tile");
+constexpr int kGemmThreads = (kDec0 + kDecWarps) * 32;
 constexpr uint32_t kABytes = kBM * kBK * 2;   // 16384
 constexpr uint32_t kWBytes = kBK * kBN / 2;   // 8192
 constexpr uint32_t kBBytes = kBN * kBK * 2;   // 32768
 constexpr uint32_t kSmemA = 0;
-constexpr uint32_t kSmemW = kSmemA + kStagesIn * kABytes;
-constexpr uint32_t kSmemB = kSmemW + kStagesIn * kWBytes;
-constexpr uint32_t kSmemTotal = kSmemB + kStagesB * kBBytes;  // 192 KB
+constexpr uint32_t kSmemW = kSmemA + kStagesX * kABytes;
+constexpr uint32_t kSmemB = kSmemW + kStagesW * kWBytes;
+constexpr uint32_t kSmemTotal = kSmemB + kStagesB * kBBytes;  // 176 KB
 constexpr uint32_t kSmemDyn = kSmemTotal + 1024;              // + alignment slack
 constexpr uint32_t kTmemCols = 256;
 // B operand (N-major, 128-byte swizzle): 1 KB atoms of 64 n x 8 k; atoms
@@ -149,8 +156,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
                                                                  const __grid_constant__ GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t bar_full[kStagesIn], bar_aempty[kStagesIn], bar_bfull[kStagesB],
-      bar_bempty[kStagesB], bar_acc;
+  __shared__ __align__(8) uint64_t bar_wfull[kStagesW], bar_wempty[kStagesW], bar_xfull[kStagesX],
+      bar_xempty[kStagesX], bar_bfull[kStagesB], bar_bempty[kStagesB], bar_acc;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -162,9 +169,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
   const int n_it = it_end - it_begin;
 
   if (tid == 0) {
-    for (int s = 0; s < kStagesIn; ++s) {
-      mbar_init(smem_u32(&bar_full[s]), 1);
-      mbar_init(smem_u32(&bar_aempty[s]), 1 + kDecWarps);
+    for (int s = 0; s < kStagesW; ++s) {
+      mbar_init(smem_u32(&bar_wfull[s]), 1);
+      mbar_init(smem_u32(&bar_wempty[s]), kDecWarps);
+    }
+    for (int s = 0; s < kStagesX; ++s) {
+      mbar_init(smem_u32(&bar_xfull[s]), 1);
+      mbar_init(smem_u32(&bar_xempty[s]), 1);
     }
     for (int b = 0; b < kStagesB; ++b) {
       mbar_init(smem_u32(&bar_bfull[b]), kDecWarps);
@@ -190,44 +201,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
     s_abort = 1;
     report(a.d_status, LT_ERR_TIMEOUT);
   };
+  // one TMA stream: step it's tile into slot it % STAGES once that slot is
+  // free again (its empty barrier completed STAGES steps earlier); on an abort,
+  // wait (bounded) for the copies in flight before the CTA exits
+  auto produce = [&](auto stages_c, uint64_t *full, uint64_t *empty, uint32_t slot0, uint32_t bytes, auto issue) {
+    constexpr int STAGES = decltype(stages_c)::value;
+    int issued = 0;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it % STAGES;
+      if (it >= STAGES && !mbar_wait(smem_u32(&empty[s]), ((it / STAGES) - 1) & 1)) {
+        fail();
+        break;
+      }
+      if (*(volatile int *)&s_abort) break;
+      mbar_expect_tx(smem_u32(&full[s]), bytes);
+      issue(slot0 + s * bytes, (it_begin + it) * kBK, smem_u32(&full[s]));
+      issued = it + 1;
+    }
+    if (*(volatile int *)&s_abort)
+      for (int it = issued > STAGES ? issued - STAGES : 0; it < issued; ++it)
+        mbar_wait(smem_u32(&full[it % STAGES]), (it / STAGES) & 1);
+  };
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      int issued = 0;
-      for (int it = 0; it < n_it; ++it) {
-        const int s = it % kStagesIn;
-        if (it >= kStagesIn && !mbar_wait(smem_u32(&bar_aempty[s]), ((it / kStagesIn) - 1) & 1)) {
-          fail();
-          break;
-        }
-        if (*(volatile int *)&s_abort) break;
-        const uint32_t full = smem_u32(&bar_full[s]);
-        mbar_expect_tx(full, kABytes + kWBytes);
-        const int32_t kk = (it_begin + it) * kBK;
-        tma_load_2d(sbase + kSmemA + s * kABytes, &map_x, kk, (int32_t)m0, full);
-        tma_load_2d(sbase + kSmemW + s * kWBytes, &map_w, (int32_t)(n0 / 2), kk, full);
-        issued = it + 1;
-      }
-      if (*(volatile int *)&s_abort) {  // let the copies in flight land before the CTA exits
-        for (int it = issued > kStagesIn ? issued - kStagesIn : 0; it < issued; ++it)
-          mbar_wait(smem_u32(&bar_full[it % kStagesIn]), (it / kStagesIn) & 1);
-      }
-    }
+    // ---------------- packed-W producer: runs up to 8 steps ahead ----------------
+    if (lane == 0)
+      produce(std::integral_constant<int, kStagesW>{}, bar_wfull, bar_wempty, sbase + kSmemW, kWBytes,
+              [&](uint32_t dst, int32_t kk, uint32_t bar) { tma_load_2d(dst, &map_w, (int32_t)(n0 / 2), kk, bar); });
+  } else if (warp == 2) {
+    // ---------------- x producer ----------------
+    if (lane == 0)
+      produce(std::integral_constant<int, kStagesX>{}, bar_xfull, bar_xempty, sbase + kSmemA, kABytes,
+              [&](uint32_t dst, int32_t kk, uint32_t bar) { tma_load_2d(dst, &map_x, kk, (int32_t)m0, bar); });
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       // kind::f16, fp32 accumulator, A and B fp16, A K-major, B N-major, N = 256, M = 128
       const uint32_t idesc = (1u << 4) | (1u << 16) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
       for (int it = 0; it < n_it; ++it) {
-        const int s = it % kStagesIn, b = it % kStagesB;
-        if (!mbar_wait(smem_u32(&bar_bfull[b]), (it / kStagesB) & 1)) {
+        const int sx = it % kStagesX, b = it % kStagesB;
+        if (!mbar_wait(smem_u32(&bar_xfull[sx]), (it / kStagesX) & 1) ||
+            !mbar_wait(smem_u32(&bar_bfull[b]), (it / kStagesB) & 1)) {
           fail();
           break;
         }
         if (*(volatile int *)&s_abort) break;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t a0 = sbase + kSmemA + s * kABytes, b0 = sbase + kSmemB + b * kBBytes;
+        const uint32_t a0 = sbase + kSmemA + sx * kABytes, b0 = sbase + kSmemB + b * kBBytes;
 #pragma unroll
         for (int ks = 0; ks < kBK / 16; ++ks) {
           // A: K-major 128-byte swizzle, 8-row atoms 1 KB apart, K = 16 slice at +32 bytes;
@@ -236,14 +256,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
           const uint64_t bd = smem_desc(b0 + 2u * kBAtomK * ks, kBAtomN, kBAtomK);
           mma_f16(tmem, ad, bd, idesc, (it | ks) != 0);
         }
-        mma_commit(smem_u32(&bar_aempty[s]));
+        mma_commit(smem_u32(&bar_xempty[sx]));
         mma_commit(smem_u32(&bar_bempty[b]));
       }
       mma_commit(smem_u32(&bar_acc));  // the accumulator is final (or abandoned) once this arrives
     }
   } else {
     // ---------------- decoders (then epilogue) ----------------
-    const int dt = tid - 64;  // 0 .. 32 kDecWarps - 1
+    const int dt = tid - 32 * kDec0;  // 0 .. 32 kDecWarps - 1
     const int klo = dt & 7, h = (dt >> 3) & 7, khi0 = dt >> 6;  // unit i: row klo + 8 (khi0 + (kDecWarps / 2) i)
     const int64_t NG = a.N / a.group_size;
     const int64_t gcol = (n0 + 32 * h) / a.group_size;  // this thread's group column
@@ -267,8 +287,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
     // one K step: wait for its packed tile and a free B slot, decode with
     // (sc, zr), refill (sc, zr) for step it + 3, hand the slot to the MMA
     auto step = [&](int it, uint32_t(&sc)[kUnits], uint32_t(&zr)[kUnits]) -> bool {
-      const int s = it % kStagesIn, b = it % kStagesB;
-      if (!mbar_wait(smem_u32(&bar_full[s]), (it / kStagesIn) & 1) ||
+      const int s = it % kStagesW, b = it % kStagesB;
+      if (!mbar_wait(smem_u32(&bar_wfull[s]), (it / kStagesW) & 1) ||
           (it >= kStagesB && !mbar_wait(smem_u32(&bar_bempty[b]), ((it / kStagesB) - 1) & 1))) {
         fail();
         return false;
@@ -298,7 +318,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(smem_u32(&bar_aempty[s]));
+        mbar_arrive(smem_u32(&bar_wempty[s]));
         mbar_arrive(smem_u32(&bar_bfull[b]));
       }
       return true;
@@ -315,8 +335,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
     if (acc_ok && !*(volatile int *)&s_abort && n_it > 0) {
       const int quarter = warp & 3;  // tensor-memory lanes 32 quarter .. + 31
       const int64_t m = m0 + 32 * quarter + lane;
-      const int cbeg = warp < 6 ? 0 : kBN / 2;  // each quarter's columns split between two warps
-      for (int c0 = cbeg; c0 < cbeg + kBN / 2; c0 += 32) {
+      // each quarter's 256 columns split among its kDecWarps / 4 decoder warps
+      constexpr int kCols = kBN / (kDecWarps / 4);
+      const int cbeg = ((warp - kDec0) / 4) * kCols;
+      for (int c0 = cbeg; c0 < cbeg + kCols; c0 += 32) {
         uint32_t r[32];
         tmem_ld32(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0, r);
         if (m < a.M) {
@@ -378,12 +400,13 @@ encode_tiled_t encoder() {
   return fn;
 }
 
-// split count for a grid of `tiles` output tiles and k_iters K steps: enough
-// CTAs to cover the SMs about once, each split at least 4 steps
+// split count for a grid of `tiles` output tiles and k_iters K steps: as
+// many CTAs as fit in one wave over the SMs (one CTA per SM), each split at
+// least 4 steps
 int choose_splits(int64_t tiles, int64_t k_iters) {
   const int64_t sms = num_sms();
   if (tiles >= sms || k_iters < 8) return 1;
-  int64_t s = (sms + tiles - 1) / tiles;
+  int64_t s = sms / tiles;
   const int64_t max_s = k_iters / 4;
   if (s > max_s) s = max_s;
   if (s > 32) s = 32;
