@@ -1062,6 +1062,60 @@ def checksum_timing(dw, hw, peak: float, reps: int = 20, warmup: int = 3):
             "checked_overhead": t_checked / t_plain - 1.0}
 
 
+def lz4_cliff_timing(dw, hw, reps: int = 10, warmup: int = 2):
+    """Blocks with more LZ4 sequences than the index holds (512 per block),
+    which the expanding CTA walks itself: 448 blocks of 64 KB (C4's count)
+    of bytes uniform over 4 values, compressed by the generator's LZ4 into
+    ~15,000 short sequences per block; raw decode (lt_lz4_decode) timed
+    against the raw decode of C4's own compressed stream (~335 sequences per
+    block). Device time by CUDA events, median of `reps`, L2 flushed before
+    each call."""
+    import numpy as np
+    import torch
+
+    from weight_dequantization_b200 import lt_decode as L
+    from weight_dequantization_b200.synth import lz4_compress_blocks, u8_uniform
+
+    nb = 448
+    raw = u8_uniform(9, nb * 65536, 0, 3)
+    comp, offs = lz4_compress_blocks(raw, 65536)
+    dcomp = torch.from_numpy(comp).cuda()
+    doffs = torch.from_numpy(offs.view(np.int64)).cuda()
+    out = torch.empty(nb * 65536, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(L.lt_lz4_workspace_bytes(nb), dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    s = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    c4 = hw["C4"]
+    out4 = torch.empty(c4["packed_bytes"], dtype=torch.uint8, device="cuda")
+
+    def timed(fn):
+        ts = []
+        for r in range(warmup + reps):
+            flush.fill_(r & 0xFF)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            fn()
+            e1.record(s)
+            torch.cuda.synchronize()
+            if r >= warmup:
+                ts.append(e0.elapsed_time(e1) / 1e3)
+        return statistics.median(ts)
+
+    t_many = timed(lambda: L.lt_lz4_decode(dcomp, int(comp.size), doffs, 65536, out, nb * 65536, ws, st, s))
+    t_c4 = timed(lambda: L.lt_lz4_decode(dw.c4["comp"], int(c4["comp"].size), dw.c4["offsets"], 65536, out4,
+                                         c4["packed_bytes"], dw.ws, st, s))
+    torch.cuda.synchronize()
+    ok = int(st.item()) == 0 and bool(torch.equal(out, torch.from_numpy(raw).cuda()))
+    del flush
+    return {"label": f"LZ4 blocks beyond the 512-sequence index ({nb} x 64 KB of bytes uniform on 4 values, "
+                     f"{comp.size} compressed bytes) against C4's stream, raw decode; L2 flushed before each call",
+            "us_many_sequences": t_many * 1e6, "GBps_many_sequences": nb * 65536 / t_many / 1e9,
+            "us_c4_raw": t_c4 * 1e6, "GBps_c4_raw": c4["packed_bytes"] / t_c4 / 1e9,
+            "slowdown": t_many / t_c4, "output_matches_input": ok}
+
+
 def stream_api_timing(hw, reps: int = 3):
     """The streaming API (LayerStreamer) over the C5 layers against
     sequential loading: streamed = each layer's host-to-device copy overlaps
@@ -1268,6 +1322,7 @@ def run_lt(args, rank, world, local):
         gemm = gemm_timing(peak, shapes=gshapes, batch=tuple(int(m) for m in args.gemm_m.split(","))) \
             if "G" in only else None
         csum = checksum_timing(dw, hw, peak) if "C4" in hw else None
+        cliff = lz4_cliff_timing(dw, hw) if "C4" in hw else None
         if vd is not None and world == 1 and not args.no_cpu_baseline:
             vd["cpu_baseline"] = cpu_baseline_value_dict()
         result = {
@@ -1278,7 +1333,7 @@ def run_lt(args, rank, world, local):
             "gpu_launches": nlaunch * K, "clocks": {"sm_mhz": ck["sm_mhz"], "sm_max_mhz": ck["sm_max_mhz"],
                                                      "reasons": ck["reasons"], "samples": ck["samples"]},
             "per_codec": per_codec, "c1_graph": c1g, "value_dict": vd, "cpu_baseline_threads": cpu_thr,
-            "parity": parity, "stream_api": sapi, "gemm": gemm, "checksum": csum,
+            "parity": parity, "stream_api": sapi, "gemm": gemm, "checksum": csum, "lz4_many_sequences": cliff,
             "impl": "lt",
         }
     if dist is not None:
