@@ -544,47 +544,79 @@ __global__ void __launch_bounds__(32) k_lz4_parse_staged(const __grid_constant__
 // fallback: warp 0 walks the block from global memory itself (lockstep,
 // warp-uniform control flow). Returns 0 or a stream status.
 // ---------------------------------------------------------------------------
-__device__ int walk_block_warp(const uint8_t *__restrict__ src, uint64_t ilen, uint8_t *win, uint32_t olen,
-                               int lane) {
+__device__ int walk_block_warp(const uint8_t *__restrict__ src, uint64_t ilen, uint8_t *win, uint32_t olen, int lane,
+                               uint8_t *ring) {
   if (ilen == 0) return olen == 0 ? 0 : LT_ERR_SIZE_MISMATCH;
+  if (ilen > 0x7FFFFFFFull) return LT_ERR_CORRUPT_STREAM;  // no valid block of <= 64 KB is this long
+  // the block's bytes stream through the parse's 2 KB cp.async ring (in
+  // `ring`), so that each header read is a shared-memory read, not a
+  // dependent global load
+  WarpRing r;
+  r.buf = ring;
+  r.lane = lane;
+  r.beg = src;
+  r.end = src + ilen;
+  r.a0 = reinterpret_cast<const uint8_t *>(reinterpret_cast<uintptr_t>(src) & ~uintptr_t(15));
+  r.total = (uint32_t)((r.end - r.a0 + kPChunk - 1) / kPChunk);
+  r.issued = 0;
+  r.done = 0;
+  r.top_up(0);
+  const uint32_t lead = (uint32_t)(src - r.a0);
+  auto byte = [&](uint64_t x) -> uint32_t {  // warp-uniform x < ilen
+    const uint32_t rel = lead + (uint32_t)x;
+    r.need(rel, rel + 1);
+    return r.at(rel);
+  };
   uint64_t ip = 0;
   uint32_t op = 0;
+  int st = 0;
   for (;;) {
-    if (ip >= ilen) return LT_ERR_CORRUPT_STREAM;
-    const uint32_t token = __ldg(src + ip++);
+    if (ip >= ilen) { st = LT_ERR_CORRUPT_STREAM; break; }
+    const uint32_t token = byte(ip++);
     uint64_t lit = token >> 4;
     if (lit == 15) {
       uint32_t bb;
       do {
-        if (ip >= ilen || lit > olen) return LT_ERR_CORRUPT_STREAM;
-        bb = __ldg(src + ip++);
+        if (ip >= ilen || lit > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
+        bb = byte(ip++);
         lit += bb;
       } while (bb == 255);
+      if (st) break;
     }
-    if (ip + lit > ilen || (uint64_t)op + lit > olen) return LT_ERR_CORRUPT_STREAM;
-    for (uint32_t i = lane; i < (uint32_t)lit; i += 32) win[op + i] = __ldg(src + ip + i);
+    if (ip + lit > ilen || (uint64_t)op + lit > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
+    for (uint32_t done = 0; done < (uint32_t)lit; done += 32) {  // the literals, 32 bytes at a time
+      const uint32_t rel = lead + (uint32_t)ip + done;
+      const uint32_t q = ((uint32_t)lit - done) < 32u ? ((uint32_t)lit - done) : 32u;
+      r.need(rel, rel + q);
+      if ((uint32_t)lane < q) win[op + done + lane] = (uint8_t)r.at(rel + lane);
+    }
     ip += lit;
     op += (uint32_t)lit;
     __syncwarp();
     if (ip == ilen) break;
-    if (ip + 2 > ilen) return LT_ERR_CORRUPT_STREAM;
-    const uint32_t d = (uint32_t)__ldg(src + ip) | ((uint32_t)__ldg(src + ip + 1) << 8);
+    if (ip + 2 > ilen) { st = LT_ERR_CORRUPT_STREAM; break; }
+    const uint32_t d0 = byte(ip), d1 = byte(ip + 1);
+    const uint32_t d = d0 | (d1 << 8);
     ip += 2;
-    if (d == 0 || d > op) return LT_ERR_CORRUPT_STREAM;
+    if (d == 0 || d > op) { st = LT_ERR_CORRUPT_STREAM; break; }
     uint64_t mlen = (token & 15u) + 4;
     if ((token & 15u) == 15u) {
       uint32_t bb;
       do {
-        if (ip >= ilen || mlen > olen) return LT_ERR_CORRUPT_STREAM;
-        bb = __ldg(src + ip++);
+        if (ip >= ilen || mlen > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
+        bb = byte(ip++);
         mlen += bb;
       } while (bb == 255);
+      if (st) break;
     }
-    if ((uint64_t)op + mlen > olen) return LT_ERR_CORRUPT_STREAM;
+    if ((uint64_t)op + mlen > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
     copy_match<32>(win, op, d, (uint32_t)mlen, lane, 0xFFFFFFFFu);
     __syncwarp();
     op += (uint32_t)mlen;
   }
+  cp_async_wait<0>();  // nothing may land in the ring after this block
+  __syncwarp();
+  if (st) return st;
   return op == olen ? 0 : LT_ERR_SIZE_MISMATCH;
 }
 
@@ -612,7 +644,7 @@ struct Seqs {
   uint32_t le[kCap];      // end of its literal run in the block
   uint16_t dist[kCap];    // its match offset (0: no match)
   uint16_t lvl[kCap];     // its match level (0: no match)
-  union {
+  union alignas(16) {  // (16-byte aligned: the checked decode keeps 8-byte hash terms in it)
     uint16_t seg[kMaxWindow / 256];  // literals: last sequence starting at or before byte 256 s
     struct {
       uint32_t start[kLevelCap + 1];  // matches: first slot of each level in `order` (level counts first)
@@ -860,9 +892,15 @@ __device__ __noinline__ bool block_hash_differs(const Batch &batch, const Job &j
 }
 
 // The same check on the block's staged copy in shared memory: window bytes
-// [S0, S0 + ilen). Out of line for the same reason.
+// [S0, S0 + ilen), by the whole CTA (every thread calls it and gets the
+// answer). The terms of up to kHashChunk scramble intervals are computed by
+// the eight warps side by side into `terms` (kHashChunk x 8 words of shared
+// memory), then warp 0 applies them in order. Out of line for the same
+// reason as above.
+constexpr int kHashChunk = 24;
 __device__ __noinline__ bool staged_hash_differs(const Batch &batch, const uint8_t *win, uint32_t S0, uint32_t ilen,
-                                                 int64_t blk, int lane) {
+                                                 int64_t blk, uint64_t *terms, uint32_t *flag) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // 8 bytes of the staged block at offset off: two aligned 8-byte loads (the
   // window is 16-byte aligned and padded past its end)
   auto rd = [&](uint64_t off) -> uint64_t {
@@ -871,13 +909,31 @@ __device__ __noinline__ bool staged_hash_differs(const Batch &batch, const uint8
     return sh ? (w[0] >> sh) | (w[1] << (64u - sh)) : w[0];
   };
   const GlobalBytes dsec{batch.secret, batch.secret + batch.secret_len};
-  uint64_t h;
-  if (ilen > 240)
-    h = xxh3::hash64_long_warp(rd, [&](uint64_t off) { return dsec.rd64(batch.secret + off); }, ilen,
-                               batch.secret_len, lane);
-  else
-    h = __shfl_sync(0xFFFFFFFFu, lane == 0 ? xxh3::hash64(win + S0, ilen, batch.secret, batch.secret_len) : 0ull, 0);
-  return h != batch.expected[blk];
+  auto rk = [&](uint64_t off) { return dsec.rd64(batch.secret + off); };
+  uint64_t h = 0;
+  if (ilen <= 240) {
+    if (tid == 0) h = xxh3::hash64(win + S0, ilen, batch.secret, batch.secret_len);
+  } else {
+    const uint64_t per_block = (batch.secret_len - 64) / 8, block_len = 64 * per_block;
+    const uint64_t nb = ((uint64_t)ilen - 1) / block_len;
+    uint64_t acc = xxh3::acc_init(lane & 7);
+    const uint64_t scr = rk(batch.secret_len - 64 + 8 * (uint64_t)(lane & 7));
+    for (uint64_t c0 = 0; c0 < nb; c0 += kHashChunk) {
+      const uint64_t cn = (nb - c0) < (uint64_t)kHashChunk ? (nb - c0) : (uint64_t)kHashChunk;
+      for (uint64_t j = (uint64_t)warp; j < cn; j += kWarps) {
+        const uint64_t t = xxh3::stripe_terms(rd, rk, (c0 + j) * block_len, per_block, 0, lane);
+        if (lane < 8) terms[8 * j + lane] = t;
+      }
+      __syncthreads();
+      if (warp == 0)
+        for (uint64_t j = 0; j < cn; ++j) acc = xxh3::scramble(acc + terms[8 * j + (lane & 7)], scr);
+      __syncthreads();
+    }
+    if (warp == 0) h = xxh3::finish_long(rd, rk, acc, ilen, batch.secret_len, nb, lane);
+  }
+  if (tid == 0) *flag = h != batch.expected[blk] ? 1u : 0u;
+  __syncthreads();
+  return *flag != 0;
 }
 
 template <bool FUSED, bool CHECKED>
@@ -887,7 +943,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
   extern __shared__ uint4 smem_u4[];
   uint8_t *win = reinterpret_cast<uint8_t *>(smem_u4) + kPad;
   __shared__ Seqs S;
-  __shared__ uint32_t s_n, s_st, s_lmax, s_badsum;
+  __shared__ uint32_t s_n, s_st, s_lmax, s_badsum, s_hashflag;
   const uint32_t wcap = win_cap(batch.max_block_bytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -940,9 +996,13 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
     if (st == 0) {
       auto check_staged = [&](uint32_t S0, uint32_t ilen) -> bool {
         if (!CHECKED) return false;
-        if (warp == 0) mismatch(staged_hash_differs(batch, win, S0, ilen, blk, lane));
+        // the hash terms use the part of S.u that the literal rounds' segment
+        // table (its first 512 bytes) leaves free until the match phase
+        uint64_t *terms = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(&S.u) + 512);
+        const bool bad = staged_hash_differs(batch, win, S0, ilen, blk, terms, &s_hashflag);
+        if (warp == 0) mismatch(bad);
         __syncthreads();
-        return s_badsum != 0;
+        return bad;
       };
       const int rs = resolve_block(win, S, jb.comp + s0, (uint32_t)(s1 - s0), olen, n, lmax, wcap,
                                    desc + blk * kCap, check_staged);
@@ -954,7 +1014,8 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
     }
     if (st != 0 && warp == 0) {
       int err = LT_ERR_CORRUPT_STREAM;
-      if (s0 <= s1 && s1 <= jb.comp_bytes) err = walk_block_warp(jb.comp + s0, s1 - s0, win, olen, lane);
+      if (s0 <= s1 && s1 <= jb.comp_bytes)
+        err = walk_block_warp(jb.comp + s0, s1 - s0, win, olen, lane, reinterpret_cast<uint8_t *>(&S));
       if (err && lane == 0) report(d_status, err);  // content unspecified after an error
     }
     __syncthreads();
