@@ -16,7 +16,7 @@
 //               an mbarrier; a slot is refilled as soon as the decoders are
 //               done with it, so this stream runs well ahead of the MMAs;
 //   warp 2      x producer: the x tile (128 x 64 fp16, 128-byte swizzle) of
-//               each step into a 3-deep ring, refilled when the MMAs that
+//               each step into a 6-deep ring, refilled when the MMAs that
 //               read a slot have completed;
 //   warps 3..18 decoders: turn the packed tile into the fp16 B operand in
 //               shared memory (N-major, 128-byte swizzle), with the exact
@@ -45,7 +45,7 @@ namespace {
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kStagesW = 8;  // packed-W slots (TMA; freed by the decoders)
-constexpr int kStagesX = 3;  // x slots (TMA; freed by the MMAs)
+constexpr int kStagesX = 6;  // x slots (TMA; freed by the MMAs): deep enough to cover a TMA round trip
 constexpr int kStagesB = 2;  // decoded-B slots
 constexpr int kDecWarps = 16;
 constexpr int kDec0 = 3;     // first decoder warp (0: packed-W producer, 1: MMA, 2: x producer)
@@ -58,7 +58,7 @@ constexpr uint32_t kBBytes = kBN * kBK * 2;   // 32768
 constexpr uint32_t kSmemA = 0;
 constexpr uint32_t kSmemW = kSmemA + kStagesX * kABytes;
 constexpr uint32_t kSmemB = kSmemW + kStagesW * kWBytes;
-constexpr uint32_t kSmemTotal = kSmemB + kStagesB * kBBytes;  // 176 KB
+constexpr uint32_t kSmemTotal = kSmemB + kStagesB * kBBytes;  // 224 KB
 constexpr uint32_t kSmemDyn = kSmemTotal + 1024;              // + alignment slack
 constexpr uint32_t kTmemCols = 256;
 // B operand (N-major, 128-byte swizzle): 1 KB atoms of 64 n x 8 k; atoms

@@ -544,79 +544,47 @@ __global__ void __launch_bounds__(32) k_lz4_parse_staged(const __grid_constant__
 // fallback: warp 0 walks the block from global memory itself (lockstep,
 // warp-uniform control flow). Returns 0 or a stream status.
 // ---------------------------------------------------------------------------
-__device__ int walk_block_warp(const uint8_t *__restrict__ src, uint64_t ilen, uint8_t *win, uint32_t olen, int lane,
-                               uint8_t *ring) {
+__device__ int walk_block_warp(const uint8_t *__restrict__ src, uint64_t ilen, uint8_t *win, uint32_t olen,
+                               int lane) {
   if (ilen == 0) return olen == 0 ? 0 : LT_ERR_SIZE_MISMATCH;
-  if (ilen > 0x7FFFFFFFull) return LT_ERR_CORRUPT_STREAM;  // no valid block of <= 64 KB is this long
-  // the block's bytes stream through the parse's 2 KB cp.async ring (in
-  // `ring`), so that each header read is a shared-memory read, not a
-  // dependent global load
-  WarpRing r;
-  r.buf = ring;
-  r.lane = lane;
-  r.beg = src;
-  r.end = src + ilen;
-  r.a0 = reinterpret_cast<const uint8_t *>(reinterpret_cast<uintptr_t>(src) & ~uintptr_t(15));
-  r.total = (uint32_t)((r.end - r.a0 + kPChunk - 1) / kPChunk);
-  r.issued = 0;
-  r.done = 0;
-  r.top_up(0);
-  const uint32_t lead = (uint32_t)(src - r.a0);
-  auto byte = [&](uint64_t x) -> uint32_t {  // warp-uniform x < ilen
-    const uint32_t rel = lead + (uint32_t)x;
-    r.need(rel, rel + 1);
-    return r.at(rel);
-  };
   uint64_t ip = 0;
   uint32_t op = 0;
-  int st = 0;
   for (;;) {
-    if (ip >= ilen) { st = LT_ERR_CORRUPT_STREAM; break; }
-    const uint32_t token = byte(ip++);
+    if (ip >= ilen) return LT_ERR_CORRUPT_STREAM;
+    const uint32_t token = __ldg(src + ip++);
     uint64_t lit = token >> 4;
     if (lit == 15) {
       uint32_t bb;
       do {
-        if (ip >= ilen || lit > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
-        bb = byte(ip++);
+        if (ip >= ilen || lit > olen) return LT_ERR_CORRUPT_STREAM;
+        bb = __ldg(src + ip++);
         lit += bb;
       } while (bb == 255);
-      if (st) break;
     }
-    if (ip + lit > ilen || (uint64_t)op + lit > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
-    for (uint32_t done = 0; done < (uint32_t)lit; done += 32) {  // the literals, 32 bytes at a time
-      const uint32_t rel = lead + (uint32_t)ip + done;
-      const uint32_t q = ((uint32_t)lit - done) < 32u ? ((uint32_t)lit - done) : 32u;
-      r.need(rel, rel + q);
-      if ((uint32_t)lane < q) win[op + done + lane] = (uint8_t)r.at(rel + lane);
-    }
+    if (ip + lit > ilen || (uint64_t)op + lit > olen) return LT_ERR_CORRUPT_STREAM;
+    for (uint32_t i = lane; i < (uint32_t)lit; i += 32) win[op + i] = __ldg(src + ip + i);
     ip += lit;
     op += (uint32_t)lit;
     __syncwarp();
     if (ip == ilen) break;
-    if (ip + 2 > ilen) { st = LT_ERR_CORRUPT_STREAM; break; }
-    const uint32_t d0 = byte(ip), d1 = byte(ip + 1);
-    const uint32_t d = d0 | (d1 << 8);
+    if (ip + 2 > ilen) return LT_ERR_CORRUPT_STREAM;
+    const uint32_t d = (uint32_t)__ldg(src + ip) | ((uint32_t)__ldg(src + ip + 1) << 8);
     ip += 2;
-    if (d == 0 || d > op) { st = LT_ERR_CORRUPT_STREAM; break; }
+    if (d == 0 || d > op) return LT_ERR_CORRUPT_STREAM;
     uint64_t mlen = (token & 15u) + 4;
     if ((token & 15u) == 15u) {
       uint32_t bb;
       do {
-        if (ip >= ilen || mlen > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
-        bb = byte(ip++);
+        if (ip >= ilen || mlen > olen) return LT_ERR_CORRUPT_STREAM;
+        bb = __ldg(src + ip++);
         mlen += bb;
       } while (bb == 255);
-      if (st) break;
     }
-    if ((uint64_t)op + mlen > olen) { st = LT_ERR_CORRUPT_STREAM; break; }
+    if ((uint64_t)op + mlen > olen) return LT_ERR_CORRUPT_STREAM;
     copy_match<32>(win, op, d, (uint32_t)mlen, lane, 0xFFFFFFFFu);
     __syncwarp();
     op += (uint32_t)mlen;
   }
-  cp_async_wait<0>();  // nothing may land in the ring after this block
-  __syncwarp();
-  if (st) return st;
   return op == olen ? 0 : LT_ERR_SIZE_MISMATCH;
 }
 
@@ -1014,8 +982,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_lz4_expand(const __grid_constan
     }
     if (st != 0 && warp == 0) {
       int err = LT_ERR_CORRUPT_STREAM;
-      if (s0 <= s1 && s1 <= jb.comp_bytes)
-        err = walk_block_warp(jb.comp + s0, s1 - s0, win, olen, lane, reinterpret_cast<uint8_t *>(&S));
+      if (s0 <= s1 && s1 <= jb.comp_bytes) err = walk_block_warp(jb.comp + s0, s1 - s0, win, olen, lane);
       if (err && lane == 0) report(d_status, err);  // content unspecified after an error
     }
     __syncthreads();
