@@ -73,7 +73,9 @@ def check(got_bits, want, absum, K, what):
                            f"{float(np.max(err - bound)):.3g} at {np.unravel_index(np.argmax(err - bound), err.shape)}")
 
 
-@pytest.mark.parametrize("M,K,N,G,zeros", [(1, 64, 256, 32, True), (5, 128, 256, 128, True), (128, 256, 512, 64, False),
+@pytest.mark.parametrize("M,K,N,G,zeros", [(1, 64, 256, 32, True), (2, 1024, 512, 128, True), (3, 4096, 256, 64, False),
+                                           (5, 128, 256, 128, True), (8, 2048, 768, 256, True), (9, 512, 256, 32, True),
+                                           (128, 256, 512, 64, False),
                                            (200, 512, 768, 256, True), (129, 1024, 256, 128, True),
                                            (300, 64, 1024, 32, False)])
 def test_gemm_small_shapes_every_element(M, K, N, G, zeros):
@@ -100,6 +102,25 @@ def test_gemm_identity_input_returns_the_decoded_weights():
     L.lt_dequant_int4(dev(p["packed"]), dev(p["scales"]), dev(p["zeros"]), K, N, G, w)
     torch.cuda.synchronize()
     assert np.array_equal(got.ravel(), host_bits(w))
+
+
+@pytest.mark.parametrize("M", [1, 3, 8])
+def test_gemm_small_batch_unit_rows_return_rows_of_the_decoded_weights(M):
+    # batches of at most 8 rows take the CUDA-core kernel: with x[m] the unit
+    # vector e_(k_m), out[m] is row k_m of W, one exact product per element,
+    # so it equals lt_dequant_int4's output bit for bit
+    K, N, G = 1024, 512, 128
+    p = make_problem(M, K, N, G, seed=40 + M)
+    ks = np.random.default_rng(M).choice(K, size=M, replace=False)
+    x = np.zeros((M, K), np.float16)
+    x[np.arange(M), ks] = 1.0
+    p["x"] = x.view(np.uint16).ravel()
+    got = run_gemm(p)
+    w = torch.empty(K * N, dtype=torch.float16, device="cuda")
+    L.lt_dequant_int4(dev(p["packed"]), dev(p["scales"]), dev(p["zeros"]), K, N, G, w)
+    torch.cuda.synchronize()
+    want = host_bits(w).reshape(K, N)[ks]
+    assert np.array_equal(got, want)
 
 
 C5_SHAPES = [("q", 8192, 8192), ("k", 8192, 1024), ("gate", 8192, 28672), ("down", 28672, 8192)]

@@ -12,16 +12,16 @@
 // fixed order). Warp roles:
 //   warp 0      packed-W producer: for each 64-wide K step one tiled bulk
 //               copy (TMA) of the packed INT4 tile (64 rows x 128 bytes,
-//               128-byte swizzle) into an 8-deep ring, completion counted on
+//               128-byte swizzle) into a 6-deep ring, completion counted on
 //               an mbarrier; a slot is refilled as soon as the decoders are
 //               done with it, so this stream runs well ahead of the MMAs;
 //   warp 2      x producer: the x tile (128 x 64 fp16, 128-byte swizzle) of
-//               each step into a 6-deep ring, refilled when the MMAs that
+//               each step into a 3-deep ring, refilled when the MMAs that
 //               read a slot have completed;
 //   warps 3..18 decoders: turn the packed tile into the fp16 B operand in
 //               shared memory (N-major, 128-byte swizzle), with the exact
 //               half2 arithmetic of lt_dequant_int4 (bit-identical to it), in
-//               a 2-deep ring; scales and zero points are loaded three steps
+//               a 4-deep ring; scales and zero points are loaded three steps
 //               before their use;
 //   warp 1      MMA issuer: one thread issues tcgen05.mma kind::f16 (fp32
 //               accumulator in tensor memory, 128 x 256 = 256 columns), four
@@ -44,9 +44,9 @@ namespace lt {
 namespace {
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
-constexpr int kStagesW = 8;  // packed-W slots (TMA; freed by the decoders)
-constexpr int kStagesX = 6;  // x slots (TMA; freed by the MMAs): deep enough to cover a TMA round trip
-constexpr int kStagesB = 2;  // decoded-B slots
+constexpr int kStagesW = 6;  // packed-W slots (TMA; freed by the decoders)
+constexpr int kStagesX = 3;  // x slots (TMA; freed by the MMAs)
+constexpr int kStagesB = 4;  // decoded-B slots: the decoders run up to three steps ahead of the MMAs
 constexpr int kDecWarps = 16;
 constexpr int kDec0 = 3;     // first decoder warp (0: packed-W producer, 1: MMA, 2: x producer)
 constexpr int kUnits = (kBK * kBN / 32) / (kDecWarps * 32);  // 16-byte packed chunks per decoder thread per step
@@ -372,6 +372,117 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
   }
 }
 
+// ---------------------------------------------------------------------------
+// Small batches (M <= 8): the same product on the CUDA cores. With a few rows
+// of x, the 128-row MMA tile is mostly padding while its operands still flow
+// through shared memory; here each code is decoded in registers and used
+// straight away, so the codes stream from HBM once and nothing is staged
+// but x. One CTA: 256 columns [n0, n0 + 256) over a range of K rows (a split
+// of K); lane l of every warp takes columns n0 + 8 l .. + 7 (one 4-byte word
+// of codes per row, a warp's loads 128 contiguous bytes), warp w rows w,
+// w + 8, ... of each chunk of 512 rows. W is decoded with the exact half2
+// arithmetic (lt_dequant_int4's values) and widened to fp32; products with x
+// are exact in fp32 and summed in fp32 per thread, then the 8 warps' sums in
+// order through shared memory.
+// ---------------------------------------------------------------------------
+constexpr int kVThreads = 256;
+constexpr int kVCols = 256;
+constexpr int kVChunk = 512;  // x rows staged per chunk
+constexpr int kVUnroll = 8;   // code words in flight per thread
+
+template <int MT>
+__global__ void __launch_bounds__(kVThreads) k_int4_gemv(const uint16_t *__restrict__ x, int64_t M, int64_t K,
+                                                          const uint32_t *__restrict__ packed,
+                                                          const uint16_t *__restrict__ scales,
+                                                          const uint8_t *__restrict__ zeros, int64_t N, int32_t G,
+                                                          uint16_t *__restrict__ out, float *__restrict__ partial,
+                                                          int splits) {
+  __shared__ float xs[MT][kVChunk];
+  __shared__ float red[MT][kVCols];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t n0 = (int64_t)blockIdx.x * kVCols;
+  const int split = blockIdx.y;
+  const int64_t k_begin = K * split / splits, k_end = K * (split + 1) / splits;
+  const int64_t NG = N / G, wpr = N / 8;  // groups and code words per row
+  const int64_t col = n0 + 8 * lane;
+  const int64_t gcol = col / G;
+  float acc[MT][8];
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[m][j] = 0.f;
+  for (int64_t c0 = k_begin; c0 < k_end; c0 += kVChunk) {
+    const int rows = (int)((k_end - c0) < kVChunk ? (k_end - c0) : kVChunk);
+    __syncthreads();  // the previous chunk's x is no longer read
+    for (int i = tid; i < MT * kVChunk; i += kVThreads) {
+      const int m = i / kVChunk, r = i % kVChunk;
+      xs[m][r] = (m < M && r < rows) ? __half2float(__ushort_as_half(x[(int64_t)m * K + c0 + r])) : 0.f;
+    }
+    __syncthreads();
+    for (int r0 = warp; r0 < rows; r0 += 8 * kVUnroll) {
+      uint32_t w[kVUnroll], sc[kVUnroll], zr[kVUnroll];
+#pragma unroll
+      for (int u = 0; u < kVUnroll; ++u) {
+        const int r = r0 + 8 * u;
+        const int64_t k = c0 + (r < rows ? r : 0);
+        w[u] = r < rows ? ld_stream_u32(packed + k * wpr + col / 8) : 0u;
+        sc[u] = r < rows ? __ldg(scales + k * NG + gcol) : 0u;
+        zr[u] = (r < rows && zeros) ? __ldg(zeros + k * NG + gcol) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kVUnroll; ++u) {
+        const int r = r0 + 8 * u;
+        if (r < rows) {
+          const uint4 h = int4x8_dequant(w[u], zeros ? int4_zero_magic(zr[u]) : 0x54006400u, bcast_half((uint16_t)sc[u]));
+          const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
+          float wv[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hw[q]));
+            wv[2 * q] = f.x;
+            wv[2 * q + 1] = f.y;
+          }
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            const float xm = xs[m][r];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[m][j] = fmaf(xm, wv[j], acc[m][j]);
+          }
+        }
+      }
+    }
+  }
+  // the 8 warps' sums, added in warp order
+  for (int wv = 0; wv < 8; ++wv) {
+    __syncthreads();
+    if (warp == wv) {
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) red[m][8 * lane + j] = (wv == 0 ? 0.f : red[m][8 * lane + j]) + acc[m][j];
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < MT * kVCols; i += kVThreads) {
+    const int m = i / kVCols, c = i % kVCols;
+    if (m >= M) continue;
+    if (splits == 1)
+      out[m * N + n0 + c] = __half_as_ushort(__float2half_rn(red[m][c]));
+    else
+      partial[((int64_t)split * M + m) * N + n0 + c] = red[m][c];
+  }
+}
+
+// K splits of the small-batch kernel: about two CTAs per SM, each split at
+// least 256 rows
+int gemv_splits(int64_t N, int64_t K) {
+  const int64_t tiles = N / kVCols;
+  int64_t s = (2 * (int64_t)num_sms() + tiles - 1) / tiles;
+  if (s > K / 256) s = K / 256;
+  if (s > 64) s = 64;
+  return (int)(s < 1 ? 1 : s);
+}
+
 // out[m, n] = fp16_rn(sum over splits s = 0, 1, ... of partial[s, m, n]), in that order
 __global__ void __launch_bounds__(256) k_gemm_reduce(const float4 *__restrict__ partial, int64_t mn4, int splits,
                                                      uint2 *__restrict__ out) {
@@ -425,8 +536,13 @@ using namespace lt;
 
 LT_API uint64_t lt_int4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < kBN || K < kBK || N % kBN != 0 || K % kBK != 0) return 0;
-  const int64_t tiles = ((M + kBM - 1) / kBM) * (N / kBN);
-  const int s = choose_splits(tiles, K / kBK);
+  int s;
+  if (M <= 8) {
+    s = gemv_splits(N, K);
+  } else {
+    const int64_t tiles = ((M + kBM - 1) / kBM) * (N / kBN);
+    s = choose_splits(tiles, K / kBK);
+  }
   return s > 1 ? (uint64_t)s * (uint64_t)M * (uint64_t)N * 4ull : 0;
 }
 
@@ -440,6 +556,32 @@ LT_API lt_status lt_int4_gemm(const lt_half *x, int64_t M, int64_t K, const uint
   if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(out, 16) || !aligned(scales, 2) ||
       !aligned(workspace, 16) || !aligned(d_status, 4))
     return LT_ERR_MISALIGNED;
+  cudaStream_t st = (cudaStream_t)stream;
+  auto reduce_splits = [&](int splits) {
+    const int64_t mn4 = M * N / 4;
+    int64_t g = (mn4 + 255) / 256;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (g > cap) g = cap;
+    k_gemm_reduce<<<(int)g, 256, 0, st>>>(reinterpret_cast<const float4 *>(workspace), mn4, splits,
+                                          reinterpret_cast<uint2 *>(out));
+  };
+  if (M <= 8) {  // small batch: the CUDA-core kernel
+    int splits = gemv_splits(N, K);
+    if (splits > 1 && (!workspace || workspace_bytes < (uint64_t)splits * (uint64_t)M * (uint64_t)N * 4ull)) splits = 1;
+    const dim3 grid((unsigned)(N / kVCols), (unsigned)splits);
+    const uint32_t *pw = reinterpret_cast<const uint32_t *>(packed);
+    float *part = reinterpret_cast<float *>(workspace);
+    if (M == 1)
+      k_int4_gemv<1><<<grid, kVThreads, 0, st>>>(x, M, K, pw, scales, zeros, N, group_size, out, part, splits);
+    else if (M == 2)
+      k_int4_gemv<2><<<grid, kVThreads, 0, st>>>(x, M, K, pw, scales, zeros, N, group_size, out, part, splits);
+    else if (M <= 4)
+      k_int4_gemv<4><<<grid, kVThreads, 0, st>>>(x, M, K, pw, scales, zeros, N, group_size, out, part, splits);
+    else
+      k_int4_gemv<8><<<grid, kVThreads, 0, st>>>(x, M, K, pw, scales, zeros, N, group_size, out, part, splits);
+    if (splits > 1) reduce_splits(splits);
+    return launch_status();
+  }
   encode_tiled_t enc = encoder();
   if (!enc) return LT_ERR_CUDA;
   CUtensorMap map_x, map_w;
@@ -487,16 +629,8 @@ LT_API lt_status lt_int4_gemm(const lt_half *x, int64_t M, int64_t K, const uint
       return LT_ERR_CUDA;
     attr_set[dev] = 1;
   }
-  cudaStream_t st = (cudaStream_t)stream;
   k_int4_gemm<<<dim3((unsigned)tiles_n, (unsigned)tiles_m, (unsigned)splits), kGemmThreads, kSmemDyn, st>>>(map_x,
                                                                                                          map_w, ga);
-  if (splits > 1) {
-    const int64_t mn4 = M * N / 4;
-    int64_t g = (mn4 + 255) / 256;
-    const int64_t cap = (int64_t)num_sms() * 8;
-    if (g > cap) g = cap;
-    k_gemm_reduce<<<(int)g, 256, 0, st>>>(reinterpret_cast<const float4 *>(workspace), mn4, splits,
-                                          reinterpret_cast<uint2 *>(out));
-  }
+  if (splits > 1) reduce_splits(splits);
   return launch_status();
 }
