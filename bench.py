@@ -868,11 +868,29 @@ def c1_graph_steady_state(hw, peak: float, n_sets: int = 64, chains: int = 8, re
             "hbm_frac_of_measured": (rd + 2 * n) / per / 1e9 / peak, "outputs_identical": bool(same)}
 
 
+class L2Flush:
+    """Before a timed call: write a 256 MB scratch buffer (twice L2), then
+    read it back (a sum into a one-element tensor). The write evicts what
+    the previous calls left in L2; the read evicts the write's dirty lines,
+    so their write-back to HBM happens here and not inside the timed call,
+    and L2 is left holding only clean lines of the scratch buffer."""
+
+    def __init__(self, nbytes: int = 256 << 20):
+        import torch
+        self.buf = torch.empty(nbytes // 4, dtype=torch.int32, device="cuda")
+        self.sink = torch.empty((), dtype=torch.int64, device="cuda")
+
+    def __call__(self, r: int):
+        import torch
+        self.buf.fill_(r & 0xFF)
+        torch.sum(self.buf, dim=0, dtype=torch.int64, out=self.sink)
+
+
 def value_dict_timing(peak: float, reps: int = 30, warmup: int = 3):
     """The value-dictionary decode on its workload (4096 x 14336 4-bit
     indices with C4's code law, one 16-entry fp16 dictionary), timed per
     call with CUDA events on the launching stream; before every call a
-    256 MB scratch write (not timed) flushes L2."""
+    256 MB scratch write and read (not timed, L2Flush) flush L2."""
     import numpy as np
     import torch
 
@@ -884,11 +902,11 @@ def value_dict_timing(peak: float, reps: int = 30, warmup: int = 3):
     packed = torch.from_numpy(d["packed"]).cuda()
     dictionary = torch.from_numpy(d["dictionary"].view(np.int16)).cuda()
     out = torch.empty(n, dtype=torch.float16, device="cuda")
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
     s = torch.cuda.current_stream()
     times = []
     for r in range(warmup + reps):
-        flush.fill_(r & 0xFF)
+        flush(r)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(s)
@@ -925,8 +943,8 @@ def gemm_timing(hbm_peak: float, reps: int = 10, warmup: int = 3, shapes=GEMM_SH
     """Fused INT4 decode -> GEMM (lt_int4_gemm) on the C5 weight shapes
     ([K, N] = [in, out], C4's code law, group 128) against decode-then-
     cuBLAS (lt_dequant_int4 into an fp16 buffer, then torch.matmul). Device
-    time per call by CUDA events, median of `reps`, a 256 MB L2-flushing
-    write before each call (not timed). Roofline: HBM bytes (x + packed
+    time per call by CUDA events, median of `reps`, an L2 flush (L2Flush)
+    before each call (not timed). Roofline: HBM bytes (x + packed
     codes + scales + zero points + out) against the measured copy peak, and
     2 M N K flops against the measured dense 16-bit tensor peak; the bound
     is whichever time is larger."""
@@ -938,12 +956,12 @@ def gemm_timing(hbm_peak: float, reps: int = 10, warmup: int = 3, shapes=GEMM_SH
 
     tpeak, tkind = read_tflops_peak()
     s = torch.cuda.current_stream()
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
 
     def timed(fn):
         ts = []
         for r in range(warmup + reps):
-            flush.fill_(r & 0xFF)
+            flush(r)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(s)
@@ -1004,8 +1022,8 @@ def checksum_timing(dw, hw, peak: float, reps: int = 20, warmup: int = 3):
     """Per-block XXH3-64 on C4's compressed stream (448 blocks): the
     standalone verifier (lt_xxh3_blocks, one warp per block) and the decode
     with the check fused in (lt_lz4_int4_decode_checked) against the plain
-    fused decode. Device time by CUDA events, median of `reps`, a 256 MB
-    L2-flushing write before each call (not timed)."""
+    fused decode. Device time by CUDA events, median of `reps`, an L2 flush
+    (L2Flush) before each call (not timed)."""
     import numpy as np
     import torch
 
@@ -1020,12 +1038,12 @@ def checksum_timing(dw, hw, peak: float, reps: int = 20, warmup: int = 3):
     s = torch.cuda.current_stream()
     comp_bytes = int(c4["comp"].size)
     L.lt_xxh3_blocks(dw.c4["comp"], comp_bytes, dw.c4["offsets"], nb, secret, 192, hashes, None, st, first, s)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
 
     def timed(fn):
         ts = []
         for r in range(warmup + reps):
-            flush.fill_(r & 0xFF)
+            flush(r)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(s)
@@ -1085,14 +1103,14 @@ def lz4_cliff_timing(dw, hw, reps: int = 10, warmup: int = 2):
     ws = torch.empty(L.lt_lz4_workspace_bytes(nb), dtype=torch.uint8, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     s = torch.cuda.current_stream()
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
     c4 = hw["C4"]
     out4 = torch.empty(c4["packed_bytes"], dtype=torch.uint8, device="cuda")
 
     def timed(fn):
         ts = []
         for r in range(warmup + reps):
-            flush.fill_(r & 0xFF)
+            flush(r)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(s)

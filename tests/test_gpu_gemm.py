@@ -75,6 +75,10 @@ def check(got_bits, want, absum, K, what):
 
 @pytest.mark.parametrize("M,K,N,G,zeros", [(1, 64, 256, 32, True), (2, 1024, 512, 128, True), (3, 4096, 256, 64, False),
                                            (5, 128, 256, 128, True), (8, 2048, 768, 256, True), (9, 512, 256, 32, True),
+                                           # small batches whose scale / zero-point rows are 16-byte multiples
+                                           # (tiles of both by TMA), and a group of 96 (boxes straddling groups)
+                                           (4, 512, 4096, 128, True), (6, 256, 512, 32, True), (2, 384, 768, 96, True),
+                                           (7, 192, 2048, 64, False),
                                            (128, 256, 512, 64, False),
                                            (200, 512, 768, 256, True), (129, 1024, 256, 128, True),
                                            (300, 64, 1024, 32, False)])
@@ -104,13 +108,14 @@ def test_gemm_identity_input_returns_the_decoded_weights():
     assert np.array_equal(got.ravel(), host_bits(w))
 
 
-@pytest.mark.parametrize("M", [1, 3, 8])
-def test_gemm_small_batch_unit_rows_return_rows_of_the_decoded_weights(M):
-    # batches of at most 8 rows take the CUDA-core kernel: with x[m] the unit
+@pytest.mark.parametrize("M,N", [(1, 512), (3, 512), (8, 512), (1, 4096), (5, 4096)])
+def test_gemm_small_batch_unit_rows_return_rows_of_the_decoded_weights(M, N):
+    # batches of at most 8 rows take the mma.sync kernel: with x[m] the unit
     # vector e_(k_m), out[m] is row k_m of W, one exact product per element,
-    # so it equals lt_dequant_int4's output bit for bit
-    K, N, G = 1024, 512, 128
-    p = make_problem(M, K, N, G, seed=40 + M)
+    # so it equals lt_dequant_int4's output bit for bit (N = 512: scales and
+    # zero points copied word by word; N = 4096: by TMA)
+    K, G = 1024, 128
+    p = make_problem(M, K, N, G, seed=40 + M + N)
     ks = np.random.default_rng(M).choice(K, size=M, replace=False)
     x = np.zeros((M, K), np.float16)
     x[np.arange(M), ks] = 1.0

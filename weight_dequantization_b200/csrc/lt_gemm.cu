@@ -37,6 +37,7 @@
 #include "lt_common.cuh"
 
 #include <cuda.h>
+#include <algorithm>
 #include <mutex>
 #include <type_traits>
 
@@ -139,6 +140,37 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// explicit shared-window accesses (32-bit shared addresses)
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t a) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds8(uint32_t a) {
+  uint16_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
 struct GemmArgs {
   const uint16_t *scales;  // [K, N / G]
   const uint8_t *zeros;    // [K, N / G] or nullptr
@@ -149,6 +181,9 @@ struct GemmArgs {
   int32_t group_size;
   int32_t k_iters;  // K / 64
   int32_t splits;
+  // small-batch kernel: TMA box widths (elements) of the scale and zero-point
+  // tiles, 0 where that tensor is copied word by word instead
+  int32_t sc_box, z_box;
 };
 
 __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_constant__ CUtensorMap map_x,
@@ -196,6 +231,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = s_tmem;
   const uint32_t sbase = smem_u32(sm);
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // see k_gemm_reduce
 
   auto fail = [&]() {
     s_abort = 1;
@@ -288,29 +324,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
     // (sc, zr), refill (sc, zr) for step it + 3, hand the slot to the MMA
     auto step = [&](int it, uint32_t(&sc)[kUnits], uint32_t(&zr)[kUnits]) -> bool {
       const int s = it % kStagesW, b = it % kStagesB;
-      if (!mbar_wait(smem_u32(&bar_wfull[s]), (it / kStagesW) & 1) ||
-          (it >= kStagesB && !mbar_wait(smem_u32(&bar_bempty[b]), ((it / kStagesB) - 1) & 1))) {
+      const bool got = mbar_wait(smem_u32(&bar_wfull[s]), (it / kStagesW) & 1) &&
+                       (it < kStagesB || mbar_wait(smem_u32(&bar_bempty[b]), ((it / kStagesB) - 1) & 1));
+      // the warp goes on only together: it meets at __syncwarp below
+      if (!__all_sync(0xffffffffu, got)) {
         fail();
         return false;
       }
       if (*(volatile int *)&s_abort) return false;
-      const uint8_t *wsrc = sm + kSmemW + s * kWBytes;
-      uint8_t *bdst = sm + kSmemB + b * kBBytes;
+      const uint32_t wsrc = sbase + kSmemW + s * kWBytes;
+      const uint32_t bdst = sbase + kSmemB + b * kBBytes;
 #pragma unroll
       for (int i = 0; i < kUnits; ++i) {
         const int kk = klo + 8 * (khi0 + (kDecWarps / 2) * i);  // row of the step, 0..63
         // packed row kk: 128 bytes (256 codes), 16-byte chunk h at chunk h ^ (kk & 7)
-        const uint4 v = *reinterpret_cast<const uint4 *>(wsrc + kk * 128 + ((h ^ klo) << 4));
+        const uint4 v = lds128(wsrc + kk * 128 + ((h ^ klo) << 4));
         const uint32_t s2 = bcast_half((uint16_t)sc[i]);
         const uint32_t zm = a.zeros ? int4_zero_magic(zr[i]) : 0x54006400u;
         const uint4 o[4] = {int4x8_dequant(v.x, zm, s2), int4x8_dequant(v.y, zm, s2), int4x8_dequant(v.z, zm, s2),
                             int4x8_dequant(v.w, zm, s2)};
         // codes n = 32 h + 8 j .. + 7 of row kk: atom (n / 64, kk / 8), row kk % 8, chunk (n % 64) / 8
-        uint8_t *atom = bdst + (h >> 1) * kBAtomN + (kk >> 3) * kBAtomK + klo * 128;
+        const uint32_t atom = bdst + (h >> 1) * kBAtomN + (kk >> 3) * kBAtomK + klo * 128;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int c = 4 * (h & 1) + j;
-          *reinterpret_cast<uint4 *>(atom + ((c ^ klo) << 4)) = o[j];
+          sts128(atom + ((c ^ klo) << 4), o[j]);
         }
       }
       if (it + 3 < n_it) load_sz(it + 3, sc, zr);
@@ -329,7 +367,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
       if (ok && it + 2 < n_it) ok = step(it + 2, scC, zrC);
     }
     // ---------------- epilogue ----------------
-    const bool acc_ok = mbar_wait(smem_u32(&bar_acc), 0);
+    const bool acc_ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_acc), 0));  // tcgen05.ld is warp-wide
     if (!acc_ok) fail();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (acc_ok && !*(volatile int *)&s_abort && n_it > 0) {
@@ -373,119 +411,320 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
 }
 
 // ---------------------------------------------------------------------------
-// Small batches (M <= 8): the same product on the CUDA cores. With a few rows
-// of x, the 128-row MMA tile is mostly padding while its operands still flow
-// through shared memory; here each code is decoded in registers and used
-// straight away, so the codes stream from HBM once and nothing is staged
-// but x. One CTA: 256 columns [n0, n0 + 256) over a range of K rows (a split
-// of K); lane l of every warp takes columns n0 + 8 l .. + 7 (one 4-byte word
-// of codes per row, a warp's loads 128 contiguous bytes), warp w rows w,
-// w + 8, ... of each chunk of 512 rows. W is decoded with the exact half2
-// arithmetic (lt_dequant_int4's values) and widened to fp32; products with x
-// are exact in fp32 and summed in fp32 per thread, then the 8 warps' sums in
-// order through shared memory.
+// Small batches (M <= 8). With a few rows of x the 128-row tcgen05 tile is
+// mostly padding, while its decoded operand still makes a round trip through
+// shared memory; the product is bound by streaming the codes from HBM. Here
+// the codes stream through a TMA ring and each thread decodes them straight
+// into the register operands of mma.sync.m16n8k16 (fp16 in, fp32
+// accumulate), computing out^T = W^T . x^T: the MMA's 16 rows are 16 columns
+// of W, its 16-deep reduction 16 rows of K, its 8 columns the batch.
+//
+// One CTA: 256 columns [n0, n0 + 256) over a range of 64-row K tiles (a
+// split of K). Warp 0 is the producer: per tile one TMA copy of the packed
+// codes (64 rows x 128 bytes, 128-byte swizzle) and one of x (8 batch rows x
+// 64 fp16, rows past M zero-filled) into an 8-deep ring, plus an L2 prefetch
+// of the tile's scales and zero points. Warps 1..8: warp 1 + 2 q + h takes
+// column half h (128 columns) and rows 16 q .. 16 q + 15 of every tile.
+// Lane (g, t) = (lane / 4, lane % 4) holds, for the 8 MMAs j = 0..7 of a
+// tile, code byte j of its 8-byte slice (columns 16 g + 2 j and + 1 of the
+// half) in rows 2t, 2t+1, 2t+8, 2t+9 of the slot: a byte of row k and the
+// same byte of row k + 1 make two half2 A registers, (W[k][c], W[k+1][c])
+// for the low nibbles and for the high ones, with the exact arithmetic of
+// lt_dequant_int4 (so W is bit-identical to its output). The products are
+// exact in fp32; sums are in fp32. At the end the four K slots' sums are
+// added in slot order through shared memory.
 // ---------------------------------------------------------------------------
-constexpr int kVThreads = 256;
-constexpr int kVCols = 256;
-constexpr int kVChunk = 512;  // x rows staged per chunk
-constexpr int kVUnroll = 8;   // code words in flight per thread
+constexpr int kVWarps = 8;                       // consumer warps
+constexpr int kVThreads = 32 * (kVWarps + 1);    // + the producer warp
+constexpr int kVStages = 8;
+constexpr int kVPerSM = 2;                       // resident CTAs per SM (launch bounds, shared memory)
+constexpr uint32_t kVXBytes = 8 * kBK * 2;       // x tile: 8 rows x 64 fp16
+// each row's scales and zero points of the strip: a TMA box of 8 or 16
+// scales / 16 or 32 zero points per row starting at a 16-byte boundary at or
+// below the strip's first group, or (where the tensors' row pitch is not a
+// multiple of 16 bytes) the 4-byte words holding them (a strip of 256
+// columns spans at most 9 groups of >= 32: <= 5 words of scales, <= 3 of
+// zero points)
+constexpr uint32_t kVScRow = 20, kVZRow = 12;  // word-copy row pitches
+constexpr uint32_t kVScOff = kWBytes + kVXBytes, kVZOff = kVScOff + kBK * 32;
+constexpr uint32_t kVStage = kVZOff + kBK * 32;  // 13312, a multiple of 1 KB (swizzle atoms stay aligned)
+static_assert(kVStage % 1024 == 0, "stage size");
+constexpr uint32_t kVRing = kVStages * kVStage;
+constexpr int kVRedPitch = 290;                  // fp32 words per batch row of the reduction buffer
+constexpr uint32_t kVRedBytes = 4u * 8u * kVRedPitch * 4u;
+static_assert(kVRedBytes <= kVRing, "the reduction buffer reuses the ring");
+constexpr uint32_t kVSmemDyn = kVRing + 1024;
 
-template <int MT>
-__global__ void __launch_bounds__(kVThreads) k_int4_gemv(const uint16_t *__restrict__ x, int64_t M, int64_t K,
-                                                          const uint32_t *__restrict__ packed,
-                                                          const uint16_t *__restrict__ scales,
-                                                          const uint8_t *__restrict__ zeros, int64_t N, int32_t G,
-                                                          uint16_t *__restrict__ out, float *__restrict__ partial,
-                                                          int splits) {
-  __shared__ float xs[MT][kVChunk];
-  __shared__ float red[MT][kVCols];
+// byte JJ of wa (row k) and of wb (row k + 1), columns c (low nibble) and
+// c + 1 (high nibble): lo = (W[k][c], W[k+1][c]), hi = (W[k][c+1], W[k+1][c+1])
+// as half2, each fp16_rn((q - z) * s) exactly as in lt_dequant_int4: the
+// low nibbles OR-ed into the fraction of 1024 (ulp 1), the high ones into
+// that of 64 (ulp 1/16) four bits up, the zero points' magic subtracted
+// exactly, one rounded multiply by the row's scale.
+template <int JJ>
+__device__ __forceinline__ void int4_rowpair(uint32_t wa, uint32_t wb, uint32_t zlo, uint32_t zhi, uint32_t s2,
+                                             uint32_t &lo, uint32_t &hi) {
+  constexpr uint32_t sel = (uint32_t)JJ | ((uint32_t)JJ << 4) | ((uint32_t)(4 + JJ) << 8) | ((uint32_t)(4 + JJ) << 12);
+  const uint32_t x = __byte_perm(wa, wb, sel);  // [wa.bJJ, wa.bJJ, wb.bJJ, wb.bJJ]
+  uint32_t l, h;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(l) : "r"(x), "r"(0x000F000Fu), "r"(0x64006400u));  // (a & b) | c
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h) : "r"(x), "r"(0x00F000F0u), "r"(0x54005400u));
+  lo = hmul2_rn(hsub2_rn(l, zlo), s2);
+  hi = hmul2_rn(hsub2_rn(h, zhi), s2);
+}
+__device__ __forceinline__ uint32_t hadd2_rn(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 4-byte copy global -> shared (only the first `bytes` bytes read, the rest
+// zero), completion tracked by the thread's next cp.async mbarrier arrive
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, uint32_t bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__global__ void __launch_bounds__(kVThreads, kVPerSM) k_int4_gemv(const __grid_constant__ CUtensorMap map_x,
+                                                                   const __grid_constant__ CUtensorMap map_w,
+                                                                   const __grid_constant__ CUtensorMap map_s,
+                                                                   const __grid_constant__ CUtensorMap map_z,
+                                                                   const __grid_constant__ GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bar_full[kVStages], bar_empty[kVStages];
+  __shared__ int s_abort;
+
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t n0 = (int64_t)blockIdx.x * kVCols;
+  const int64_t n0 = (int64_t)blockIdx.x * kBN;
   const int split = blockIdx.y;
-  const int64_t k_begin = K * split / splits, k_end = K * (split + 1) / splits;
-  const int64_t NG = N / G, wpr = N / 8;  // groups and code words per row
-  const int64_t col = n0 + 8 * lane;
-  const int64_t gcol = col / G;
-  float acc[MT][8];
-#pragma unroll
-  for (int m = 0; m < MT; ++m)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[m][j] = 0.f;
-  for (int64_t c0 = k_begin; c0 < k_end; c0 += kVChunk) {
-    const int rows = (int)((k_end - c0) < kVChunk ? (k_end - c0) : kVChunk);
-    __syncthreads();  // the previous chunk's x is no longer read
-    for (int i = tid; i < MT * kVChunk; i += kVThreads) {
-      const int m = i / kVChunk, r = i % kVChunk;
-      xs[m][r] = (m < M && r < rows) ? __half2float(__ushort_as_half(x[(int64_t)m * K + c0 + r])) : 0.f;
+  const int it_begin = (int)((int64_t)a.k_iters * split / a.splits);
+  const int n_it = (int)((int64_t)a.k_iters * (split + 1) / a.splits) - it_begin;
+  const int64_t NG = a.N / a.group_size;
+
+  if (tid == 0) {
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(smem_u32(&bar_full[s]), 1 + 32);  // the TMA's arrive + each producer lane's copies
+      mbar_init(smem_u32(&bar_empty[s]), kVWarps);
     }
-    __syncthreads();
-    for (int r0 = warp; r0 < rows; r0 += 8 * kVUnroll) {
-      uint32_t w[kVUnroll], sc[kVUnroll], zr[kVUnroll];
-#pragma unroll
-      for (int u = 0; u < kVUnroll; ++u) {
-        const int r = r0 + 8 * u;
-        const int64_t k = c0 + (r < rows ? r : 0);
-        w[u] = r < rows ? ld_stream_u32(packed + k * wpr + col / 8) : 0u;
-        sc[u] = r < rows ? __ldg(scales + k * NG + gcol) : 0u;
-        zr[u] = (r < rows && zeros) ? __ldg(zeros + k * NG + gcol) : 0u;
-      }
-#pragma unroll
-      for (int u = 0; u < kVUnroll; ++u) {
-        const int r = r0 + 8 * u;
-        if (r < rows) {
-          const uint4 h = int4x8_dequant(w[u], zeros ? int4_zero_magic(zr[u]) : 0x54006400u, bcast_half((uint16_t)sc[u]));
-          const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
-          float wv[8];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hw[q]));
-            wv[2 * q] = f.x;
-            wv[2 * q + 1] = f.y;
-          }
-#pragma unroll
-          for (int m = 0; m < MT; ++m) {
-            const float xm = xs[m][r];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[m][j] = fmaf(xm, wv[j], acc[m][j]);
-          }
-        }
-      }
-    }
-  }
-  // the 8 warps' sums, added in warp order
-  for (int wv = 0; wv < 8; ++wv) {
-    __syncthreads();
-    if (warp == wv) {
-#pragma unroll
-      for (int m = 0; m < MT; ++m)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) red[m][8 * lane + j] = (wv == 0 ? 0.f : red[m][8 * lane + j]) + acc[m][j];
-    }
+    s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  for (int i = tid; i < MT * kVCols; i += kVThreads) {
-    const int m = i / kVCols, c = i % kVCols;
-    if (m >= M) continue;
-    if (splits == 1)
-      out[m * N + n0 + c] = __half_as_ushort(__float2half_rn(red[m][c]));
-    else
-      partial[((int64_t)split * M + m) * N + n0 + c] = red[m][c];
+  // the split-sum kernel that follows on the stream may start launching now;
+  // it waits for this grid's completion before reading anything
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const uint32_t sbase = smem_u32(sm);
+  auto fail = [&]() {
+    s_abort = 1;
+    report(a.d_status, LT_ERR_TIMEOUT);
+  };
+
+  float acc[8][4];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+  const int cw = warp - 1, h = cw & 1, q = cw >> 1, g = lane >> 2, t = lane & 3;
+
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    const int64_t gc0 = n0 / a.group_size, gc1 = (n0 + kBN - 1) / a.group_size;
+    const uint64_t sc_bytes = 2ull * (uint64_t)a.K * (uint64_t)NG, z_bytes = (uint64_t)a.K * (uint64_t)NG;
+    const uint8_t *sc8 = reinterpret_cast<const uint8_t *>(a.scales);
+    // per row of a tile (lane, lane + 32): the first word and the word counts
+    // do not depend on the tile (k0 is a multiple of 64)
+    uint64_t sw0[2], zw0[2];
+    uint32_t nws[2], nwz[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const uint64_t e = (uint64_t)(lane + 32 * r) * (uint64_t)NG;
+      const uint64_t sb = 2 * (e + gc0), se = 2 * (e + gc1) + 2, zb = e + gc0, ze = e + gc1 + 1;
+      sw0[r] = sb & ~uint64_t(3);
+      zw0[r] = zb & ~uint64_t(3);
+      nws[r] = a.sc_box ? 0u : (uint32_t)((se - sw0[r] + 3) / 4);
+      nwz[r] = (a.zeros && !a.z_box) ? (uint32_t)((ze - zw0[r] + 3) / 4) : 0u;
+    }
+    const int64_t xs = (gc0 / 8) * 8, xz = (gc0 / 16) * 16;  // TMA boxes start at 16-byte boundaries
+    const uint32_t tx_bytes = kWBytes + kVXBytes + (uint32_t)(kBK * 2 * a.sc_box) + (uint32_t)(kBK * a.z_box);
+    int issued = 0;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it % kVStages;
+      bool ok = true;
+      if (it >= kVStages && lane == 0) ok = mbar_wait(smem_u32(&bar_empty[s]), ((it / kVStages) - 1) & 1);
+      if (!__shfl_sync(0xffffffffu, (int)ok, 0)) {
+        if (lane == 0) fail();
+        break;
+      }
+      if (*(volatile int *)&s_abort) break;
+      const int32_t k0 = (it_begin + it) * kBK;
+      const uint32_t dst = sbase + s * kVStage, bar = smem_u32(&bar_full[s]);
+      if (lane == 0) {
+        mbar_expect_tx(bar, tx_bytes);
+        tma_load_2d(dst, &map_w, (int32_t)(n0 / 2), k0, bar);
+        tma_load_2d(dst + kWBytes, &map_x, k0, 0, bar);
+        if (a.sc_box) tma_load_2d(dst + kVScOff, &map_s, (int32_t)xs, k0, bar);
+        if (a.z_box) tma_load_2d(dst + kVZOff, &map_z, (int32_t)xz, k0, bar);
+      }
+      // the tile's scales and zero points: rows lane and lane + 32, the
+      // 4-byte words covering groups gc0 .. gc1 (a word reaching past a
+      // tensor's end is read only up to it: the last tile of K)
+      const uint64_t step_sc = 2ull * (uint64_t)(it_begin + it) * kBK * (uint64_t)NG;
+      const uint64_t step_z = (uint64_t)(it_begin + it) * kBK * (uint64_t)NG;
+      const bool last = it_begin + it == a.k_iters - 1;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int rr = lane + 32 * r;
+        for (uint32_t j = 0; j < nws[r]; ++j) {  // (nws = 0 when the scales come by TMA; nwz likewise)
+          const uint64_t o = sw0[r] + step_sc + 4 * j;
+          cp_async4(dst + kVScOff + rr * kVScRow + 4 * j, sc8 + o, last && sc_bytes - o < 4 ? (uint32_t)(sc_bytes - o) : 4u);
+        }
+        for (uint32_t j = 0; j < nwz[r]; ++j) {
+          const uint64_t o = zw0[r] + step_z + 4 * j;
+          cp_async4(dst + kVZOff + rr * kVZRow + 4 * j, a.zeros + o, last && z_bytes - o < 4 ? (uint32_t)(z_bytes - o) : 4u);
+        }
+      }
+      cp_async_arrive(bar);
+      issued = it + 1;
+    }
+    // on an abort, let the copies in flight land before the CTA exits
+    if (*(volatile int *)&s_abort && lane == 0)
+      for (int it = issued > kVStages ? issued - kVStages : 0; it < issued; ++it)
+        mbar_wait(smem_u32(&bar_full[it % kVStages]), (it / kVStages) & 1);
+  } else {
+    // ---------------- consumers ----------------
+    const int r0 = 16 * q + 2 * t;  // rows r0, r0 + 1, r0 + 8, r0 + 9 of every tile
+    // 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
+    const uint32_t chunk = 4 * h + (g >> 1), within = 8 * (g & 1);
+    const uint32_t off0 = r0 * 128 + ((chunk ^ (uint32_t)(2 * t)) << 4) + within;
+    const uint32_t off1 = (r0 + 1) * 128 + ((chunk ^ (uint32_t)(2 * t + 1)) << 4) + within;
+    const uint32_t xo0 = kWBytes + g * 128 + (((uint32_t)(2 * q) ^ (uint32_t)g) << 4) + 4 * t;
+    const uint32_t xo1 = kWBytes + g * 128 + (((uint32_t)(2 * q + 1) ^ (uint32_t)g) << 4) + 4 * t;
+    const int64_t gcol = (n0 + 128 * h + 16 * g) / a.group_size, gc0 = n0 / a.group_size;
+    const bool has_z = a.zeros != nullptr;
+    // where this thread's scale and zero point sit in a row's words: row k's
+    // words start at 4-byte boundary below element k NG + gc0; the offset
+    // depends on k only through k mod 4, and the thread's rows r0 + {0, 1,
+    // 8, 9} of a tile (k0 a multiple of 64) have k mod 4 = (r0 + {0, 1}) mod 4
+    // (from a TMA box: the offset of gcol from the box's first element, the
+    // same in every row)
+    uint32_t soff[2], zoff[2];
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      const uint64_t e = (uint64_t)((r0 + p) & 3) * (uint64_t)(NG & 3) + (uint64_t)gc0;
+      soff[p] = a.sc_box ? 2u * (uint32_t)(gcol - (gc0 / 8) * 8) : 2u * (uint32_t)(e & 1) + 2u * (uint32_t)(gcol - gc0);
+      zoff[p] = a.z_box ? (uint32_t)(gcol - (gc0 / 16) * 16) : (uint32_t)(e & 3) + (uint32_t)(gcol - gc0);
+    }
+    const uint32_t sp = a.sc_box ? 2u * (uint32_t)a.sc_box : kVScRow, zp = a.z_box ? (uint32_t)a.z_box : kVZRow;
+    const uint32_t srow0 = kVScOff + r0 * sp, zrow0 = kVZOff + r0 * zp;
+    bool ok = true;
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int s = it % kVStages;
+      // the warp goes on only together (a wait that ran out in one lane ends the whole warp's loop)
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_full[s]), (it / kVStages) & 1))) {
+        if (lane == 0) fail();
+        ok = false;
+        break;
+      }
+      if (*(volatile int *)&s_abort) break;
+      const uint32_t st = sbase + s * kVStage;  // shared-window address of the slot
+      const uint2 w0 = lds64(st + off0);
+      const uint2 w1 = lds64(st + off1);
+      const uint2 w2 = lds64(st + off0 + 8 * 128);
+      const uint2 w3 = lds64(st + off1 + 8 * 128);
+      const uint32_t b0 = lds32(st + xo0);
+      const uint32_t b1 = lds32(st + xo1);
+      uint32_t sc[4], zr[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t row = (i & 1) + 8 * (i >> 1);
+        sc[i] = lds16(st + srow0 + row * sp + soff[i & 1]);
+        zr[i] = has_z ? lds8(st + zrow0 + row * zp + zoff[i & 1]) : 0u;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_empty[s]));  // the slot is in registers now
+      // zero-point magics (1024 + z, 64 + z) and scales of the row pairs (r0, r0 + 1), (r0 + 8, r0 + 9)
+      const uint32_t zloA = 0x64006400u | zr[0] | (zr[1] << 16), zloB = 0x64006400u | zr[2] | (zr[3] << 16);
+      const uint32_t zhiA = has_z ? hadd2_rn(hsub2_rn(zloA, 0x64006400u), 0x54005400u) : 0x54005400u;
+      const uint32_t zhiB = has_z ? hadd2_rn(hsub2_rn(zloB, 0x64006400u), 0x54005400u) : 0x54005400u;
+      const uint32_t sA = sc[0] | (sc[1] << 16), sB = sc[2] | (sc[3] << 16);
+      uint32_t a0, a1, a2, a3;
+#define LT_GEMV_MMA(J, WA, WB, WC, WD)                  \
+  int4_rowpair<(J) & 3>(WA, WB, zloA, zhiA, sA, a0, a1); \
+  int4_rowpair<(J) & 3>(WC, WD, zloB, zhiB, sB, a2, a3); \
+  mma_16816(acc[J], a0, a1, a2, a3, b0, b1);
+      LT_GEMV_MMA(0, w0.x, w1.x, w2.x, w3.x)
+      LT_GEMV_MMA(1, w0.x, w1.x, w2.x, w3.x)
+      LT_GEMV_MMA(2, w0.x, w1.x, w2.x, w3.x)
+      LT_GEMV_MMA(3, w0.x, w1.x, w2.x, w3.x)
+      LT_GEMV_MMA(4, w0.y, w1.y, w2.y, w3.y)
+      LT_GEMV_MMA(5, w0.y, w1.y, w2.y, w3.y)
+      LT_GEMV_MMA(6, w0.y, w1.y, w2.y, w3.y)
+      LT_GEMV_MMA(7, w0.y, w1.y, w2.y, w3.y)
+#undef LT_GEMV_MMA
+    }
+  }
+  __syncthreads();  // every tile consumed (or the CTA aborted): the ring is free
+  if (*(volatile int *)&s_abort || n_it <= 0) return;
+  // ---------------- the four K slots' sums, in slot order ----------------
+  // red[q][m][c + c / 32]: the padding and the pitch (290 = 2 mod 32) make
+  // both the scattered stores below and the row reads after them conflict-free
+  float *red = reinterpret_cast<float *>(sm);
+  if (warp > 0) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = 128 * h + 16 * g + 2 * j + (e >> 1), m = 2 * t + (e & 1);
+        red[(q * 8 + m) * kVRedPitch + c + (c >> 5)] = acc[j][e];
+      }
+  }
+  __syncthreads();
+  if (warp > 0) {
+    const int c = tid - 32;  // 0 .. 255
+    for (int m = 0; m < 8 && m < a.M; ++m) {
+      float v = red[(0 * 8 + m) * kVRedPitch + c + (c >> 5)];
+#pragma unroll
+      for (int qq = 1; qq < 4; ++qq) v += red[(qq * 8 + m) * kVRedPitch + c + (c >> 5)];
+      if (a.splits == 1)
+        a.out[(int64_t)m * a.N + n0 + c] = __half_as_ushort(__float2half_rn(v));
+      else
+        a.partial[((int64_t)split * a.M + m) * a.N + n0 + c] = v;
+    }
   }
 }
 
-// K splits of the small-batch kernel: about two CTAs per SM, each split at
-// least 256 rows
+// K splits of the small-batch kernel: the fewest that fill at least 90 % of
+// the resident CTA slots of the waves they take (else the best fill), each
+// split at least one tile
 int gemv_splits(int64_t N, int64_t K) {
-  const int64_t tiles = N / kVCols;
-  int64_t s = (2 * (int64_t)num_sms() + tiles - 1) / tiles;
-  if (s > K / 256) s = K / 256;
-  if (s > 64) s = 64;
-  return (int)(s < 1 ? 1 : s);
+  const int64_t strips = N / kBN, k_tiles = K / kBK, slots = (int64_t)kVPerSM * num_sms();
+  int best = 1;
+  double best_fill = 0.0;
+  for (int64_t s = 1; s <= 64 && s <= k_tiles; ++s) {
+    const int64_t ctas = strips * s, waves = (ctas + slots - 1) / slots;
+    const double fill = (double)ctas / (double)(waves * slots);
+    if (fill >= 0.9) return (int)s;
+    if (fill > best_fill + 1e-9) {
+      best_fill = fill;
+      best = (int)s;
+    }
+  }
+  return best;
 }
 
 // out[m, n] = fp16_rn(sum over splits s = 0, 1, ... of partial[s, m, n]), in that order
 __global__ void __launch_bounds__(256) k_gemm_reduce(const float4 *__restrict__ partial, int64_t mn4, int splits,
                                                      uint2 *__restrict__ out) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the partials are complete (no-op in a plain launch)
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < mn4; i += (int64_t)gridDim.x * blockDim.x) {
     float4 acc = partial[i];
     for (int s = 1; s < splits; ++s) {
@@ -556,39 +795,14 @@ LT_API lt_status lt_int4_gemm(const lt_half *x, int64_t M, int64_t K, const uint
   if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(out, 16) || !aligned(scales, 2) ||
       !aligned(workspace, 16) || !aligned(d_status, 4))
     return LT_ERR_MISALIGNED;
-  cudaStream_t st = (cudaStream_t)stream;
-  auto reduce_splits = [&](int splits) {
-    const int64_t mn4 = M * N / 4;
-    int64_t g = (mn4 + 255) / 256;
-    const int64_t cap = (int64_t)num_sms() * 8;
-    if (g > cap) g = cap;
-    k_gemm_reduce<<<(int)g, 256, 0, st>>>(reinterpret_cast<const float4 *>(workspace), mn4, splits,
-                                          reinterpret_cast<uint2 *>(out));
-  };
-  if (M <= 8) {  // small batch: the CUDA-core kernel
-    int splits = gemv_splits(N, K);
-    if (splits > 1 && (!workspace || workspace_bytes < (uint64_t)splits * (uint64_t)M * (uint64_t)N * 4ull)) splits = 1;
-    const dim3 grid((unsigned)(N / kVCols), (unsigned)splits);
-    const uint32_t *pw = reinterpret_cast<const uint32_t *>(packed);
-    float *part = reinterpret_cast<float *>(workspace);
-    if (M == 1)
-      k_int4_gemv<1><<<grid, kVThreads, 0, st>>>(x, M, K, pw, scales, zeros, N, group_size, out, part, splits);
-    else if (M == 2)
-      k_int4_gemv<2><<<grid, kVThreads, 0, st>>>(x, M, K, pw, scales, zeros, N, group_size, out, part, splits);
-    else if (M <= 4)
-      k_int4_gemv<4><<<grid, kVThreads, 0, st>>>(x, M, K, pw, scales, zeros, N, group_size, out, part, splits);
-    else
-      k_int4_gemv<8><<<grid, kVThreads, 0, st>>>(x, M, K, pw, scales, zeros, N, group_size, out, part, splits);
-    if (splits > 1) reduce_splits(splits);
-    return launch_status();
-  }
+  const bool small = M <= 8;  // the mma.sync kernel (x tile of 8 rows) instead of the tcgen05 one (128 rows)
   encode_tiled_t enc = encoder();
   if (!enc) return LT_ERR_CUDA;
   CUtensorMap map_x, map_w;
   {
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kBM};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)(small ? 8 : kBM)};
     const cuuint32_t es[2] = {1, 1};
     if (enc(&map_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void *)x, dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -606,10 +820,48 @@ LT_API lt_status lt_int4_gemm(const lt_half *x, int64_t M, int64_t K, const uint
       return LT_ERR_CUDA;
   }
   const int64_t tiles_m = (M + kBM - 1) / kBM, tiles_n = N / kBN;
-  int splits = choose_splits(tiles_m * tiles_n, K / kBK);
-  if (splits > 1 && (!workspace || workspace_bytes < (uint64_t)splits * (uint64_t)M * (uint64_t)N * 4ull)) splits = 1;
   if (tiles_m > 65535) return LT_ERR_UNSUPPORTED;
+  int splits = small ? gemv_splits(N, K) : choose_splits(tiles_m * tiles_n, K / kBK);
+  if (splits > 1 && (!workspace || workspace_bytes < (uint64_t)splits * (uint64_t)M * (uint64_t)N * 4ull)) splits = 1;
+  // small batch: scale / zero-point tiles by TMA where the row pitch is a
+  // multiple of 16 bytes and a box of the chosen width, started at the
+  // 16-byte boundary at or below each strip's first group, covers the
+  // strip's last group (else word copies)
+  int sc_box = 0, z_box = 0;
+  CUtensorMap map_s = map_w, map_z = map_w;
+  if (small) {
+    const int64_t NG = N / group_size, strips = N / kBN;
+    int64_t span_s = 0, span_z = 0;  // max over strips of last group - box start
+    for (int64_t j = 0; j < strips; ++j) {
+      const int64_t g0 = j * kBN / group_size, g1 = (j * kBN + kBN - 1) / group_size;
+      span_s = std::max(span_s, g1 - (g0 / 8) * 8);
+      span_z = std::max(span_z, g1 - (g0 / 16) * 16);
+    }
+    if (aligned(scales, 16) && (NG * 2) % 16 == 0 && span_s < 16) sc_box = span_s < 8 ? 8 : 16;
+    if (zeros && aligned(zeros, 16) && NG % 16 == 0 && span_z < 32) z_box = span_z < 16 ? 16 : 32;
+    const cuuint32_t es[2] = {1, 1};
+    if (sc_box) {
+      const cuuint64_t dims[2] = {(cuuint64_t)NG, (cuuint64_t)K};
+      const cuuint64_t strides[1] = {(cuuint64_t)NG * 2};
+      const cuuint32_t box[2] = {(cuuint32_t)sc_box, (cuuint32_t)kBK};
+      if (enc(&map_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (void *)scales, dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return LT_ERR_CUDA;
+    }
+    if (z_box) {
+      const cuuint64_t dims[2] = {(cuuint64_t)NG, (cuuint64_t)K};
+      const cuuint64_t strides[1] = {(cuuint64_t)NG};
+      const cuuint32_t box[2] = {(cuuint32_t)z_box, (cuuint32_t)kBK};
+      if (enc(&map_z, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void *)zeros, dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return LT_ERR_CUDA;
+    }
+  }
   GemmArgs ga;
+  ga.sc_box = sc_box;
+  ga.z_box = z_box;
   ga.scales = scales;
   ga.zeros = zeros;
   ga.out = out;
@@ -621,16 +873,43 @@ LT_API lt_status lt_int4_gemm(const lt_half *x, int64_t M, int64_t K, const uint
   ga.group_size = group_size;
   ga.k_iters = (int32_t)(K / kBK);
   ga.splits = splits;
-  static int attr_set[64] = {0};
+  static int attr_set[2][64] = {{0}};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(k_int4_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemDyn) != cudaSuccess)
+  if (dev >= 0 && dev < 64 && !attr_set[small][dev]) {
+    if (cudaFuncSetAttribute(small ? (const void *)k_int4_gemv : (const void *)k_int4_gemm,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(small ? kVSmemDyn : kSmemDyn)) !=
+        cudaSuccess)
       return LT_ERR_CUDA;
-    attr_set[dev] = 1;
+    attr_set[small][dev] = 1;
   }
-  k_int4_gemm<<<dim3((unsigned)tiles_n, (unsigned)tiles_m, (unsigned)splits), kGemmThreads, kSmemDyn, st>>>(map_x,
-                                                                                                         map_w, ga);
-  if (splits > 1) reduce_splits(splits);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (small)
+    k_int4_gemv<<<dim3((unsigned)tiles_n, (unsigned)splits), kVThreads, kVSmemDyn, st>>>(map_x, map_w, map_s, map_z,
+                                                                                           ga);
+  else
+    k_int4_gemm<<<dim3((unsigned)tiles_n, (unsigned)tiles_m, (unsigned)splits), kGemmThreads, kSmemDyn, st>>>(
+        map_x, map_w, ga);
+  if (splits > 1) {
+    // the split sums in order; launched as a programmatic dependent of the
+    // product kernel, so its launch overlaps that kernel's tail (it waits for
+    // the kernel's completion and memory before reading a partial)
+    const int64_t mn4 = M * N / 4;
+    int64_t g = (mn4 + 255) / 256;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (g > cap) g = cap;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)g);
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_gemm_reduce, reinterpret_cast<const float4 *>(workspace), mn4, splits,
+                           reinterpret_cast<uint2 *>(out)) != cudaSuccess)
+      return launch_status();
+  }
   return launch_status();
 }
