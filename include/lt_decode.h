@@ -435,7 +435,9 @@ lt_status lt_lz4_int4_decode_noalloc(const uint8_t *comp, uint64_t comp_bytes, c
  *            binary16 scales and uint8 zero points (or NULL) laid out
  *            [K, N/group_size]. W[k, n] is exactly lt_dequant_int4's output
  *            element k*N + n; it is never written to memory: each tile is
- *            decoded into shared memory and fed to the tensor cores.
+ *            decoded on chip and fed to the tensor cores (for M > 16 into
+ *            shared memory as the B operand of tcgen05.mma; for M <= 16
+ *            straight into the registers of mma.sync).
  *   out      M x N binary16, row-major, 16-byte aligned: the fp32 sum of the
  *            exact products x[m, k] * W[k, n] over k, rounded once to
  *            binary16. The order of the fp32 additions is the hardware's

@@ -79,6 +79,8 @@ def check(got_bits, want, absum, K, what):
                                            # (tiles of both by TMA), and a group of 96 (boxes straddling groups)
                                            (4, 512, 4096, 128, True), (6, 256, 512, 32, True), (2, 384, 768, 96, True),
                                            (7, 192, 2048, 64, False),
+                                           # two blocks of 8 batch rows (9 .. 16 rows)
+                                           (12, 512, 1024, 128, True), (16, 256, 4096, 128, True), (16, 320, 256, 32, False),
                                            (128, 256, 512, 64, False),
                                            (200, 512, 768, 256, True), (129, 1024, 256, 128, True),
                                            (300, 64, 1024, 32, False)])
@@ -108,9 +110,9 @@ def test_gemm_identity_input_returns_the_decoded_weights():
     assert np.array_equal(got.ravel(), host_bits(w))
 
 
-@pytest.mark.parametrize("M,N", [(1, 512), (3, 512), (8, 512), (1, 4096), (5, 4096)])
+@pytest.mark.parametrize("M,N", [(1, 512), (3, 512), (8, 512), (1, 4096), (5, 4096), (11, 512), (16, 4096)])
 def test_gemm_small_batch_unit_rows_return_rows_of_the_decoded_weights(M, N):
-    # batches of at most 8 rows take the mma.sync kernel: with x[m] the unit
+    # batches of at most 16 rows take the mma.sync kernel: with x[m] the unit
     # vector e_(k_m), out[m] is row k_m of W, one exact product per element,
     # so it equals lt_dequant_int4's output bit for bit (N = 512: scales and
     # zero points copied word by word; N = 4096: by TMA)

@@ -411,19 +411,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
 }
 
 // ---------------------------------------------------------------------------
-// Small batches (M <= 8). With a few rows of x the 128-row tcgen05 tile is
+// Small batches (M <= 16). With a few rows of x the 128-row tcgen05 tile is
 // mostly padding, while its decoded operand still makes a round trip through
 // shared memory; the product is bound by streaming the codes from HBM. Here
 // the codes stream through a TMA ring and each thread decodes them straight
 // into the register operands of mma.sync.m16n8k16 (fp16 in, fp32
 // accumulate), computing out^T = W^T . x^T: the MMA's 16 rows are 16 columns
-// of W, its 16-deep reduction 16 rows of K, its 8 columns the batch.
+// of W, its 16-deep reduction 16 rows of K, its 8 columns 8 rows of the
+// batch (two MMAs per A fragment for 9 .. 16 rows).
 //
 // One CTA: 256 columns [n0, n0 + 256) over a range of 64-row K tiles (a
 // split of K). Warp 0 is the producer: per tile one TMA copy of the packed
-// codes (64 rows x 128 bytes, 128-byte swizzle) and one of x (8 batch rows x
-// 64 fp16, rows past M zero-filled) into an 8-deep ring, plus an L2 prefetch
-// of the tile's scales and zero points. Warps 1..8: warp 1 + 2 q + h takes
+// codes (64 rows x 128 bytes, 128-byte swizzle), one of x (8 or 16 batch
+// rows x 64 fp16, rows past M zero-filled) and the tile's scales and zero
+// points (TMA boxes or word copies, below) into a 7-deep ring, completion
+// counted on the slot's full barrier. Warps 1..8: warp 1 + 2 q + h takes
 // column half h (128 columns) and rows 16 q .. 16 q + 15 of every tile.
 // Lane (g, t) = (lane / 4, lane % 4) holds, for the 8 MMAs j = 0..7 of a
 // tile, code byte j of its 8-byte slice (columns 16 g + 2 j and + 1 of the
@@ -436,9 +438,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
 // ---------------------------------------------------------------------------
 constexpr int kVWarps = 8;                       // consumer warps
 constexpr int kVThreads = 32 * (kVWarps + 1);    // + the producer warp
-constexpr int kVStages = 8;
+constexpr int kVStages = 7;
 constexpr int kVPerSM = 2;                       // resident CTAs per SM (launch bounds, shared memory)
-constexpr uint32_t kVXBytes = 8 * kBK * 2;       // x tile: 8 rows x 64 fp16
+constexpr uint32_t kVXBytes = 16 * kBK * 2;      // x tile: up to 16 rows x 64 fp16
 // each row's scales and zero points of the strip: a TMA box of 8 or 16
 // scales / 16 or 32 zero points per row starting at a 16-byte boundary at or
 // below the strip's first group, or (where the tensors' row pitch is not a
@@ -447,11 +449,11 @@ constexpr uint32_t kVXBytes = 8 * kBK * 2;       // x tile: 8 rows x 64 fp16
 // zero points)
 constexpr uint32_t kVScRow = 20, kVZRow = 12;  // word-copy row pitches
 constexpr uint32_t kVScOff = kWBytes + kVXBytes, kVZOff = kVScOff + kBK * 32;
-constexpr uint32_t kVStage = kVZOff + kBK * 32;  // 13312, a multiple of 1 KB (swizzle atoms stay aligned)
+constexpr uint32_t kVStage = kVZOff + kBK * 32;  // 14336, a multiple of 1 KB (swizzle atoms stay aligned)
 static_assert(kVStage % 1024 == 0, "stage size");
 constexpr uint32_t kVRing = kVStages * kVStage;
 constexpr int kVRedPitch = 290;                  // fp32 words per batch row of the reduction buffer
-constexpr uint32_t kVRedBytes = 4u * 8u * kVRedPitch * 4u;
+constexpr uint32_t kVRedBytes = 4u * 16u * kVRedPitch * 4u;
 static_assert(kVRedBytes <= kVRing, "the reduction buffer reuses the ring");
 constexpr uint32_t kVSmemDyn = kVRing + 1024;
 
@@ -493,6 +495,7 @@ __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+template <int NB>  // batch rows in blocks of 8 (the MMA's N): 1 or 2
 __global__ void __launch_bounds__(kVThreads, kVPerSM) k_int4_gemv(const __grid_constant__ CUtensorMap map_x,
                                                                    const __grid_constant__ CUtensorMap map_w,
                                                                    const __grid_constant__ CUtensorMap map_s,
@@ -528,11 +531,13 @@ __global__ void __launch_bounds__(kVThreads, kVPerSM) k_int4_gemv(const __grid_c
     report(a.d_status, LT_ERR_TIMEOUT);
   };
 
-  float acc[8][4];
+  float acc[NB][8][4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
+  for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[nb][j][e] = 0.f;
   const int cw = warp - 1, h = cw & 1, q = cw >> 1, g = lane >> 2, t = lane & 3;
 
   if (warp == 0) {
@@ -554,7 +559,7 @@ __global__ void __launch_bounds__(kVThreads, kVPerSM) k_int4_gemv(const __grid_c
       nwz[r] = (a.zeros && !a.z_box) ? (uint32_t)((ze - zw0[r] + 3) / 4) : 0u;
     }
     const int64_t xs = (gc0 / 8) * 8, xz = (gc0 / 16) * 16;  // TMA boxes start at 16-byte boundaries
-    const uint32_t tx_bytes = kWBytes + kVXBytes + (uint32_t)(kBK * 2 * a.sc_box) + (uint32_t)(kBK * a.z_box);
+    const uint32_t tx_bytes = kWBytes + (uint32_t)(NB * 8 * kBK * 2) + (uint32_t)(kBK * 2 * a.sc_box) + (uint32_t)(kBK * a.z_box);
     int issued = 0;
     for (int it = 0; it < n_it; ++it) {
       const int s = it % kVStages;
@@ -640,8 +645,12 @@ __global__ void __launch_bounds__(kVThreads, kVPerSM) k_int4_gemv(const __grid_c
       const uint2 w1 = lds64(st + off1);
       const uint2 w2 = lds64(st + off0 + 8 * 128);
       const uint2 w3 = lds64(st + off1 + 8 * 128);
-      const uint32_t b0 = lds32(st + xo0);
-      const uint32_t b1 = lds32(st + xo1);
+      uint32_t b0[NB], b1[NB];
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {  // batch rows g + 8 nb: 8 x rows (1 KB) further, the same swizzle
+        b0[nb] = lds32(st + xo0 + 1024 * nb);
+        b1[nb] = lds32(st + xo1 + 1024 * nb);
+      }
       uint32_t sc[4], zr[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -660,7 +669,7 @@ __global__ void __launch_bounds__(kVThreads, kVPerSM) k_int4_gemv(const __grid_c
 #define LT_GEMV_MMA(J, WA, WB, WC, WD)                  \
   int4_rowpair<(J) & 3>(WA, WB, zloA, zhiA, sA, a0, a1); \
   int4_rowpair<(J) & 3>(WC, WD, zloB, zhiB, sB, a2, a3); \
-  mma_16816(acc[J], a0, a1, a2, a3, b0, b1);
+  for (int nb = 0; nb < NB; ++nb) mma_16816(acc[nb][J], a0, a1, a2, a3, b0[nb], b1[nb]);
       LT_GEMV_MMA(0, w0.x, w1.x, w2.x, w3.x)
       LT_GEMV_MMA(1, w0.x, w1.x, w2.x, w3.x)
       LT_GEMV_MMA(2, w0.x, w1.x, w2.x, w3.x)
@@ -675,25 +684,27 @@ __global__ void __launch_bounds__(kVThreads, kVPerSM) k_int4_gemv(const __grid_c
   __syncthreads();  // every tile consumed (or the CTA aborted): the ring is free
   if (*(volatile int *)&s_abort || n_it <= 0) return;
   // ---------------- the four K slots' sums, in slot order ----------------
-  // red[q][m][c + c / 32]: the padding and the pitch (290 = 2 mod 32) make
+  // red[q][m][c + c / 32] (m < 16): the padding and the pitch (290 = 2 mod 32) make
   // both the scattered stores below and the row reads after them conflict-free
   float *red = reinterpret_cast<float *>(sm);
   if (warp > 0) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = 128 * h + 16 * g + 2 * j + (e >> 1), m = 2 * t + (e & 1);
-        red[(q * 8 + m) * kVRedPitch + c + (c >> 5)] = acc[j][e];
-      }
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = 128 * h + 16 * g + 2 * j + (e >> 1), m = 8 * nb + 2 * t + (e & 1);
+          red[(q * 16 + m) * kVRedPitch + c + (c >> 5)] = acc[nb][j][e];
+        }
   }
   __syncthreads();
   if (warp > 0) {
     const int c = tid - 32;  // 0 .. 255
-    for (int m = 0; m < 8 && m < a.M; ++m) {
-      float v = red[(0 * 8 + m) * kVRedPitch + c + (c >> 5)];
+    for (int m = 0; m < 8 * NB && m < a.M; ++m) {
+      float v = red[(0 * 16 + m) * kVRedPitch + c + (c >> 5)];
 #pragma unroll
-      for (int qq = 1; qq < 4; ++qq) v += red[(qq * 8 + m) * kVRedPitch + c + (c >> 5)];
+      for (int qq = 1; qq < 4; ++qq) v += red[(qq * 16 + m) * kVRedPitch + c + (c >> 5)];
       if (a.splits == 1)
         a.out[(int64_t)m * a.N + n0 + c] = __half_as_ushort(__float2half_rn(v));
       else
@@ -776,7 +787,7 @@ using namespace lt;
 LT_API uint64_t lt_int4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < kBN || K < kBK || N % kBN != 0 || K % kBK != 0) return 0;
   int s;
-  if (M <= 8) {
+  if (M <= 16) {
     s = gemv_splits(N, K);
   } else {
     const int64_t tiles = ((M + kBM - 1) / kBM) * (N / kBN);
@@ -795,14 +806,15 @@ LT_API lt_status lt_int4_gemm(const lt_half *x, int64_t M, int64_t K, const uint
   if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(out, 16) || !aligned(scales, 2) ||
       !aligned(workspace, 16) || !aligned(d_status, 4))
     return LT_ERR_MISALIGNED;
-  const bool small = M <= 8;  // the mma.sync kernel (x tile of 8 rows) instead of the tcgen05 one (128 rows)
+  const bool small = M <= 16;  // the mma.sync kernel (x tile of 8 or 16 rows) instead of the tcgen05 one (128 rows)
+  const int nb = M <= 8 ? 1 : 2;
   encode_tiled_t enc = encoder();
   if (!enc) return LT_ERR_CUDA;
   CUtensorMap map_x, map_w;
   {
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)(small ? 8 : kBM)};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)(small ? 8 * nb : kBM)};
     const cuuint32_t es[2] = {1, 1};
     if (enc(&map_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void *)x, dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -873,20 +885,26 @@ LT_API lt_status lt_int4_gemm(const lt_half *x, int64_t M, int64_t K, const uint
   ga.group_size = group_size;
   ga.k_iters = (int32_t)(K / kBK);
   ga.splits = splits;
-  static int attr_set[2][64] = {{0}};
+  static int attr_set[3][64] = {{0}};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[small][dev]) {
-    if (cudaFuncSetAttribute(small ? (const void *)k_int4_gemv : (const void *)k_int4_gemm,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(small ? kVSmemDyn : kSmemDyn)) !=
+  const int which = small ? nb : 0;
+  if (dev >= 0 && dev < 64 && !attr_set[which][dev]) {
+    const void *fn = which == 0 ? (const void *)k_int4_gemm
+                                : which == 1 ? (const void *)k_int4_gemv<1> : (const void *)k_int4_gemv<2>;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(small ? kVSmemDyn : kSmemDyn)) !=
         cudaSuccess)
       return LT_ERR_CUDA;
-    attr_set[small][dev] = 1;
+    attr_set[which][dev] = 1;
   }
   cudaStream_t st = (cudaStream_t)stream;
   if (small)
-    k_int4_gemv<<<dim3((unsigned)tiles_n, (unsigned)splits), kVThreads, kVSmemDyn, st>>>(map_x, map_w, map_s, map_z,
-                                                                                           ga);
+    if (nb == 1)
+      k_int4_gemv<1><<<dim3((unsigned)tiles_n, (unsigned)splits), kVThreads, kVSmemDyn, st>>>(map_x, map_w, map_s,
+                                                                                              map_z, ga);
+    else
+      k_int4_gemv<2><<<dim3((unsigned)tiles_n, (unsigned)splits), kVThreads, kVSmemDyn, st>>>(map_x, map_w, map_s,
+                                                                                              map_z, ga);
   else
     k_int4_gemm<<<dim3((unsigned)tiles_n, (unsigned)tiles_m, (unsigned)splits), kGemmThreads, kSmemDyn, st>>>(
         map_x, map_w, ga);
