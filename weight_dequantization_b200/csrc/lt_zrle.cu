@@ -127,28 +127,56 @@ __global__ void __launch_bounds__(kThreads, 6) k_zrle(const uint8_t *__restrict_
       //    and header go to lane k
       const int32_t lim = nbytes >= q + 4 ? (int32_t)((nbytes - q - 4) / 2 < 62 ? (nbytes - q - 4) / 2 : 62) : -1;
       const uint32_t rem = len - done;
-      uint32_t pp = p, k = 0, dsum = 0, myP = 0, myV = 0;
-      while ((int32_t)pp <= lim && dsum < rem) {  // at most 32 records: each takes >= 2 slots
-        const uint32_t v = __shfl_sync(0xFFFFFFFFu, (pp & 1) ? podd : pair, (int)(pp >> 1));
-        if (lane == k) {
-          myP = pp;
-          myV = v;
-        }
-        ++k;
-        dsum += (v & 0xFFFFu) + (v >> 16);
-        pp += 2 + (v >> 16);
+      // Record r of the window (at most 32: each takes >= 2 slots) goes to
+      // lane r by pointer jumping instead of a serial walk: for every slot s,
+      // the next record would start at nxt(s) = s + 2 + n_lit(s); jump[b]
+      // holds nxt^(2^b) for this lane's slots 2 lane and 2 lane + 1 (low and
+      // high halves; positions past the window saturate at 64), and lane r
+      // follows the binary digits of r from p.
+      uint32_t jump[5];
+      jump[0] = min(2 * lane + 2 + (pair >> 16), 64u) | (min(2 * lane + 3 + (podd >> 16), 64u) << 16);
+#pragma unroll
+      for (int b = 1; b < 5; ++b) {
+        const uint32_t q0 = jump[b - 1] & 0xFFFFu, q1 = jump[b - 1] >> 16;
+        const uint32_t t0 = __shfl_sync(0xFFFFFFFFu, jump[b - 1], (int)(q0 < 64 ? q0 >> 1 : 0));
+        const uint32_t t1 = __shfl_sync(0xFFFFFFFFu, jump[b - 1], (int)(q1 < 64 ? q1 >> 1 : 0));
+        const uint32_t r0 = q0 < 64 ? ((q0 & 1) ? t0 >> 16 : t0 & 0xFFFFu) : 64u;
+        const uint32_t r1 = q1 < 64 ? ((q1 & 1) ? t1 >> 16 : t1 & 0xFFFFu) : 64u;
+        jump[b] = r0 | (r1 << 16);
       }
-      // 3. the walked records, in parallel
-      const bool rec = lane < k;
-      const uint32_t zr = myV & 0xFFFFu, nl = myV >> 16;
-      const uint32_t lk = rec ? zr + nl : 0u;
-      uint32_t incl = lk;
+      uint32_t myP = p < 64 ? p : 64u;
+#pragma unroll
+      for (int b = 0; b < 5; ++b) {
+        const uint32_t t = __shfl_sync(0xFFFFFFFFu, jump[b], (int)(myP < 64 ? myP >> 1 : 0));
+        const uint32_t nx = myP < 64 ? ((myP & 1) ? t >> 16 : t & 0xFFFFu) : 64u;
+        if ((lane >> b) & 1) myP = nx;
+      }
+      const uint32_t vsrc = myP < 64 ? myP >> 1 : 0;
+      const uint32_t vp = __shfl_sync(0xFFFFFFFFu, pair, (int)vsrc), vo = __shfl_sync(0xFFFFFFFFu, podd, (int)vsrc);
+      const bool inwin = (int32_t)myP <= lim;  // a header in the window and in the chunk's bytes
+      uint32_t myV = inwin ? ((myP & 1) ? vo : vp) : 0u;
+      // the records before the chunk is full (the serial walk's stop rule)
+      const uint32_t lk0 = (myV & 0xFFFFu) + (myV >> 16);
+      uint32_t incl = lk0;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, off);
         if ((int)lane >= off) incl += t;
       }
-      const uint32_t before = incl - lk;  // elements of the window's earlier records
+      const unsigned validm = __ballot_sync(0xFFFFFFFFu, inwin && incl - lk0 < rem);
+      const uint32_t k = (~validm) ? (uint32_t)(__ffs(~validm) - 1) : 32u;  // leading valid records
+      uint32_t dsum = 0, pp = p;
+      if (k) {
+        dsum = __shfl_sync(0xFFFFFFFFu, incl, (int)k - 1);
+        const uint32_t lp = __shfl_sync(0xFFFFFFFFu, myP, (int)k - 1), lv = __shfl_sync(0xFFFFFFFFu, myV, (int)k - 1);
+        pp = lp + 2 + (lv >> 16);
+      }
+      // 3. the walked records, in parallel
+      const bool rec = lane < k;
+      if (!rec) myV = 0;
+      const uint32_t zr = myV & 0xFFFFu, nl = myV >> 16;
+      const uint32_t lk = rec ? zr + nl : 0u;
+      const uint32_t before = incl - lk0;  // elements of the window's earlier records
       const bool bad = rec && ((uint64_t)done + before + lk > len || q + 2 * ((uint64_t)myP + 2 + nl) > nbytes);
       const unsigned badm = __ballot_sync(0xFFFFFFFFu, bad);
       const uint32_t ok = badm ? (uint32_t)(__ffs(badm) - 1) : k;  // records before the first bad one
