@@ -1020,7 +1020,7 @@ def gemm_timing(hbm_peak: float, reps: int = 10, warmup: int = 3, shapes=GEMM_SH
 
 def checksum_timing(dw, hw, peak: float, reps: int = 20, warmup: int = 3):
     """Per-block XXH3-64 on C4's compressed stream (448 blocks): the
-    standalone verifier (lt_xxh3_blocks, one warp per block) and the decode
+    standalone verifier (lt_xxh3_blocks, one CTA per block) and the decode
     with the check fused in (lt_lz4_int4_decode_checked) against the plain
     fused decode. Device time by CUDA events, median of `reps`, an L2 flush
     (L2Flush) before each call (not timed)."""
@@ -1074,7 +1074,7 @@ def checksum_timing(dw, hw, peak: float, reps: int = 20, warmup: int = 3):
     del flush
     return {"label": f"XXH3-64 per LZ4 block of C4 ({nb} blocks, {comp_bytes} compressed bytes, 192-byte secret); "
                      f"L2 flushed before each of {reps} calls",
-            "kernel": "k_xxh3_blocks (warp per block)", "us_verify": t_hash * 1e6, "verify_GBps": hb / t_hash / 1e9,
+            "kernel": "k_xxh3_blocks (one CTA per block)", "us_verify": t_hash * 1e6, "verify_GBps": hb / t_hash / 1e9,
             "verify_hbm_frac_of_measured": hb / t_hash / 1e9 / peak,
             "us_decode_plain": t_plain * 1e6, "us_decode_checked": t_checked * 1e6,
             "checked_overhead": t_checked / t_plain - 1.0}
