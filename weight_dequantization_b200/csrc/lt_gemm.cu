@@ -45,23 +45,31 @@ namespace lt {
 namespace {
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
-constexpr int kStagesW = 6;  // packed-W slots (TMA; freed by the decoders)
-constexpr int kStagesX = 3;  // x slots (TMA; freed by the MMAs)
-constexpr int kStagesB = 4;  // decoded-B slots: the decoders run up to three steps ahead of the MMAs
 constexpr int kDecWarps = 16;
 constexpr int kDec0 = 3;     // first decoder warp (0: packed-W producer, 1: MMA, 2: x producer)
 constexpr int kUnits = (kBK * kBN / 32) / (kDecWarps * 32);  // 16-byte packed chunks per decoder thread per step
 static_assert(kUnits * kDecWarps * 32 == kBK * kBN / 32, "decoder units must cover a packed tile");
 constexpr int kGemmThreads = (kDec0 + kDecWarps) * 32;
-constexpr uint32_t kABytes = kBM * kBK * 2;   // 16384
 constexpr uint32_t kWBytes = kBK * kBN / 2;   // 8192
 constexpr uint32_t kBBytes = kBN * kBK * 2;   // 32768
-constexpr uint32_t kSmemA = 0;
-constexpr uint32_t kSmemW = kSmemA + kStagesX * kABytes;
-constexpr uint32_t kSmemB = kSmemW + kStagesW * kWBytes;
-constexpr uint32_t kSmemTotal = kSmemB + kStagesB * kBBytes;  // 224 KB
-constexpr uint32_t kSmemDyn = kSmemTotal + 1024;              // + alignment slack
-constexpr uint32_t kTmemCols = 256;
+// A CTA of the tcgen05 kernel computes MT 128-row tiles of out (MT = 1 or
+// 2) against one 256-column tile: its MT accumulators (256 tensor-memory
+// columns each) share every decoded B tile, so with MT = 2 the decode and the
+// shared-memory round trip of B are spent once per 256 rows of x.
+template <int MT>
+struct Tile {
+  static constexpr int kStagesW = MT == 1 ? 6 : 4;  // packed-W slots (TMA; freed by the decoders)
+  static constexpr int kStagesX = 3;                // x slots (TMA; freed by the MMAs)
+  static constexpr int kStagesB = MT == 1 ? 4 : 3;  // decoded-B slots (the decoders run ahead of the MMAs)
+  static constexpr uint32_t kABytes = MT * kBM * kBK * 2;  // x tile: 16 or 32 KB
+  static constexpr uint32_t kSmemA = 0;
+  static constexpr uint32_t kSmemW = kSmemA + kStagesX * kABytes;
+  static constexpr uint32_t kSmemB = kSmemW + kStagesW * kWBytes;
+  static constexpr uint32_t kSmemTotal = kSmemB + kStagesB * kBBytes;  // 224 KB either way
+  static constexpr uint32_t kSmemDyn = kSmemTotal + 1024;              // + alignment slack
+  static constexpr uint32_t kTmemCols = 256 * MT;
+};
+static_assert(Tile<1>::kSmemDyn <= 227 * 1024 - 256 && Tile<2>::kSmemDyn <= 227 * 1024 - 256, "shared memory");
 // B operand (N-major, 128-byte swizzle): 1 KB atoms of 64 n x 8 k; atoms
 // along N are kBAtomN bytes apart, atoms along K 1 KB apart.
 constexpr uint32_t kBAtomN = (kBK / 8) * 1024;  // 8192
@@ -186,9 +194,14 @@ struct GemmArgs {
   int32_t sc_box, z_box;
 };
 
+template <int MT>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_constant__ CUtensorMap map_x,
                                                                  const __grid_constant__ CUtensorMap map_w,
                                                                  const __grid_constant__ GemmArgs a) {
+  using T = Tile<MT>;
+  constexpr int kStagesW = T::kStagesW, kStagesX = T::kStagesX, kStagesB = T::kStagesB;
+  constexpr uint32_t kABytes = T::kABytes, kSmemA = T::kSmemA, kSmemW = T::kSmemW, kSmemB = T::kSmemB;
+  constexpr uint32_t kTmemCols = T::kTmemCols;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t bar_wfull[kStagesW], bar_wempty[kStagesW], bar_xfull[kStagesX],
@@ -198,7 +211,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_tile = blockIdx.x, m_tile = blockIdx.y, split = blockIdx.z;
-  const int64_t n0 = (int64_t)n_tile * kBN, m0 = (int64_t)m_tile * kBM;
+  const int64_t n0 = (int64_t)n_tile * kBN, m0 = (int64_t)m_tile * kBM * MT;
   const int it_begin = (int)((int64_t)a.k_iters * split / a.splits);
   const int it_end = (int)((int64_t)a.k_iters * (split + 1) / a.splits);
   const int n_it = it_end - it_begin;
@@ -286,11 +299,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
         const uint32_t a0 = sbase + kSmemA + sx * kABytes, b0 = sbase + kSmemB + b * kBBytes;
 #pragma unroll
         for (int ks = 0; ks < kBK / 16; ++ks) {
-          // A: K-major 128-byte swizzle, 8-row atoms 1 KB apart, K = 16 slice at +32 bytes;
+          // A: K-major 128-byte swizzle, 8-row atoms 1 KB apart, K = 16 slice at +32 bytes
+          // (rows 128 mt ... of the x tile start 16 KB further per mt);
           // B: N-major 128-byte swizzle, K = 16 slice = two 1 KB atoms along K
-          const uint64_t ad = smem_desc(a0 + 32u * ks, 16, 1024);
           const uint64_t bd = smem_desc(b0 + 2u * kBAtomK * ks, kBAtomN, kBAtomK);
-          mma_f16(tmem, ad, bd, idesc, (it | ks) != 0);
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            const uint64_t ad = smem_desc(a0 + (uint32_t)mt * (kBM * 128u) + 32u * ks, 16, 1024);
+            mma_f16(tmem + 256u * mt, ad, bd, idesc, (it | ks) != 0);
+          }
         }
         mma_commit(smem_u32(&bar_xempty[sx]));
         mma_commit(smem_u32(&bar_bempty[b]));
@@ -372,13 +389,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_int4_gemm(const __grid_cons
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (acc_ok && !*(volatile int *)&s_abort && n_it > 0) {
       const int quarter = warp & 3;  // tensor-memory lanes 32 quarter .. + 31
-      const int64_t m = m0 + 32 * quarter + lane;
       // each quarter's 256 columns split among its kDecWarps / 4 decoder warps
       constexpr int kCols = kBN / (kDecWarps / 4);
       const int cbeg = ((warp - kDec0) / 4) * kCols;
-      for (int c0 = cbeg; c0 < cbeg + kCols; c0 += 32) {
+      for (int cm = 0; cm < MT * kCols; cm += 32) {
+        const int mt = cm / kCols, c0 = cbeg + cm % kCols;  // accumulator mt, columns c0 .. c0 + 31
+        const int64_t m = m0 + kBM * mt + 32 * quarter + lane;
         uint32_t r[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0, r);
+        tmem_ld32(tmem + ((uint32_t)(32 * quarter) << 16) + 256u * mt + (uint32_t)c0, r);
         if (m < a.M) {
           if (a.splits == 1) {
             uint4 *o = reinterpret_cast<uint4 *>(a.out + m * a.N + n0 + c0);
@@ -790,7 +808,8 @@ LT_API uint64_t lt_int4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= 16) {
     s = gemv_splits(N, K);
   } else {
-    const int64_t tiles = ((M + kBM - 1) / kBM) * (N / kBN);
+    const int64_t rows = M > kBM ? 2 * kBM : kBM;  // rows of out per CTA (the tcgen05 kernel's MT)
+    const int64_t tiles = ((M + rows - 1) / rows) * (N / kBN);
     s = choose_splits(tiles, K / kBK);
   }
   return s > 1 ? (uint64_t)s * (uint64_t)M * (uint64_t)N * 4ull : 0;
@@ -808,13 +827,14 @@ LT_API lt_status lt_int4_gemm(const lt_half *x, int64_t M, int64_t K, const uint
     return LT_ERR_MISALIGNED;
   const bool small = M <= 16;  // the mma.sync kernel (x tile of 8 or 16 rows) instead of the tcgen05 one (128 rows)
   const int nb = M <= 8 ? 1 : 2;
+  const int mt = M > kBM ? 2 : 1;  // tcgen05 kernel: 128-row tiles of out per CTA
   encode_tiled_t enc = encoder();
   if (!enc) return LT_ERR_CUDA;
   CUtensorMap map_x, map_w;
   {
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)(small ? 8 * nb : kBM)};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)(small ? 8 * nb : kBM * mt)};
     const cuuint32_t es[2] = {1, 1};
     if (enc(&map_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void *)x, dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -831,7 +851,7 @@ LT_API lt_status lt_int4_gemm(const lt_half *x, int64_t M, int64_t K, const uint
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return LT_ERR_CUDA;
   }
-  const int64_t tiles_m = (M + kBM - 1) / kBM, tiles_n = N / kBN;
+  const int64_t tiles_m = (M + kBM * mt - 1) / (kBM * mt), tiles_n = N / kBN;
   if (tiles_m > 65535) return LT_ERR_UNSUPPORTED;
   int splits = small ? gemv_splits(N, K) : choose_splits(tiles_m * tiles_n, K / kBK);
   if (splits > 1 && (!workspace || workspace_bytes < (uint64_t)splits * (uint64_t)M * (uint64_t)N * 4ull)) splits = 1;
@@ -885,29 +905,34 @@ LT_API lt_status lt_int4_gemm(const lt_half *x, int64_t M, int64_t K, const uint
   ga.group_size = group_size;
   ga.k_iters = (int32_t)(K / kBK);
   ga.splits = splits;
-  static int attr_set[3][64] = {{0}};
+  static int attr_set[4][64] = {{0}};
   int dev = 0;
   cudaGetDevice(&dev);
-  const int which = small ? nb : 0;
-  if (dev >= 0 && dev < 64 && !attr_set[which][dev]) {
-    const void *fn = which == 0 ? (const void *)k_int4_gemm
-                                : which == 1 ? (const void *)k_int4_gemv<1> : (const void *)k_int4_gemv<2>;
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(small ? kVSmemDyn : kSmemDyn)) !=
-        cudaSuccess)
+  const int which = small ? nb : 2 + mt;  // 1, 2: k_int4_gemv<nb>; 3, 4: k_int4_gemm<mt>
+  if (dev >= 0 && dev < 64 && !attr_set[which - 1][dev]) {
+    const void *fn = which == 1   ? (const void *)k_int4_gemv<1>
+                     : which == 2 ? (const void *)k_int4_gemv<2>
+                     : which == 3 ? (const void *)k_int4_gemm<1>
+                                  : (const void *)k_int4_gemm<2>;
+    const int bytes = (int)(small ? kVSmemDyn : (mt == 1 ? Tile<1>::kSmemDyn : Tile<2>::kSmemDyn));
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
       return LT_ERR_CUDA;
-    attr_set[which][dev] = 1;
+    attr_set[which - 1][dev] = 1;
   }
   cudaStream_t st = (cudaStream_t)stream;
-  if (small)
+  const dim3 grid_tc((unsigned)tiles_n, (unsigned)tiles_m, (unsigned)splits);
+  if (small) {
     if (nb == 1)
       k_int4_gemv<1><<<dim3((unsigned)tiles_n, (unsigned)splits), kVThreads, kVSmemDyn, st>>>(map_x, map_w, map_s,
                                                                                               map_z, ga);
     else
       k_int4_gemv<2><<<dim3((unsigned)tiles_n, (unsigned)splits), kVThreads, kVSmemDyn, st>>>(map_x, map_w, map_s,
                                                                                               map_z, ga);
-  else
-    k_int4_gemm<<<dim3((unsigned)tiles_n, (unsigned)tiles_m, (unsigned)splits), kGemmThreads, kSmemDyn, st>>>(
-        map_x, map_w, ga);
+  } else if (mt == 1) {
+    k_int4_gemm<1><<<grid_tc, kGemmThreads, Tile<1>::kSmemDyn, st>>>(map_x, map_w, ga);
+  } else {
+    k_int4_gemm<2><<<grid_tc, kGemmThreads, Tile<2>::kSmemDyn, st>>>(map_x, map_w, ga);
+  }
   if (splits > 1) {
     // the split sums in order; launched as a programmatic dependent of the
     // product kernel, so its launch overlaps that kernel's tail (it waits for
