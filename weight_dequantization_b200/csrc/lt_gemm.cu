@@ -7,27 +7,30 @@
 //   [K, N] code matrix exactly as lt_dequant_int4 computes it (groups of G
 //   along each row of W), x and out binary16, products summed in fp32.
 //
-// One CTA computes a 128 x 256 tile of out over a range of K (the whole of
-// K, or a split of it whose fp32 partial sums a second kernel adds in a
-// fixed order). Warp roles:
+// Batches of more than 16 rows: one CTA computes MT x 128 rows (MT = 1, or
+// 2 when M > 128) by 256 columns of out over a range of K (the whole of K,
+// or a split of it whose fp32 partial sums a second kernel adds in a fixed
+// order). Warp roles:
 //   warp 0      packed-W producer: for each 64-wide K step one tiled bulk
 //               copy (TMA) of the packed INT4 tile (64 rows x 128 bytes,
-//               128-byte swizzle) into a 6-deep ring, completion counted on
-//               an mbarrier; a slot is refilled as soon as the decoders are
-//               done with it, so this stream runs well ahead of the MMAs;
-//   warp 2      x producer: the x tile (128 x 64 fp16, 128-byte swizzle) of
-//               each step into a 3-deep ring, refilled when the MMAs that
-//               read a slot have completed;
+//               128-byte swizzle) into a 6-deep (MT = 2: 4-deep) ring,
+//               completion counted on an mbarrier; a slot is refilled as soon
+//               as the decoders are done with it, so this stream runs well
+//               ahead of the MMAs;
+//   warp 2      x producer: the x tile (MT x 128 rows x 64 fp16, 128-byte
+//               swizzle) of each step into a 3-deep ring, refilled when the
+//               MMAs that read a slot have completed;
 //   warps 3..18 decoders: turn the packed tile into the fp16 B operand in
 //               shared memory (N-major, 128-byte swizzle), with the exact
 //               half2 arithmetic of lt_dequant_int4 (bit-identical to it), in
-//               a 4-deep ring; scales and zero points are loaded three steps
-//               before their use;
+//               a 4-deep (MT = 2: 3-deep) ring; scales and zero points are
+//               loaded three steps before their use;
 //   warp 1      MMA issuer: one thread issues tcgen05.mma kind::f16 (fp32
-//               accumulator in tensor memory, 128 x 256 = 256 columns), four
-//               K = 16 instructions per step, and tcgen05.commit releases the
-//               ring slots;
-//   warps 3..18 epilogue: tcgen05.ld of the accumulator (warp w reads lanes
+//               accumulators in tensor memory, MT x (128 x 256) = 256 MT
+//               columns), 4 MT K = 16 instructions per step, every B tile
+//               shared by the MT accumulators, and tcgen05.commit releases
+//               the ring slots;
+//   warps 3..18 epilogue: tcgen05.ld of the accumulators (warp w reads lanes
 //               32 (w % 4) ... and a quarter of the columns), conversion to
 //               binary16 (or the fp32 partial of a split), 16-byte stores.
 // Every mbarrier wait is bounded (about a second of clock); a wait that runs
