@@ -603,7 +603,7 @@ def parity_pass(dw, hw):
     """Issue one step's decode calls in order; after each call read its
     output back and compare every element with the oracle's (computed on
     all host cores, independent row / chunk / block ranges). Returns
-    ({unit: verdict}, ok). Dequantized outputs must be within 1 binary16
+    ({unit: outcome}, ok). Dequantized outputs must be within 1 binary16
     ulp of the oracle (0 expected), zero-run output bit for bit."""
     from concurrent.futures import ThreadPoolExecutor
 
@@ -614,7 +614,7 @@ def parity_pass(dw, hw):
 
     s = torch.cuda.current_stream()
     threads = os.cpu_count() or 1
-    verdict, ok = {}, True
+    outcome, ok = {}, True
 
     def host_bits(t):
         return t.cpu().view(torch.int16).numpy().view(np.uint16)
@@ -632,13 +632,13 @@ def parity_pass(dw, hw):
     def record(name, res, total, exact):
         nonlocal ok
         if res is None:
-            verdict[name] = "oracle reported an error"
+            outcome[name] = "oracle reported an error"
             ok = False
             return
         n, bad, worst = res
         good = n == total and worst <= (0 if exact else 1)
         ok = ok and good
-        verdict[name] = (f"bit-exact, {n} of {total} elements" if bad == 0 and n == total else
+        outcome[name] = (f"bit-exact, {n} of {total} elements" if bad == 0 and n == total else
                          f"{bad} of {n} elements differ (max {worst} ulp){'' if good else ': FAILED'}")
 
     with ThreadPoolExecutor(max_workers=threads) as ex:
@@ -683,21 +683,21 @@ def parity_pass(dw, hw):
                     base += m["rows"] * m["cols"]
                 got = host_bits(dw.c5_out[:base])
                 res = run(ex, tasks, got)
-                prev = verdict.get("C5")
+                prev = outcome.get("C5")
                 if res is not None and isinstance(prev, tuple):
                     res = (prev[0] + res[0], prev[1] + res[1], max(prev[2], res[2]))
-                verdict["C5"] = res if res is not None else None
+                outcome["C5"] = res if res is not None else None
                 if li == len(hw["C5"]) - 1 or res is None:
                     total = sum(m["rows"] * m["cols"] for ms in hw["C5"] for m in ms)
-                    record(f"C5 ({len(hw['C5'])} layers)", verdict.pop("C5"), total, False)
+                    record(f"C5 ({len(hw['C5'])} layers)", outcome.pop("C5"), total, False)
                     if res is None:
                         break
     torch.cuda.synchronize()
     st = int(dw.status.item())
     if st != 0:
-        verdict["status"] = f"decoder status {st}"
+        outcome["status"] = f"decoder status {st}"
         ok = False
-    return verdict, ok
+    return outcome, ok
 
 
 def cpu_model() -> str:

@@ -86,11 +86,11 @@ def no_cuda(monkeypatch):
 
 def test_parity_pass_accepts_the_oracles_own_output(no_cuda):
     hw = _hw()
-    verdict, ok = bench.parity_pass(FakeDeviceWorkload(hw), hw)
-    assert ok, verdict
+    outcome, ok = bench.parity_pass(FakeDeviceWorkload(hw), hw)
+    assert ok, outcome
     for u in ("C1", "C2", "C3", "C4", "C4u"):
-        assert verdict[u].startswith("bit-exact"), verdict
-    assert verdict["C5 (2 layers)"].startswith("bit-exact")
+        assert outcome[u].startswith("bit-exact"), outcome
+    assert outcome["C5 (2 layers)"].startswith("bit-exact")
 
 
 @pytest.mark.parametrize("plant,key", [((("C5x", 1), 777, 2), "C5 (2 layers)"), (("C3", 5000, 1), "C3"),
@@ -99,6 +99,6 @@ def test_parity_pass_refuses_a_planted_difference(no_cuda, plant, key):
     hw = _hw()
     if plant[0] == "C3":  # a non-zero element of the activations, so the change is 1 ulp of a literal
         plant = (plant[0], int(np.flatnonzero(hw["C3"]["x"])[0]), 1)
-    verdict, ok = bench.parity_pass(FakeDeviceWorkload(hw, plant), hw)
+    outcome, ok = bench.parity_pass(FakeDeviceWorkload(hw, plant), hw)
     assert not ok
-    assert "FAILED" in verdict[key], verdict
+    assert "FAILED" in outcome[key], outcome
