@@ -239,6 +239,29 @@ def test_fused_corrupt_stream_reports_and_stays_in_bounds():
     assert np.array_equal(got[:131072], want[:131072])
 
 
+@pytest.mark.parametrize("bad", [0, 5, 11])
+def test_fused_one_bad_block_among_many_is_the_only_one_that_differs(bad):
+    # one block of twelve replaced by random bytes of the same length: the
+    # status is the oracle's (one bad block, so no race between errors), and
+    # every other block's output is the oracle's, bit for bit -- the failure
+    # stays inside the bad block's 131,072 elements
+    d = make_matrix(192, 8192, 128, 65536, seed=91)
+    nb = len(d["offsets"]) - 1
+    assert nb == 12
+    comp = d["comp"].copy()
+    s0, s1 = int(d["offsets"][bad]), int(d["offsets"][bad + 1])
+    comp[s0:s1] = np.random.default_rng(bad).integers(0, 256, s1 - s0, dtype=np.uint8)
+    d["comp"] = comp
+    want, st_o = oracle_fused(d)
+    assert st_o != 0
+    got, st_g = run_fused(d)
+    assert st_g == st_o
+    per = 131072  # elements per 64 KB block of INT4 codes
+    keep = np.ones(d["rows"] * d["cols"], bool)
+    keep[bad * per:(bad + 1) * per] = False
+    assert np.array_equal(got[keep], want[keep])
+
+
 def test_fused_batch_matches_per_matrix_oracle():
     # a Llama-shaped layer at 1/64 of the rows, one launch for all matrices
     mats = W.c5_layers(layers=1, scale=1 / 64)[0]
